@@ -1,0 +1,306 @@
+/*
+ * attn_oracle.c -- plain fp64 CPU attention. TEST INFRASTRUCTURE ONLY.
+ *
+ * This is the oracle that the CUDA path is checked against. It is slow and
+ * literal on purpose. For every query row it materialises that row of scores,
+ * applies the mask, takes a two-pass softmax (max, then sum of exponentials),
+ * and forms the probability-weighted sum of value rows. Nothing is tiled,
+ * fused or reordered. Only the tests, the smoke check and the benchmark's CPU
+ * baseline may call it. The library never does, and the two share no code.
+ *
+ * What it computes, and where that is defined:
+ *  - Scores = Q K^T / sqrt(d_k), a row-wise softmax whose rows are
+ *    probabilities summing to 1, and Attention(Q,K,V) = softmax(Scores) V:
+ *    "Self-attention, CUDA kernels and FlashAttention" (russian.itimpress.au),
+ *    section 1, the Scores and Attention(Q,K,V) formulas. The scale is passed
+ *    in explicitly; callers use 1/sqrt(D) unless a workload fixes another.
+ *  - Several heads run the same computation independently: same page,
+ *    section 1, last paragraph.
+ *  - causal=True "for autoregressive models": "Flash Attention" skill page
+ *    (hermes-agent-app.ru), Scenario 2, step 2. Reading taken: key j is
+ *    visible to query i iff j <= i + (Lk - Lq) (bottom-right alignment; the
+ *    same as top-left when Lq == Lk, and a single decode query sees all keys).
+ *  - Fewer K/V heads than query heads (multi-query / grouped-query): same
+ *    page, Scenario 2, step 3. Reading taken: consecutive query heads share a
+ *    K/V head, h_kv = h_q / (H_q / H_kv).
+ *  - Only small normalisation statistics are kept for the backward pass:
+ *    "Self-attention, CUDA kernels and FlashAttention", section 3. Reading
+ *    taken: lse = m + ln(sum_j exp(s_j - m)), natural log, over the scaled,
+ *    masked scores of the row.
+ *  - A row with no visible key has no softmax. Reading taken: O = 0 and
+ *    lse = -inf.
+ *  - Paged KV cache: storage in fixed-size blocks plus a table from logical
+ *    position to physical block, resolved for every position inside the
+ *    attention: "Fast attention kernels and operator fusion" (the-ai.news),
+ *    section "FlashAttention-style attention and paged attention". Layout
+ *    taken: cache[num_blocks][H_kv][block_size][D]; token t of sequence s is
+ *    row t % block_size of physical block block_table[s][t / block_size].
+ *
+ * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math, so
+ * every operation is the IEEE double operation written here).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG (-1)
+#define ORACLE_ERR_INDEX (-2)
+#define ORACLE_ERR_NOMEM (-3)
+
+/*
+ * One query row of attention.
+ *   qi      : the query row, D values
+ *   K, V    : Lk rows of D values each
+ *   n_vis   : keys 0 .. n_vis-1 are visible (the causal mask is a prefix)
+ *   s       : scratch for the Lk scores
+ *   o       : output row, D values
+ *   lse     : output log-sum-exp of the row (may be NULL)
+ *   p_out   : if not NULL, receives the Lk softmax probabilities
+ */
+static void attention_row(const double* qi, const double* K, const double* V,
+                          int64_t Lk, int64_t n_vis, int64_t D, double scale,
+                          double* s, double* o, double* lse, double* p_out) {
+    int64_t j, d;
+    /* Scores: scale * (q_i . k_j); masked keys get -inf. */
+    for (j = 0; j < Lk; ++j) {
+        if (j < n_vis) {
+            double dot = 0.0;
+            for (d = 0; d < D; ++d) dot += qi[d] * K[j * D + d];
+            s[j] = scale * dot;
+        } else {
+            s[j] = -INFINITY;
+        }
+    }
+    /* Pass 1: the row maximum. */
+    double m = -INFINITY;
+    for (j = 0; j < Lk; ++j)
+        if (s[j] > m) m = s[j];
+    for (d = 0; d < D; ++d) o[d] = 0.0;
+    if (m == -INFINITY) { /* no visible key */
+        if (lse) *lse = -INFINITY;
+        if (p_out)
+            for (j = 0; j < Lk; ++j) p_out[j] = 0.0;
+        return;
+    }
+    /* Pass 2: the normaliser l = sum_j exp(s_j - m). */
+    double l = 0.0;
+    for (j = 0; j < Lk; ++j) l += exp(s[j] - m);
+    /* Probabilities P_j = exp(s_j - m) / l and O = sum_j P_j v_j. */
+    for (j = 0; j < Lk; ++j) {
+        double p = exp(s[j] - m) / l;
+        if (p_out) p_out[j] = p;
+        for (d = 0; d < D; ++d) o[d] += p * V[j * D + d];
+    }
+    if (lse) *lse = m + log(l);
+}
+
+/* Number of keys visible to query row i (keys form a prefix). */
+static int64_t visible_keys(int64_t i, int64_t Lq, int64_t Lk, int causal) {
+    if (!causal) return Lk;
+    int64_t last = i + (Lk - Lq); /* highest visible key index */
+    if (last < 0) return 0;
+    if (last >= Lk) return Lk;
+    return last + 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dense attention over [B, H, L, D] tensors.                               */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const double *q, *k, *v;
+    double *out, *lse, *probs;
+    int64_t B, Hq, Hkv, Lq, Lk, D;
+    double scale;
+    int causal;
+    const int64_t* rows; /* NULL: every row, in order */
+    int64_t n_rows;
+    int64_t next; /* shared work counter */
+    int status;
+} dense_job;
+
+static void* dense_worker(void* arg) {
+    dense_job* J = (dense_job*)arg;
+    double* s = (double*)malloc(sizeof(double) * (size_t)(J->Lk > 0 ? J->Lk : 1));
+    if (!s) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    for (;;) {
+        int64_t r = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (r >= J->n_rows) break;
+        /* Flattened row id = (b * Hq + h) * Lq + i. */
+        int64_t id = J->rows ? J->rows[r] : r;
+        int64_t i = id % J->Lq;
+        int64_t bh = id / J->Lq;
+        int64_t h = bh % J->Hq;
+        int64_t b = bh / J->Hq;
+        int64_t hkv = h / group;
+        const double* qi = J->q + id * J->D;
+        const double* K = J->k + (b * J->Hkv + hkv) * J->Lk * J->D;
+        const double* V = J->v + (b * J->Hkv + hkv) * J->Lk * J->D;
+        double* o = J->out + r * J->D;
+        double* lse = J->lse ? J->lse + r : NULL;
+        double* p = J->probs ? J->probs + r * J->Lk : NULL;
+        attention_row(qi, K, V, J->Lk, visible_keys(i, J->Lq, J->Lk, J->causal), J->D,
+                      J->scale, s, o, lse, p);
+    }
+    free(s);
+    return NULL;
+}
+
+static int run_dense(dense_job* J, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (J->n_rows < nthreads) nthreads = (int)(J->n_rows > 0 ? J->n_rows : 1);
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t) {
+        if (pthread_create(&tid[started], NULL, dense_worker, J) == 0) ++started;
+    }
+    dense_worker(J);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return J->status;
+}
+
+static int check_dims(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t D) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || D < 1) return ORACLE_ERR_ARG;
+    if (Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    return ORACLE_OK;
+}
+
+/*
+ * out[B,Hq,Lq,D], lse[B,Hq,Lq] (lse may be NULL) from q[B,Hq,Lq,D],
+ * k[B,Hkv,Lk,D], v[B,Hkv,Lk,D].
+ */
+int oracle_attn_fwd(const double* q, const double* k, const double* v, double* out,
+                    double* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                    int64_t D, double scale, int causal, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+                   NULL, B * Hq * Lq, 0, ORACLE_OK};
+    return run_dense(&J, nthreads);
+}
+
+/*
+ * Selected rows only. rows[r] is a flattened row id (b*Hq + h)*Lq + i;
+ * out[r, D] and lse[r] receive that row's result.
+ */
+int oracle_attn_fwd_rows(const double* q, const double* k, const double* v,
+                         const int64_t* rows, int64_t n_rows, double* out, double* lse,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                         int64_t D, double scale, int causal, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= B * Hq * Lq) return ORACLE_ERR_INDEX;
+    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+                   rows, n_rows, 0, ORACLE_OK};
+    return run_dense(&J, nthreads);
+}
+
+/* The softmax matrix itself: probs[B,Hq,Lq,Lk] (small problems only). */
+int oracle_attn_probs(const double* q, const double* k, const double* v, double* probs,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t D,
+                      double scale, int causal) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    double* out = (double*)malloc(sizeof(double) * (size_t)(B * Hq * Lq * D + 1));
+    if (!out) return ORACLE_ERR_NOMEM;
+    dense_job J = {q, k, v, out, NULL, probs, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+                   NULL, B * Hq * Lq, 0, ORACLE_OK};
+    rc = run_dense(&J, 1);
+    free(out);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Paged decode: one query per sequence, keys resolved through a table.     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const double *q, *kc, *vc;
+    const int32_t *block_table, *seq_lens;
+    double *out, *lse;
+    int64_t block_size, num_seqs, Hq, Hkv, D, max_blocks, num_blocks;
+    double scale;
+    int64_t next;
+    int status;
+} paged_job;
+
+static void* paged_worker(void* arg) {
+    paged_job* J = (paged_job*)arg;
+    const int64_t cap = J->max_blocks * J->block_size;
+    double* Kd = (double*)malloc(sizeof(double) * (size_t)(cap * J->D + 1));
+    double* Vd = (double*)malloc(sizeof(double) * (size_t)(cap * J->D + 1));
+    double* s = (double*)malloc(sizeof(double) * (size_t)(cap + 1));
+    if (!Kd || !Vd || !s) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        free(Kd); free(Vd); free(s);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    for (;;) {
+        int64_t u = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (u >= J->num_seqs * J->Hkv) break;
+        int64_t sq = u / J->Hkv, hkv = u % J->Hkv;
+        int64_t len = J->seq_lens[sq];
+        /* Gather this sequence's keys and values in logical order. */
+        for (int64_t t = 0; t < len; ++t) {
+            int64_t phys = J->block_table[sq * J->max_blocks + t / J->block_size];
+            if (phys < 0 || phys >= J->num_blocks) {
+                __atomic_store_n(&J->status, ORACLE_ERR_INDEX, __ATOMIC_RELAXED);
+                len = 0;
+                break;
+            }
+            const int64_t row = ((phys * J->Hkv + hkv) * J->block_size + t % J->block_size) * J->D;
+            memcpy(Kd + t * J->D, J->kc + row, sizeof(double) * (size_t)J->D);
+            memcpy(Vd + t * J->D, J->vc + row, sizeof(double) * (size_t)J->D);
+        }
+        /* The query heads of this K/V head attend over all len keys. */
+        for (int64_t g = 0; g < group; ++g) {
+            int64_t h = hkv * group + g;
+            const double* qi = J->q + (sq * J->Hq + h) * J->D;
+            attention_row(qi, Kd, Vd, len, len, J->D, J->scale, s,
+                          J->out + (sq * J->Hq + h) * J->D,
+                          J->lse ? J->lse + sq * J->Hq + h : NULL, NULL);
+        }
+    }
+    free(Kd); free(Vd); free(s);
+    return NULL;
+}
+
+/*
+ * q[num_seqs,Hq,D]; k_cache, v_cache [num_blocks,Hkv,block_size,D];
+ * block_table[num_seqs,max_blocks]; seq_lens[num_seqs];
+ * out[num_seqs,Hq,D]; lse[num_seqs,Hq] (may be NULL).
+ */
+int oracle_attn_paged(const double* q, const double* k_cache, const double* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens, int64_t block_size,
+                      double* out, double* lse, int64_t num_seqs, int64_t Hq, int64_t Hkv,
+                      int64_t D, int64_t max_blocks, int64_t num_blocks, double scale,
+                      int nthreads) {
+    if (num_seqs < 0 || Hq < 1 || Hkv < 1 || D < 1 || block_size < 1 || max_blocks < 0 ||
+        num_blocks < 0 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t s = 0; s < num_seqs; ++s)
+        if (seq_lens[s] < 0 || seq_lens[s] > max_blocks * block_size) return ORACLE_ERR_INDEX;
+    paged_job J = {q, k_cache, v_cache, block_table, seq_lens, out, lse, block_size,
+                   num_seqs, Hq, Hkv, D, max_blocks, num_blocks, scale, 0, ORACLE_OK};
+    int64_t units = num_seqs * Hkv;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (units < nthreads) nthreads = (int)(units > 0 ? units : 1);
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&tid[started], NULL, paged_worker, &J) == 0) ++started;
+    paged_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return J.status;
+}

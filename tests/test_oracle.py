@@ -1,0 +1,415 @@
+"""Pins for the oracle: each check ties it to something other than itself.
+
+* A brute force in 60-digit decimal arithmetic (exact products, Decimal.exp/ln, no
+  max subtraction) on tiny random shapes.
+* Closed-form worked examples derived by hand (tests/golden/).
+* Invariants fixed by the definition: probability rows sum to 1, constant V, identical
+  keys, the argmax limit, causal row 0, shift invariance, permutation equivariance,
+  grouped-query heads equal repeated heads, paged equals the gathered dense problem,
+  fully masked rows.
+* Restatements of the algebra the GPU kernels use (a tiled online softmax with lazy
+  rescaling, and a split-KV log-sum-exp combine), checked against the oracle.
+
+Every ``pin_*`` function takes an optional oracle library handle so that
+test_pins_catch_planted_mistakes can run the same pins on deliberately broken builds
+of the oracle and show that each planted mistake fails at least one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+from decimal import Decimal, localcontext
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_examples.json")
+
+
+# --------------------------------------------------------------------------- helpers
+def brute_attention(q, k, v, scale, causal):
+    """Independent brute force: exact decimal products, Decimal exp/ln at 60 digits,
+    no max subtraction. Returns (out, lse) as float64 arrays."""
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, Lq, D))
+    lse = np.zeros((B, Hq, Lq))
+    with localcontext() as ctx:
+        ctx.prec = 60
+        sc = Decimal(float(scale))
+        for b in range(B):
+            for h in range(Hq):
+                hk = h // G
+                for i in range(Lq):
+                    vis = [j for j in range(Lk) if (not causal) or j <= i + Lk - Lq]
+                    if not vis:
+                        lse[b, h, i] = -math.inf
+                        continue
+                    w = []
+                    for j in vis:
+                        dot = sum(Decimal(float(q[b, h, i, d])) * Decimal(float(k[b, hk, j, d]))
+                                  for d in range(D))
+                        w.append((sc * dot).exp())
+                    z = sum(w)
+                    for d in range(D):
+                        num = sum(wj * Decimal(float(v[b, hk, j, d])) for wj, j in zip(w, vis))
+                        out[b, h, i, d] = float(num / z)
+                    lse[b, h, i] = float(z.ln())
+    return out, lse
+
+
+def close(a, b, tol=1e-12):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    fin = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), fin) and np.array_equal(a[~fin], b[~fin])
+    err = np.abs(a[fin] - b[fin]) / np.maximum(1.0, np.abs(b[fin]))
+    assert err.size == 0 or err.max() <= tol, f"max scaled error {err.max():.3e} > {tol}"
+
+
+def rand(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float64) * scale).numpy()
+
+
+def online_softmax_attention(q, K, V, n_vis, scale, tile, thr=0.0):
+    """fp64 restatement of the tiled recurrence the prefill kernel runs for one row:
+    per key tile, a running reference max m (moved only when the tile max exceeds it
+    by more than ``thr``, natural-log units), a running sum l and an accumulator that
+    is rescaled by exp(m_old - m_new) whenever m moves."""
+    Lk, D = K.shape
+    m, l, acc = -math.inf, 0.0, np.zeros(D)
+    for t0 in range(0, Lk, tile):
+        s = scale * (K[t0:t0 + tile] @ q)
+        idx = np.arange(t0, min(t0 + tile, Lk))
+        s = np.where(idx < n_vis, s, -math.inf)
+        mx = s.max()
+        m_new = mx if (m == -math.inf or mx > m + thr) else m
+        if m_new == -math.inf:
+            continue
+        alpha = 0.0 if m == -math.inf else math.exp(m - m_new)
+        p = np.exp(s - m_new)
+        l = alpha * l + p.sum()
+        acc = alpha * acc + p @ V[t0:t0 + tile]
+        m = m_new
+    if l == 0.0:
+        return np.zeros(D), -math.inf
+    return acc / l, m + math.log(l)
+
+
+# ------------------------------------------------------------------------------ pins
+def pin_brute_force(lib=None):
+    cases = [
+        # B, Hq, Hkv, Lq, Lk, D, causal, scale
+        (1, 1, 1, 1, 1, 1, False, 1.0),
+        (1, 2, 1, 3, 5, 4, False, 0.5),
+        (2, 2, 2, 4, 4, 3, True, 0.7),
+        (1, 4, 2, 5, 3, 8, True, 0.35),   # Lq > Lk causal: some rows fully masked
+        (1, 3, 1, 2, 7, 5, True, 1.3),    # Lq < Lk causal: bottom-right alignment
+        (2, 4, 1, 3, 6, 2, False, 0.25),
+    ]
+    for n, (B, Hq, Hkv, Lq, Lk, D, causal, scale) in enumerate(cases):
+        q = rand((B, Hq, Lq, D), 100 + n)
+        k = rand((B, Hkv, Lk, D), 200 + n)
+        v = rand((B, Hkv, Lk, D), 300 + n)
+        o_ref, l_ref = brute_attention(q, k, v, scale, causal)
+        o, l = oracle.attn_fwd(q, k, v, scale, causal, lib=lib)
+        close(o, o_ref)
+        close(l, l_ref)
+
+
+def pin_golden(lib=None):
+    with open(GOLDEN) as f:
+        examples = json.load(f)["examples"]
+    for ex in examples:
+        if ex["kind"] == "dense":
+            o, l = oracle.attn_fwd(np.array(ex["q"]), np.array(ex["k"]), np.array(ex["v"]),
+                                   ex["scale"], ex["causal"], lib=lib)
+        else:
+            o, l = oracle.attn_paged(np.array(ex["q"]), np.array(ex["k_cache"]),
+                                     np.array(ex["v_cache"]),
+                                     torch.tensor(ex["block_table"], dtype=torch.int32),
+                                     torch.tensor(ex["seq_lens"], dtype=torch.int32),
+                                     ex["scale"], lib=lib)
+        close(o, np.array(ex["out"]), 1e-14)
+        close(l, np.array(ex["lse"]), 1e-14)
+
+
+def pin_probability_rows(lib=None):
+    for causal in (False, True):
+        q = rand((1, 2, 6, 4), 1)
+        k = rand((1, 2, 6, 4), 2)
+        P = oracle.attn_probs(q, k, k, 0.6, causal, lib=lib).numpy()
+        assert (P >= 0).all()
+        close(P.sum(-1), np.ones(P.shape[:-1]))
+        if causal:  # masked entries are exactly zero
+            assert np.all(np.triu(P[0, 0], 1) == 0.0) and np.all(np.triu(P[0, 1], 1) == 0.0)
+        # P must be the softmax of the scaled scores (pins P itself, not just O)
+        s = 0.6 * np.einsum("bhid,bhjd->bhij", q, k)
+        if causal:
+            s = np.where(np.triu(np.ones((6, 6), bool), 1), -np.inf, s)
+        e = np.exp(s - s.max(-1, keepdims=True))
+        close(P, e / e.sum(-1, keepdims=True))
+
+
+def pin_constant_values(lib=None):
+    q = rand((2, 3, 5, 4), 3)
+    k = rand((2, 3, 9, 4), 4)
+    c = rand((4,), 5)
+    v = np.broadcast_to(c, (2, 3, 9, 4)).copy()
+    for causal in (False, True):
+        o, _ = oracle.attn_fwd(q, k, v, 0.5, causal, lib=lib)
+        close(o, np.broadcast_to(c, o.shape))
+
+
+def pin_identical_keys(lib=None):
+    q = rand((1, 2, 4, 3), 6)
+    k = np.broadcast_to(rand((3,), 7), (1, 2, 4, 3)).copy()
+    v = rand((1, 2, 4, 3), 8)
+    o, l = oracle.attn_fwd(q, k, v, 0.9, True, lib=lib)
+    s = 0.9 * np.einsum("bhid,bhjd->bhij", q, k)[..., 0]  # every key scores the same
+    for i in range(4):  # causal: row i averages the first i+1 values uniformly
+        close(o[:, :, i], v[:, :, : i + 1].mean(axis=2))
+        close(l[:, :, i], s[:, :, i] + math.log(i + 1))
+
+
+def pin_argmax_limit(lib=None):
+    D, Lk = 4, 6
+    k = rand((1, 1, Lk, D), 9)
+    d = 2
+    k[0, 0, :, d] = np.arange(Lk, dtype=np.float64)  # unique argmax (key 5) with margin 1
+    q = np.zeros((1, 1, 1, D))
+    q[0, 0, 0, d] = 1e4
+    v = rand((1, 1, Lk, D), 10)
+    o, l = oracle.attn_fwd(q, k, v, 0.1, False, lib=lib)  # scale * margin = 1000 nats
+    close(o[0, 0, 0], v[0, 0, Lk - 1], 1e-9)
+    close(l[0, 0, 0], 0.1 * 1e4 * (Lk - 1), 1e-12)
+
+
+def pin_causal_row0(lib=None):
+    q = rand((2, 2, 7, 5), 11)
+    k = rand((2, 2, 7, 5), 12)
+    v = rand((2, 2, 7, 5), 13)
+    o, l = oracle.attn_fwd(q, k, v, 0.4, True, lib=lib)
+    assert np.array_equal(o[:, :, 0].numpy(), v[:, :, 0])
+    close(l[:, :, 0], 0.4 * np.einsum("bhd,bhd->bh", q[:, :, 0], k[:, :, 0]))
+
+
+def pin_shift_invariance(lib=None):
+    # adding u to every key shifts each row's scores by scale*(q.u): P, O unchanged,
+    # lse shifted by the same amount
+    q = rand((1, 2, 5, 4), 14)
+    k = rand((1, 2, 8, 4), 15)
+    v = rand((1, 2, 8, 4), 16)
+    u = rand((4,), 17, 3.0)
+    for causal in (False, True):
+        o1, l1 = oracle.attn_fwd(q, k, v, 0.7, causal, lib=lib)
+        o2, l2 = oracle.attn_fwd(q, k + u, v, 0.7, causal, lib=lib)
+        close(o2, o1, 1e-10)
+        close(l2, l1.numpy() + 0.7 * np.einsum("bhid,d->bhi", q, u), 1e-10)
+
+
+def pin_permutation_equivariance(lib=None):
+    q = rand((1, 1, 3, 4), 18)
+    k = rand((1, 1, 9, 4), 19)
+    v = rand((1, 1, 9, 4), 20)
+    perm = np.random.default_rng(0).permutation(9)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.5, False, lib=lib)
+    o2, l2 = oracle.attn_fwd(q, k[:, :, perm], v[:, :, perm], 0.5, False, lib=lib)
+    close(o2, o1)
+    close(l2, l1)
+
+
+def pin_gqa_equals_repeat(lib=None):
+    B, Hq, Hkv, L, D = 2, 6, 2, 5, 4
+    q = rand((B, Hq, L, D), 21)
+    k = rand((B, Hkv, L, D), 22)
+    v = rand((B, Hkv, L, D), 23)
+    for causal in (False, True):
+        o1, l1 = oracle.attn_fwd(q, k, v, 0.5, causal, lib=lib)
+        kr = np.repeat(k, Hq // Hkv, axis=1)  # consecutive query heads share a K/V head
+        vr = np.repeat(v, Hq // Hkv, axis=1)
+        o2, l2 = oracle.attn_fwd(q, kr, vr, 0.5, causal, lib=lib)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        # and it really is the grouped mapping, not a coincidence of the inputs
+        o3, _ = oracle.attn_fwd(q, np.tile(k, (1, Hq // Hkv, 1, 1)),
+                                np.tile(v, (1, Hq // Hkv, 1, 1)), 0.5, causal, lib=lib)
+        assert not torch.allclose(o1, o3)
+
+
+def pin_paged_equals_dense(lib=None):
+    g = np.random.default_rng(1)
+    S, Hq, Hkv, D, bs, MB = 3, 4, 2, 8, 4, 5
+    NB = S * MB + 2
+    kc = g.standard_normal((NB, Hkv, bs, D))
+    vc = g.standard_normal((NB, Hkv, bs, D))
+    q = g.standard_normal((S, Hq, D))
+    bt = g.permutation(NB)[: S * MB].reshape(S, MB).astype(np.int32)
+    lens = np.array([1, 7, MB * bs], np.int32)
+    o, l = oracle.attn_paged(q, kc, vc, torch.from_numpy(bt), torch.from_numpy(lens), 0.3,
+                             lib=lib)
+    for s in range(S):
+        t = np.arange(lens[s])
+        kd = kc[bt[s, t // bs], :, t % bs]  # [len, Hkv, D]
+        vd = vc[bt[s, t // bs], :, t % bs]
+        od, ld = oracle.attn_fwd(q[s][None, :, None], kd.transpose(1, 0, 2)[None],
+                                 vd.transpose(1, 0, 2)[None], 0.3, False, lib=lib)
+        assert torch.equal(o[s], od[0, :, 0]) and torch.equal(l[s], ld[0, :, 0])
+
+
+def pin_fully_masked_rows(lib=None):
+    q = rand((1, 1, 6, 3), 24)
+    k = rand((1, 1, 2, 3), 25)
+    v = rand((1, 1, 2, 3), 26)
+    o, l = oracle.attn_fwd(q, k, v, 1.0, True, lib=lib)  # rows 0..3 see no key
+    assert np.all(o[0, 0, :4].numpy() == 0.0) and np.all(np.isneginf(l[0, 0, :4].numpy()))
+    assert np.all(np.isfinite(l[0, 0, 4:].numpy()))
+    # empty key set, and empty sequences in paged decode
+    o, l = oracle.attn_fwd(q, k[:, :, :0], v[:, :, :0], 1.0, False, lib=lib)
+    assert np.all(o.numpy() == 0.0) and np.all(np.isneginf(l.numpy()))
+    o, l = oracle.attn_paged(q[0, 0][:1, None, :], np.zeros((1, 1, 16, 3)), np.zeros((1, 1, 16, 3)),
+                             torch.zeros((1, 1), dtype=torch.int32),
+                             torch.zeros((1,), dtype=torch.int32), 1.0, lib=lib)
+    assert np.all(o.numpy() == 0.0) and np.all(np.isneginf(l.numpy()))
+
+
+def pin_online_softmax(lib=None):
+    # the tiled recurrence (any tile size, with or without lazy rescaling) reaches the
+    # two-pass definition; threshold 8*ln2 is the kernel's lazy-rescale margin
+    D, Lq, Lk = 6, 5, 37
+    q = rand((1, 1, Lq, D), 27, 2.0)
+    k = rand((1, 1, Lk, D), 28, 2.0)
+    v = rand((1, 1, Lk, D), 29)
+    for causal in (False, True):
+        o, l = oracle.attn_fwd(q, k, v, 0.8, causal, lib=lib)
+        for tile in (1, 4, 16, 128):
+            for thr in (0.0, 8 * math.log(2)):
+                for i in range(Lq):
+                    n_vis = min(Lk, i + Lk - Lq + 1) if causal else Lk
+                    oi, li = online_softmax_attention(q[0, 0, i], k[0, 0], v[0, 0], n_vis, 0.8,
+                                                      tile, thr)
+                    close(oi, o[0, 0, i])
+                    close(li, l[0, 0, i])
+
+
+def pin_split_combine(lib=None):
+    # partial results over disjoint key chunks, merged with log-sum-exp weights,
+    # equal the result over all keys (the decode kernel's split-KV combine)
+    q = rand((1, 3, 1, 8), 30)
+    k = rand((1, 3, 50, 8), 31)
+    v = rand((1, 3, 50, 8), 32)
+    o, l = oracle.attn_fwd(q, k, v, 0.5, False, lib=lib)
+    for bounds in ([0, 50], [0, 16, 32, 48, 50], [0, 1, 2, 49, 50], [0, 0, 25, 50]):
+        parts = [oracle.attn_fwd(q, k[:, :, a:b], v[:, :, a:b], 0.5, False, lib=lib)
+                 for a, b in zip(bounds[:-1], bounds[1:])]
+        lses = np.stack([p[1].numpy() for p in parts])
+        m = lses.max(0)
+        w = np.exp(lses - m)
+        lse = m + np.log(w.sum(0))
+        out = sum(np.exp(p[1].numpy() - lse)[..., None] * p[0].numpy() for p in parts)
+        close(out, o)
+        close(lse, l)
+
+
+PINS = [pin_brute_force, pin_golden, pin_probability_rows, pin_constant_values,
+        pin_identical_keys, pin_argmax_limit, pin_causal_row0, pin_shift_invariance,
+        pin_permutation_equivariance, pin_gqa_equals_repeat, pin_paged_equals_dense,
+        pin_fully_masked_rows, pin_online_softmax, pin_split_combine]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin()
+
+
+def test_rows_subset_matches_full():
+    q = rand((2, 4, 9, 8), 33)
+    k = rand((2, 2, 11, 8), 34)
+    v = rand((2, 2, 11, 8), 35)
+    o, l = oracle.attn_fwd(q, k, v, 0.5, True)
+    rows = np.array([0, 5, 17, 35, 71, 40], np.int64)
+    orr, lr = oracle.attn_fwd_rows(q, k, v, rows, 0.5, True)
+    assert torch.equal(orr, o.reshape(-1, 8)[rows]) and torch.equal(lr, l.reshape(-1)[rows])
+
+
+def test_threads_do_not_change_results():
+    q = rand((1, 4, 33, 16), 36)
+    k = rand((1, 4, 33, 16), 37)
+    v = rand((1, 4, 33, 16), 38)
+    a = oracle.attn_fwd(q, k, v, 0.25, True, threads=1)
+    b = oracle.attn_fwd(q, k, v, 0.25, True, threads=7)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_oracle_rejects_bad_table():
+    with pytest.raises(ValueError):
+        oracle.attn_paged(np.zeros((1, 1, 4)), np.zeros((2, 1, 4, 4)), np.zeros((2, 1, 4, 4)),
+                          torch.tensor([[0, 5]], dtype=torch.int32),
+                          torch.tensor([6], dtype=torch.int32), 1.0)
+
+
+# Plausible mistakes, each planted in a temporary copy of the oracle source.
+MUTANTS = {
+    "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
+    "causal_off_by_one": ("int64_t last = i + (Lk - Lq);", "int64_t last = i + (Lk - Lq) - 1;"),
+    "causal_top_left": ("int64_t last = i + (Lk - Lq);", "int64_t last = i;"),
+    "gqa_modulo_mapping": ("int64_t hkv = h / group;", "int64_t hkv = h % J->Hkv;"),
+    "keys_used_as_values": ("o[d] += p * V[j * D + d];", "o[d] += p * K[j * D + d];"),
+    "values_used_as_keys": ("dot += qi[d] * K[j * D + d];", "dot += qi[d] * V[j * D + d];"),
+    "max_not_subtracted_in_sum": ("l += exp(s[j] - m);", "l += exp(s[j]);"),
+    "lse_log2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
+    "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "paged_row_index": ("t % J->block_size) * J->D;", "t / J->block_size) * J->D;"),
+    "paged_head_index": ("((phys * J->Hkv + hkv) * J->block_size", "((phys * J->Hkv) * J->block_size"),
+    "paged_len_plus_one": ("int64_t len = J->seq_lens[sq];", "int64_t len = J->seq_lens[sq] + 1;"),
+    "masked_row_nan": ("if (m == -INFINITY) { /* no visible key */",
+                       "if (0) { /* no visible key */"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name):
+    old, new = MUTANTS[name]
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
+    try:
+        c = os.path.join(tmp, "m.c")
+        so = os.path.join(tmp, "m.so")
+        with open(c, "w") as f:
+            f.write(src.replace(old, new))
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+                               "-o", so, c, "-lm"])
+        # A mutant may also overrun a buffer, so it runs in a process of its own; a
+        # crash counts as caught.
+        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+        proc = subprocess.run([sys.executable, "-c", _CHILD, so], cwd=root, capture_output=True,
+                              text=True, timeout=300)
+        caught = proc.stdout.split() if proc.returncode == 0 else [f"crash:{proc.returncode}"]
+        assert caught, f"no pin caught the planted mistake {name}"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+_CHILD = """
+import sys
+import oracle
+from tests import test_oracle as t
+lib = oracle.load(sys.argv[1])
+for pin in t.PINS:
+    try:
+        pin(lib)
+    except (AssertionError, ValueError):
+        print(pin.__name__)
+"""
