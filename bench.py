@@ -1,0 +1,461 @@
+"""Benchmark: exact attention forward (long causal prefill) + paged-KV decode on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  1. attn_fwd on prefill_causal_b1_h16_l8192_d128_bf16 (tcgen05 prefill kernel), and
+  2. attn_fwd_paged on paged_decode_s16_hq12_hkv2_d128_bf16 (paged decode kernel).
+``value`` is the prefill's forward TFLOP/s (4*B*H*Lq*Lk*D, halved for causal) over the
+prefill kernel's device time; the decode's HBM GB/s is reported beside it. Both kernels
+are timed with CUDA events on the stream they run on. Inputs rotate over enough copies
+that every step reads data that is not in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 (launched by torch.distributed.run) every rank runs the same step on its own
+GPU with its own inputs: independent problems, no collective on the data path (weak
+scaling); rank 0 prints the whole-job throughput over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tiled_attention_19_b200 import inputs  # noqa: E402
+
+PREFILL = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
+DECODE = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
+METRIC = "fwd attention TFLOP/s & % of FP16 tensor peak; paged decode HBM GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["tiled_attention_19_b200/csrc/" + f for f in
+                  ("api.cu", "common.cuh", "ptx.cuh", "prefill_sm100.cuh", "paged_decode.cuh")]
+
+
+# ------------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel sources as they are now (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return {}
+    return d.get("kernels", {})
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.index, self.period, self.rows, self.proc = index, period_ms, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return None
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- our GPU arm
+class Workload:
+    """Device copies of the step's inputs (rotated) and its outputs."""
+
+    def __init__(self, device, copies: int):
+        self.device = device
+        xp = inputs.make(PREFILL)
+        xd = inputs.make(DECODE)
+        self.xp_host, self.xd_host = xp, xd
+        self.pf = [{k: v.to(device) for k, v in xp.items()} for _ in range(copies)]
+        self.dc = [{k: v.to(device) for k, v in xd.items()} for _ in range(copies)]
+        self.copies = copies
+        self.p_out = torch.empty_like(self.pf[0]["q"])
+        self.p_lse = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Lq, device=device)
+        self.d_out = torch.empty_like(self.dc[0]["q"])
+        self.d_lse = torch.empty(DECODE.num_seqs, DECODE.Hq, device=device)
+        self.prefill_flops = PREFILL.flops()
+        self.decode_bytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
+
+
+def run_ours(args, ws, rank, local):
+    import tiled_attention_19_b200 as ta
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    ta.load()
+    copies = 4  # 4 x (96 MiB prefill inputs) and 4 x (67 MB decode pool): well past L2
+    w = Workload(device, copies)
+    stream = torch.cuda.current_stream()
+    ws_buf = ta.paged_workspace(DECODE.num_seqs, DECODE.Hq, DECODE.Hkv, DECODE.D,
+                                DECODE.max_blocks, device)
+
+    def step(i, ev=None):
+        p = w.pf[i % copies]
+        d = w.dc[i % copies]
+        if ev is not None:
+            ev[0].record(stream)
+        ta.fwd(p["q"], p["k"], p["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
+               lse=w.p_lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        ta.fwd_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seq_lens"],
+                     scale=DECODE.scale, out=w.d_out, lse=w.d_lse, workspace=ws_buf,
+                     stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    status = ta.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    total_ms = t0.elapsed_time(t1)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    total_ms = reduce_max(total_ms, ws, device)
+    pre_avg = reduce_max(sum(pre_ms) / len(pre_ms), ws, device)
+    dec_avg = reduce_max(sum(dec_ms) / len(dec_ms), ws, device)
+
+    e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)))
+    e2e_pre = reduce_max(e2e["prefill_ms"], ws, device)
+    e2e_dec = reduce_max(e2e["decode_ms"], ws, device)
+
+    if rank != 0:
+        return None
+    peaks, peaks_src = load_peaks()
+    tflops = ws * w.prefill_flops / (pre_avg * 1e-3) / 1e12
+    gbs = ws * w.decode_bytes / (dec_avg * 1e-3) / 1e9
+    per_gpu_tflops = tflops / ws
+    per_gpu_gbs = gbs / ws
+    traffic = profiled_traffic()
+    pk_t = peaks["bf16_tflops_sustained"]
+    pk_h = peaks["hbm_gbs"]
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs shaped like the pages' workloads)",
+        "config": {
+            "workload": f"{PREFILL.name} + {DECODE.name}",
+            "prefill": {"B": PREFILL.B, "H": PREFILL.Hq, "L": PREFILL.Lq, "D": PREFILL.D,
+                        "causal": True, "dtype": "bf16", "flops": w.prefill_flops},
+            "decode": {"seqs": DECODE.num_seqs, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv,
+                       "D": DECODE.D, "block_size": DECODE.block_size,
+                       "tokens": int(w.xd_host["seq_lens"].sum()),
+                       "bytes": w.decode_bytes},
+            "l2": "inputs rotate over 4 device copies (prefill 4 x 96 MiB, decode pool 4 x 67 MB), "
+                  "larger than the 126 MB L2",
+            "parallelism": f"replicas x{ws} (independent problems per GPU)",
+        },
+        "roofline": {
+            "kernel": "prefill_fwd_kernel<128,bf16,causal>",
+            "bound": "tensor",
+            "achieved": round(per_gpu_tflops, 2),
+            "peak": pk_t,
+            "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long loop)",
+            "unit": "TFLOP/s",
+            "frac": round(per_gpu_tflops / pk_t, 4),
+            "frac_of_burst_peak": round(per_gpu_tflops / peaks["bf16_tflops"], 4),
+            "traffic": traffic.get("prefill"),
+            "avg_launch_ms": round(pre_avg, 5),
+        },
+        "paged_decode": {
+            "kernel": "paged_decode_kernel<128,bf16>",
+            "value": round(gbs, 1),
+            "unit": "GB/s",
+            "bound": "hbm",
+            "achieved": round(per_gpu_gbs, 1),
+            "peak": pk_h,
+            "peak_source": f"{peaks_src} hbm_gbs",
+            "frac": round(per_gpu_gbs / pk_h, 4),
+            "traffic": traffic.get("decode"),
+            "avg_launch_ms": round(dec_avg, 5),
+        },
+        "e2e": {
+            "value": round(ws * w.prefill_flops / (e2e_pre * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": e2e["h2d_bytes"],
+            "d2h_bytes_per_step": e2e["d2h_bytes"],
+            "paged_decode_gbs": round(ws * w.decode_bytes / (e2e_dec * 1e-3) / 1e9, 2),
+            "how": "pinned host inputs copied to the device, the C-ABI call, outputs copied back, "
+                   "all on one stream inside the timed region",
+        },
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if args.cpu_baseline and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+def measure_e2e(w, ta, stream, device, steps: int):
+    """Same metric through the public API with host buffers: H2D of the step's inputs
+    from pinned memory, the call, D2H of its outputs, all inside the timed region."""
+    hp = {k: v.pin_memory() for k, v in w.xp_host.items()}
+    hd = {k: v.pin_memory() for k, v in w.xd_host.items()}
+    dp = {k: torch.empty_like(v, device=device) for k, v in hp.items()}
+    dd = {k: torch.empty_like(v, device=device) for k, v in hd.items()}
+    op = torch.empty_like(w.p_out, device="cpu").pin_memory()
+    lp = torch.empty_like(w.p_lse, device="cpu").pin_memory()
+    od = torch.empty_like(w.d_out, device="cpu").pin_memory()
+    ld = torch.empty_like(w.d_lse, device="cpu").pin_memory()
+    wsb = ta.paged_workspace(DECODE.num_seqs, DECODE.Hq, DECODE.Hkv, DECODE.D, DECODE.max_blocks,
+                             device)
+    h2d = sum(v.numel() * v.element_size() for v in list(hp.values()) + list(hd.values()))
+    d2h = sum(t.numel() * t.element_size() for t in (op, lp, od, ld))
+    pre, dec = [], []
+    for it in range(steps + 1):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        for k in dp:
+            dp[k].copy_(hp[k], non_blocking=True)
+        ta.fwd(dp["q"], dp["k"], dp["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
+               lse=w.p_lse, stream=stream)
+        op.copy_(w.p_out, non_blocking=True)
+        lp.copy_(w.p_lse, non_blocking=True)
+        e[1].record(stream)
+        for k in dd:
+            dd[k].copy_(hd[k], non_blocking=True)
+        ta.fwd_paged(dd["q"], dd["k_cache"], dd["v_cache"], dd["block_table"], dd["seq_lens"],
+                     scale=DECODE.scale, out=w.d_out, lse=w.d_lse, workspace=wsb, stream=stream)
+        od.copy_(w.d_out, non_blocking=True)
+        ld.copy_(w.d_lse, non_blocking=True)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        if it > 0:  # the first pass warms up
+            pre.append(e[0].elapsed_time(e[1]))
+            dec.append(e[1].elapsed_time(e[2]))
+    return {"prefill_ms": sum(pre) / len(pre), "decode_ms": sum(dec) / len(dec),
+            "h2d_bytes": h2d, "d2h_bytes": d2h}
+
+
+# ------------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(seconds: float):
+    """Time the fp64 oracle on a bounded sample of the same step: rows of the long
+    prefill spread over heads and positions, and whole decode sequences. Returns the
+    measured TFLOP/s (prefill convention 4*D per visible key per row) and GB/s."""
+    import oracle
+    xp = inputs.make(PREFILL)
+    xd = inputs.make(DECODE)
+    L, D = PREFILL.Lq, PREFILL.D
+    threads = oracle.default_threads()
+
+    def rows_for(n):
+        g = torch.Generator().manual_seed(7)
+        heads = torch.randint(0, PREFILL.Hq, (n,), generator=g)
+        pos = torch.randint(0, L, (n,), generator=g)
+        return (heads * L + pos).tolist(), int((pos + 1).sum())
+
+    # calibrate, then size the sample to about `seconds` of prefill work
+    rows, keys = rows_for(64)
+    t = time.perf_counter()
+    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, True, threads)
+    dt = time.perf_counter() - t
+    n = int(max(64, min(200000, 64 * (0.7 * seconds) / max(dt, 1e-3))))
+    rows, keys = rows_for(n)
+    t = time.perf_counter()
+    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, True, threads)
+    t_pre = time.perf_counter() - t
+    flops = 4.0 * D * keys
+    t = time.perf_counter()
+    oracle.attn_paged(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"], xd["seq_lens"],
+                      DECODE.scale, threads)
+    t_dec = time.perf_counter() - t
+    nbytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
+    return {"tflops": flops / t_pre / 1e12, "gbs": nbytes / t_dec / 1e9, "rows": n,
+            "prefill_s": t_pre, "decode_s": t_dec, "threads": threads}
+
+
+def cpu_baseline(seconds: float):
+    r = oracle_sample(seconds)
+    return {"value": r["tflops"], "unit": "TFLOP/s", "cores": r["threads"], "kind": "oracle",
+            "sample": f"{r['rows']} random query rows of {PREFILL.name} (all their visible keys, "
+                      f"{r['prefill_s']:.1f} s) + the whole {DECODE.name} decode "
+                      f"({r['decode_s']:.2f} s, {r['gbs']:.3f} GB/s)",
+            "paged_decode_gbs": r["gbs"]}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(0.5)
+    res = []
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        res.append(oracle_sample(per_step))
+    total = time.perf_counter() - t
+    tf = statistics.mean(r["tflops"] for r in res)
+    gb = statistics.mean(r["gbs"] for r in res)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": tf,
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) inputs shaped like the pages' workloads)",
+        "config": {"workload": f"{PREFILL.name} + {DECODE.name}",
+                   "note": "the fp64 CPU oracle on a bounded sample of each step"},
+        "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": res[0]["threads"],
+                         "kind": "oracle",
+                         "sample": f"per step {res[0]['rows']} random prefill rows + the whole "
+                                   f"decode workload"},
+        "paged_decode": {"value": gb, "unit": "GB/s"},
+        "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU seconds for the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, ws, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, ws, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

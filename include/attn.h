@@ -1,0 +1,154 @@
+/*
+ * attn.h -- C ABI of libattn_b200: exact tiled attention forward and paged-KV
+ * decode for NVIDIA B200 (sm_100a), one GPU.
+ *
+ * What the library computes
+ *   O = softmax(Q K^T * scale [+ causal mask]) V, exactly (no approximation of
+ *   the softmax), in tiles with an online softmax so the T x T score matrix is
+ *   never written to device memory. Definitions:
+ *   - Scores = Q K^T / sqrt(d_k), row-wise softmax, times V, computed per head:
+ *     "Self-attention, CUDA kernels and FlashAttention" (russian.itimpress.au),
+ *     section 1, the Scores and Attention(Q,K,V) formulas.
+ *   - Tiles of Q, K, V held on chip, a running max and normaliser that rescale
+ *     partial outputs, only O written back, small normalisation statistics
+ *     saved: same page, section 3 (tiling, the online-softmax trick,
+ *     recomputation in the backward pass).
+ *   - causal=True and fewer K/V heads than query heads: "Flash Attention"
+ *     skill page (hermes-agent-app.ru), Scenario 2, steps 2 and 3.
+ *   - Paged KV cache with a block table, block size 16: "Fast attention
+ *     kernels and operator fusion" (the-ai.news), section on FlashAttention-
+ *     style and paged attention.
+ *
+ * Conventions for every call
+ *   - Pointers: device memory owned by the caller (e.g. from cudaMalloc or a
+ *     framework's allocator). The library keeps no pointer after the call
+ *     returns and allocates no device memory per call.
+ *   - Streams: `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream. Calls enqueue work and return; they never synchronise the
+ *     device. Results are valid once the stream reaches that point.
+ *   - Errors: every call returns an attn_status_t and never aborts. Arguments
+ *     are validated before anything is launched; on a non-OK return nothing was
+ *     enqueued. A launch failure returns ATTN_ERR_CUDA. Device-side bounded
+ *     waits and device-side index checks report through
+ *     attn_get_device_status().
+ *   - There is no CPU fallback: without an sm_100 device the compute calls
+ *     return ATTN_ERR_DEVICE.
+ *   - Dtypes: f16 or bf16 in and out (fp32 is not accepted, as on the pages);
+ *     scores, softmax and accumulation run in fp32; lse is fp32.
+ */
+#ifndef TILED_ATTENTION_19_B200_ATTN_H
+#define TILED_ATTENTION_19_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_F16 = 0,
+    ATTN_BF16 = 1
+} attn_dtype_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID = -1,     /* null pointer, negative size, H_q % H_kv != 0,
+                                  scale not finite and > 0, bad table sizes */
+    ATTN_ERR_UNSUPPORTED = -2, /* D not in {64, 128}, dtype, block_size != 16,
+                                  H_q / H_kv > 16 (paged), a size past the limits */
+    ATTN_ERR_MISALIGNED = -3,  /* a tensor base pointer not 16-byte aligned
+                                  (lse, block_table, seq_lens: 4-byte) */
+    ATTN_ERR_DEVICE = -4,      /* no CUDA device, or the current device is not
+                                  compute capability 10.0 (B200) */
+    ATTN_ERR_CUDA = -5,        /* a CUDA call (tensor-map encode, launch) failed */
+    ATTN_ERR_TIMEOUT = -6,     /* from attn_get_device_status: a device-side
+                                  bounded wait expired; the kernel gave up */
+    ATTN_ERR_WORKSPACE = -7,   /* workspace NULL or smaller than required */
+    ATTN_ERR_BAD_INDEX = -8    /* from attn_get_device_status: a block-table entry
+                                  or sequence length out of range was skipped */
+} attn_status_t;
+
+/*
+ * attn_fwd -- dense attention forward (prefill), tcgen05 tensor cores.
+ *
+ *   q    [B, H_q,  Lq, D]  dtype, contiguous, 16-byte aligned
+ *   k    [B, H_kv, Lk, D]  dtype, contiguous, 16-byte aligned
+ *   v    [B, H_kv, Lk, D]  dtype, contiguous, 16-byte aligned
+ *   out  [B, H_q,  Lq, D]  dtype, written (every element)
+ *   lse  [B, H_q,  Lq]     fp32, written if non-NULL: natural-log
+ *        log-sum-exp of the row's scaled, masked scores
+ *
+ *   Query head h reads K/V head h / (H_q / H_kv) (consecutive query heads share
+ *   a K/V head; H_q must be a multiple of H_kv). With causal != 0, key j is
+ *   visible to query i iff j <= i + (Lk - Lq) (bottom-right aligned; top-left
+ *   when Lq == Lk). A row that sees no key gets O = 0 and lse = -inf.
+ *   scale multiplies Q K^T; pass 1/sqrt(D) for the textbook scaling. It must be
+ *   finite and > 0.
+ *
+ *   D in {64, 128}. B, H_q, H_kv >= 1; Lq, Lk >= 0 (Lq == 0 or B == 0 is a
+ *   no-op; Lk == 0 writes O = 0, lse = -inf). Lq, Lk <= 2^22.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                       int causal, attn_dtype_t dtype, void* stream);
+
+/*
+ * attn_paged_workspace_size -- bytes of device workspace attn_fwd_paged needs
+ * for these sizes (0 when no split is ever needed). The workspace holds the
+ * partial results of the split-KV chunks and one completion counter per
+ * (sequence, K/V head).
+ */
+size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D,
+                                 int max_blocks_per_seq, int block_size);
+
+/*
+ * attn_fwd_paged -- decode attention over a paged KV cache (one query token per
+ * sequence), memory-bound, split over KV chunks with an in-kernel combine.
+ *
+ *   q            [num_seqs, H_q, D]                        dtype
+ *   k_cache      [num_blocks, H_kv, block_size, D]         dtype
+ *   v_cache      [num_blocks, H_kv, block_size, D]         dtype
+ *   block_table  [num_seqs, max_blocks_per_seq] int32: token t of sequence s
+ *                is row t % block_size of physical block block_table[s][t / block_size]
+ *   seq_lens     [num_seqs] int32, 0 <= seq_lens[s] <= max_blocks_per_seq * block_size
+ *   out          [num_seqs, H_q, D] dtype, written
+ *   lse          [num_seqs, H_q] fp32, written if non-NULL
+ *
+ *   block_size must be 16; H_q / H_kv <= 16; D in {64, 128}. Entries of
+ *   block_table past ceil(seq_lens[s] / 16) are never read. An entry outside
+ *   [0, num_blocks), or a seq_len past the table, is skipped on the device and
+ *   reported as ATTN_ERR_BAD_INDEX by attn_get_device_status(). A sequence of
+ *   length 0 gets O = 0 and lse = -inf.
+ *
+ *   workspace: device memory of at least attn_paged_workspace_size(...) bytes,
+ *   256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE (its first bytes are
+ *   the completion counters). Every call that completes returns the counters
+ *   to zero, so one workspace serves any number of calls without clearing, as
+ *   long as the calls do not overlap on the device. May be NULL only when the
+ *   size query returns 0.
+ */
+attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_table, const int32_t* seq_lens,
+                             int block_size, void* out, float* lse, int num_seqs, int H_q,
+                             int H_kv, int D, int max_blocks_per_seq, int num_blocks,
+                             float scale, attn_dtype_t dtype, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Static text for a status code (never NULL). */
+const char* attn_error_string(attn_status_t status);
+
+/*
+ * attn_get_device_status -- read and clear the device-side status word that
+ * kernels set when a bounded wait expires (ATTN_ERR_TIMEOUT) or an index is out
+ * of range (ATTN_ERR_BAD_INDEX). Synchronises `stream` to read it. Returns
+ * ATTN_OK if no kernel on the current device reported anything since the last
+ * call, ATTN_ERR_CUDA if the read itself failed.
+ */
+attn_status_t attn_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILED_ATTENTION_19_B200_ATTN_H */

@@ -1,0 +1,51 @@
+"""Shared parity helpers for the GPU tests.
+
+Tolerances (fp32 accumulation, f16/bf16 outputs), compared element by element against
+the fp64 oracle on the same inputs:
+  O:   max |O_gpu - O_ref| <= 2e-3 (f16 outputs), <= 1.6e-2 (bf16 outputs)
+  lse: |lse_gpu - lse_ref| <= 1e-4 * max(1, |lse_ref|); -inf exactly where the oracle has it
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+O_TOL = {torch.float16: 2e-3, torch.bfloat16: 1.6e-2}
+LSE_REL = 1e-4
+SENTINEL = 0x7BCD  # 16-bit pattern written around outputs to catch stray writes
+
+
+def check_parity(out_gpu, lse_gpu, out_ref, lse_ref, dtype, what=""):
+    o = out_gpu.detach().to("cpu", torch.float64)
+    assert o.shape == out_ref.shape, (o.shape, out_ref.shape)
+    assert torch.isfinite(o).all(), f"{what}: non-finite output"
+    err = (o - out_ref).abs()
+    tol = O_TOL[dtype]
+    mx = float(err.max()) if err.numel() else 0.0
+    assert mx <= tol, f"{what}: max |O err| {mx:.3e} > {tol} at {tuple(int(i) for i in torch.nonzero(err == err.max())[0])}"
+    if lse_gpu is not None:
+        lg = lse_gpu.detach().to("cpu", torch.float64)
+        fin = torch.isfinite(lse_ref)
+        assert torch.equal(torch.isfinite(lg), fin), f"{what}: lse finiteness differs"
+        assert torch.all(lg[~fin] == lse_ref[~fin]), f"{what}: lse -inf rows differ"
+        if fin.any():
+            rel = ((lg[fin] - lse_ref[fin]).abs() / lse_ref[fin].abs().clamp_min(1.0)).max()
+            assert float(rel) <= LSE_REL, f"{what}: lse error {float(rel):.3e} > {LSE_REL}"
+    return mx
+
+
+def guarded_empty(shape, dtype, device, guard=4096):
+    """A tensor whose storage sits between two guard bands filled with a sentinel."""
+    n = math.prod(shape)
+    el = torch.tensor([], dtype=dtype).element_size()
+    g = guard // el
+    buf = torch.empty(n + 2 * g, dtype=dtype, device=device)
+    buf.view(torch.int16 if el == 2 else torch.int32).fill_(SENTINEL)
+    return buf, buf[g:g + n].view(shape), g
+
+
+def guards_intact(buf, g):
+    el = buf.element_size()
+    raw = buf.view(torch.int16 if el == 2 else torch.int32)
+    return bool((raw[:g] == SENTINEL).all() and (raw[-g:] == SENTINEL).all())

@@ -1,0 +1,147 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+* The shared library loads and exports every function include/attn.h declares.
+* Status strings exist for every status code.
+* Argument validation returns the documented code before anything is launched. Each
+  case below carries at least one invalid argument, so even on a GPU host no kernel
+  can run on the fake pointers these tests pass.
+* The workspace size query is pure host arithmetic.
+"""
+from __future__ import annotations
+
+import os
+import re
+
+import pytest
+import torch
+
+import tiled_attention_19_b200 as ta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+P = 0x10000  # a 16-byte-aligned fake address (never dereferenced: every call is invalid)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_fwd_paged", "attn_paged_workspace_size", "attn_error_string",
+              "attn_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ta.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+        assert name in ta.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_error_strings():
+    for code in ta.STATUS:
+        s = ta.error_string(code)
+        assert s and s != "unknown status"
+    assert ta.error_string(12345) == "unknown status"
+
+
+def fwd_args(**kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=P, B=1, Hq=2, Hkv=1, Lq=8, Lk=8, D=64, scale=0.125,
+             causal=0, dtype=0, stream=None)
+    a.update(kw)
+    return a
+
+
+FWD_BAD = [
+    ("null_q", dict(q=None), -1),
+    ("null_out", dict(out=None), -1),
+    ("neg_B", dict(B=-1), -1),
+    ("zero_Hq", dict(Hq=0), -1),
+    ("zero_Hkv", dict(Hkv=0), -1),
+    ("neg_Lq", dict(Lq=-3), -1),
+    ("neg_Lk", dict(Lk=-3), -1),
+    ("group_not_divisible", dict(Hq=3, Hkv=2), -1),
+    ("scale_zero", dict(scale=0.0), -1),
+    ("scale_negative", dict(scale=-0.5), -1),
+    ("scale_nan", dict(scale=float("nan")), -1),
+    ("scale_inf", dict(scale=float("inf")), -1),
+    ("D_96", dict(D=96), -2),
+    ("D_256", dict(D=256), -2),
+    ("dtype_fp32", dict(dtype=7), -2),
+    ("Lq_too_long", dict(Lq=(1 << 22) + 1), -2),
+    ("misaligned_q", dict(q=P + 2), -3),
+    ("misaligned_v", dict(v=P + 8), -3),
+    ("misaligned_lse", dict(lse=P + 2), -3),
+]
+
+
+@pytest.mark.parametrize("name,kw,code", FWD_BAD, ids=[c[0] for c in FWD_BAD])
+def test_attn_fwd_validation(name, kw, code):
+    a = fwd_args(**kw)
+    rc = ta.load().attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                            a["Lq"], a["Lk"], a["D"], a["scale"], a["causal"], a["dtype"],
+                            a["stream"])
+    assert rc == code, (rc, ta.STATUS.get(rc))
+
+
+def paged_args(**kw):
+    a = dict(q=P, kc=P, vc=P, bt=P, sl=P, bs=16, out=P, lse=P, S=4, Hq=12, Hkv=2, D=128, MB=256,
+             NB=1024, scale=0.088, dtype=1, ws=P, ws_n=1 << 30, stream=None)
+    a.update(kw)
+    return a
+
+
+PAGED_BAD = [
+    ("null_block_table", dict(bt=None), -1),
+    ("null_seq_lens", dict(sl=None), -1),
+    ("neg_seqs", dict(S=-1), -1),
+    ("group_not_divisible", dict(Hq=12, Hkv=5), -1),
+    ("neg_blocks", dict(NB=-1), -1),
+    ("scale_nan", dict(scale=float("nan")), -1),
+    ("block_size_32", dict(bs=32), -2),
+    ("D_80", dict(D=80), -2),
+    ("group_too_large", dict(Hq=32, Hkv=1), -2),
+    ("misaligned_cache", dict(kc=P + 4), -3),
+    ("misaligned_table", dict(bt=P + 2), -3),
+    ("workspace_missing", dict(ws=None, ws_n=0), -7),
+    ("workspace_small", dict(ws_n=1024), -7),
+    ("workspace_misaligned", dict(ws=P + 16), -3),
+]
+
+
+@pytest.mark.parametrize("name,kw,code", PAGED_BAD, ids=[c[0] for c in PAGED_BAD])
+def test_attn_fwd_paged_validation(name, kw, code):
+    a = paged_args(**kw)
+    rc = ta.load().attn_fwd_paged(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["bs"], a["out"],
+                                  a["lse"], a["S"], a["Hq"], a["Hkv"], a["D"], a["MB"], a["NB"],
+                                  a["scale"], a["dtype"], a["ws"], a["ws_n"], a["stream"])
+    assert rc == code, (rc, ta.STATUS.get(rc))
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
+def test_valid_call_without_gpu_reports_device_error():
+    # Arguments are valid, so validation passes and the device check must refuse: there
+    # is no CPU fallback.
+    a = fwd_args()
+    rc = ta.load().attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                            a["Lq"], a["Lk"], a["D"], a["scale"], a["causal"], a["dtype"], None)
+    assert rc == -4
+    assert ta.load().attn_get_device_status(None) == -4
+
+
+def test_workspace_size():
+    ws = ta.paged_workspace_size
+    assert ws(16, 12, 2, 128, 8) == 0          # one chunk per sequence: no split, no workspace
+    n = ws(16, 12, 2, 128, 256)
+    # counters + per-chunk lse + per-chunk O, each region 256-byte aligned
+    splits = 256 // 8
+    expect = 256 + (16 * 2 * splits * 6 * 4 + 255) // 256 * 256 + 16 * 2 * splits * 6 * 128 * 4
+    assert n == expect
+    assert ws(16, 12, 2, 128, 256, 32) == 0    # unsupported block size -> 0
+    assert ws(0, 12, 2, 128, 256) == 0
+    assert ws(1, 4, 4, 64, 9) > 0

@@ -1,0 +1,108 @@
+"""Parity of attn_fwd_paged (paged-KV decode kernel) with the fp64 oracle, on the GPU.
+
+Calls go through the C ABI (ctypes). The decode workload is compared on every output;
+a sweep covers sequence lengths around the 16-token block and the 128-token chunk
+edges, empty sequences, group sizes 1..16, both head dims and both dtypes. Out-of-range
+block-table entries and sequence lengths must be caught by the kernel's own checks and
+reported through the status word.
+"""
+from __future__ import annotations
+
+import math
+
+import pytest
+import torch
+
+import oracle
+import tiled_attention_19_b200 as ta
+from tiled_attention_19_b200 import inputs
+from tests.parity import check_parity, guarded_empty, guards_intact
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def to_dev(x):
+    return {k: v.to(DEV) for k, v in x.items()}
+
+
+def run_paged(x, scale, guard=False, workspace=None):
+    d = to_dev(x)
+    S, Hq, D = x["q"].shape
+    if guard:
+        ob, out, og = guarded_empty((S, Hq, D), x["q"].dtype, DEV)
+        lb, lse, lg = guarded_empty((S, Hq), torch.float32, DEV)
+        ta.fwd_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seq_lens"],
+                     scale=scale, out=out, lse=lse, workspace=workspace)
+        torch.cuda.synchronize()
+        assert guards_intact(ob, og) and guards_intact(lb, lg)
+    else:
+        out, lse = ta.fwd_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
+                                d["seq_lens"], scale=scale, workspace=workspace)
+        torch.cuda.synchronize()
+    return out.cpu(), lse.cpu()
+
+
+def test_decode_workload_all_outputs():
+    s = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
+    x = inputs.make(s)
+    out, lse = run_paged(x, s.scale, guard=True)
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out, lse, ro, rl, s.dtype, "decode workload")
+
+
+LENS = (0, 1, 15, 16, 17, 127, 128, 129, 255, 256, 257, 1000, 4096)
+CASES = [
+    (12, 2, 128, torch.bfloat16),
+    (8, 8, 64, torch.float16),
+    (16, 1, 128, torch.float16),
+    (4, 2, 64, torch.bfloat16),
+    (3, 3, 128, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"Hq{c[0]}_Hkv{c[1]}_D{c[2]}_{str(c[3]).split('.')[-1]}")
+def test_decode_length_sweep(case):
+    Hq, Hkv, D, dtype = case
+    s = inputs.PagedSpec("t", len(LENS), Hq, Hkv, D, 16, 4096, dtype, 1 / math.sqrt(D),
+                         seed=D + Hq, fixed_lens=LENS)
+    x = inputs.make(s)
+    out, lse = run_paged(x, s.scale, guard=True)
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out, lse, ro, rl, dtype, str(case))
+
+
+def test_workspace_reused_and_left_clean():
+    s = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
+    x = inputs.make(s)
+    n = ta.paged_workspace_size(s.num_seqs, s.Hq, s.Hkv, s.D, s.max_blocks)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
+    o1, l1 = run_paged(x, s.scale, workspace=ws)
+    o2, l2 = run_paged(x, s.scale, workspace=ws)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    # the completion counters (first bytes of the workspace) are back at zero
+    assert torch.all(ws[: 4 * s.num_seqs * s.Hkv] == 0)
+
+
+def test_bad_table_entry_is_reported_not_faulted():
+    s = inputs.PagedSpec("t", 2, 4, 1, 64, 16, 256, torch.float16, 0.125, seed=3,
+                         fixed_lens=(200, 40))
+    x = inputs.make(s)
+    x["block_table"][0, 3] = s.num_blocks + 5   # out of range
+    x["block_table"][1, 1] = -1                 # negative
+    run_paged(x, s.scale)
+    assert ta.device_status() == -8
+    assert ta.device_status() == 0              # reading clears it
+
+
+def test_bad_seq_len_is_reported_not_faulted():
+    s = inputs.PagedSpec("t", 2, 4, 1, 64, 16, 256, torch.float16, 0.125, seed=4,
+                         fixed_lens=(10, 20))
+    x = inputs.make(s)
+    x["seq_lens"][1] = 10 ** 6  # past the table
+    run_paged(x, s.scale)
+    assert ta.device_status() == -8

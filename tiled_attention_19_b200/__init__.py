@@ -1,0 +1,182 @@
+"""Python binding of libattn_b200: exact tiled attention forward and paged-KV decode on
+B200 (sm_100a).
+
+The binding only marshals arguments: tensors become raw device pointers and sizes, the
+stream is torch's current stream, and every step of the computation runs in the CUDA
+kernels behind the C ABI in ``include/attn.h``. There is no CPU fallback: if the
+library is missing or the device is not sm_100, calls raise.
+
+    out, lse = fwd(q, k, v, causal=True)                  # q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D]
+    out, lse = fwd_paged(q, k_cache, v_cache, block_table, seq_lens)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libattn_b200.so")
+
+ATTN_F16, ATTN_BF16 = 0, 1
+STATUS = {
+    0: "ATTN_OK", -1: "ATTN_ERR_INVALID", -2: "ATTN_ERR_UNSUPPORTED", -3: "ATTN_ERR_MISALIGNED",
+    -4: "ATTN_ERR_DEVICE", -5: "ATTN_ERR_CUDA", -6: "ATTN_ERR_TIMEOUT", -7: "ATTN_ERR_WORKSPACE",
+    -8: "ATTN_ERR_BAD_INDEX",
+}
+# Every function include/attn.h declares, with its ctypes signature.
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                            _i, _vp, _sz, _vp]),
+    "attn_error_string": (ctypes.c_char_p, [_i]),
+    "attn_get_device_status": (_i, [_vp]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({error_string(code)})")
+
+
+def load(path: str = LIB_PATH):
+    """The loaded C library. Raises if it has not been built (no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with "
+                                   "`python -m tiled_attention_19_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return load().attn_error_string(int(code)).decode()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float16:
+        return ATTN_F16
+    if dt == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"unsupported dtype {dt}: float16 or bfloat16 only")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise AttnError(rc, what)
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: float | None = None, out: torch.Tensor | None = None,
+        lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """softmax(q k^T * scale [+ causal mask]) v.  q [B,Hq,Lq,D]; k, v [B,Hkv,Lk,D].
+    Returns (out [B,Hq,Lq,D], lse [B,Hq,Lq] fp32 or None). scale defaults to 1/sqrt(D)."""
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k, v must share a dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    rc = load().attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                         _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv, Lq, Lk, D,
+                         float(scale), int(bool(causal)), _dtype_code(q.dtype), _stream(stream))
+    _check(rc, "attn_fwd")
+    return out, lse
+
+
+def paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, D: int, max_blocks_per_seq: int,
+                         block_size: int = 16) -> int:
+    return int(load().attn_paged_workspace_size(num_seqs, Hq, Hkv, D, max_blocks_per_seq,
+                                                block_size))
+
+
+_workspaces: dict = {}
+
+
+def paged_workspace(num_seqs: int, Hq: int, Hkv: int, D: int, max_blocks_per_seq: int,
+                    device, block_size: int = 16) -> torch.Tensor | None:
+    """A zero-filled workspace for these sizes, cached per device. Completed calls leave
+    its counters at zero, so it is reused as is."""
+    n = paged_workspace_size(num_seqs, Hq, Hkv, D, max_blocks_per_seq, block_size)
+    if n == 0:
+        return None
+    device = torch.device(device)
+    key = (device.index, n)
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_table: torch.Tensor, seq_lens: torch.Tensor, scale: float | None = None,
+              out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+              return_lse: bool = True, workspace: torch.Tensor | None = None, stream=None):
+    """Decode attention over a paged cache. q [S,Hq,D]; k_cache, v_cache [NB,Hkv,16,D];
+    block_table [S,MB] int32; seq_lens [S] int32. Returns (out [S,Hq,D], lse [S,Hq])."""
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("cache shape mismatch")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_table and seq_lens must be int32")
+    MB = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = paged_workspace(S, Hq, Hkv, D, MB, q.device, bs)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = load().attn_fwd_paged(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                               _dev(block_table, "block_table"), _dev(seq_lens, "seq_lens"), bs,
+                               _dev(out, "out"), _dev(lse, "lse") if lse is not None else None,
+                               S, Hq, Hkv, D, MB, NB, float(scale), _dtype_code(q.dtype), ws_ptr,
+                               ws_n, _stream(stream))
+    _check(rc, "attn_fwd_paged")
+    return out, lse
+
+
+def device_status(stream=None) -> int:
+    """Read and clear the device-side status word (0 = nothing reported)."""
+    return int(load().attn_get_device_status(_stream(stream)))

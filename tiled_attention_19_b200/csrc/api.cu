@@ -1,0 +1,279 @@
+// api.cu -- the C ABI declared in include/attn.h: argument validation, TMA tensor-map
+// encoding and kernel launches. No per-call allocation, no synchronisation, no CPU
+// fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "paged_decode.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+using attn::PagedArgs;
+using attn::PrefillArgs;
+using attn::PrefillCfg;
+
+constexpr int kMaxSeq = 1 << 22;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ---------------------------------------------------------------- device check
+// The kernels are built for sm_100a only: require compute capability 10.0.
+attn_status_t check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_DEVICE;
+    }
+    static std::mutex mu;
+    static int known[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+    if (dev < 0 || dev >= 64) return ATTN_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (known[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_DEVICE;
+        }
+        known[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return known[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 3-D view (D, L, planes) of a contiguous [planes, L, D] tensor; box 64 x 128 x 1 with
+// 128-byte swizzle. Rows past L read as zero and are never written.
+bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, long long planes) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(planes)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(L) * D * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(attn::kBM), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launchers
+template <int D, bool BF16, bool CAUSAL>
+attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const PrefillArgs& args, int planes, cudaStream_t stream) {
+    auto kern = attn::prefill_fwd_kernel<D, BF16, CAUSAL>;
+    constexpr int smem = PrefillCfg<D>::kSmemBytes;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_tiles));
+    kern<<<grid, attn::kPrefillThreads, smem, stream>>>(tq, tk, tv, args);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+attn_status_t dispatch_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const PrefillArgs& args, int planes,
+                              cudaStream_t stream) {
+    return causal ? launch_prefill<D, BF16, true>(tq, tk, tv, args, planes, stream)
+                  : launch_prefill<D, BF16, false>(tq, tk, tv, args, planes, stream);
+}
+
+template <int D, bool BF16>
+attn_status_t launch_paged(const PagedArgs& a, int num_seqs, cudaStream_t stream) {
+    const dim3 grid(static_cast<unsigned>(a.max_splits), static_cast<unsigned>(a.Hkv),
+                    static_cast<unsigned>(num_seqs));
+    attn::paged_decode_kernel<D, BF16><<<grid, attn::kDecWarps * 32, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,
+                       attn_dtype_t dtype, void* stream_) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID;
+    if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (Lq > kMaxSeq || Lk > kMaxSeq) return ATTN_ERR_UNSUPPORTED;
+    const long long planes_q = static_cast<long long>(B) * H_q;
+    if (planes_q > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    if (B == 0 || Lq == 0) return ATTN_OK;  // nothing to compute
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool bf16 = dtype == ATTN_BF16;
+
+    if (Lk == 0) {  // no keys at all: O = 0, lse = -inf
+        const size_t rows = static_cast<size_t>(planes_q) * Lq;
+        if (bf16)
+            attn::fill_empty_kernel<true><<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(out), lse,
+                                                                    rows * D, rows);
+        else
+            attn::fill_empty_kernel<false><<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(out), lse,
+                                                                     rows * D, rows);
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
+
+    alignas(64) CUtensorMap tq, tk, tv;
+    const long long planes_kv = static_cast<long long>(B) * H_kv;
+    if (!encode_tile_map(&tq, q, bf16, D, Lq, planes_q) ||
+        !encode_tile_map(&tk, k, bf16, D, Lk, planes_kv) ||
+        !encode_tile_map(&tv, v, bf16, D, Lk, planes_kv))
+        return ATTN_ERR_CUDA;
+
+    PrefillArgs args{};
+    args.out = out;
+    args.lse = lse;
+    args.Hq = H_q;
+    args.Hkv = H_kv;
+    args.group = H_q / H_kv;
+    args.Lq = Lq;
+    args.Lk = Lk;
+    args.n_q_tiles = (Lq + attn::kBM - 1) / attn::kBM;
+    args.scale_log2 = scale * attn::kLog2e;
+    if (args.n_q_tiles > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int planes = static_cast<int>(planes_q);
+    const bool c = causal != 0;
+    if (D == 64)
+        return bf16 ? dispatch_causal<64, true>(c, tq, tk, tv, args, planes, stream)
+                    : dispatch_causal<64, false>(c, tq, tk, tv, args, planes, stream);
+    return bf16 ? dispatch_causal<128, true>(c, tq, tk, tv, args, planes, stream)
+                : dispatch_causal<128, false>(c, tq, tk, tv, args, planes, stream);
+}
+
+size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D, int max_blocks_per_seq,
+                                 int block_size) {
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || (D != 64 && D != 128) ||
+        max_blocks_per_seq < 0 || block_size != attn::kPageSize)
+        return 0;
+    return attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq).total;
+}
+
+attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_table, const int32_t* seq_lens, int block_size,
+                             void* out, float* lse, int num_seqs, int H_q, int H_kv, int D,
+                             int max_blocks_per_seq, int num_blocks, float scale,
+                             attn_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                             void* stream_) {
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
+        seq_lens == nullptr || out == nullptr)
+        return ATTN_ERR_INVALID;
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (H_q / H_kv > attn::kMaxGroup) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(max_blocks_per_seq) * attn::kPageSize > kMaxSeq || num_seqs > 65535 ||
+        H_kv > 65535)
+        return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    const attn::PagedLayout L = attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq);
+    if (L.total > 0 && (workspace == nullptr || workspace_bytes < L.total)) return ATTN_ERR_WORKSPACE;
+    if (workspace != nullptr && !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    if (num_seqs == 0) return ATTN_OK;
+
+    PagedArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.kc = static_cast<const uint16_t*>(k_cache);
+    a.vc = static_cast<const uint16_t*>(v_cache);
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.out = static_cast<uint16_t*>(out);
+    a.lse = lse;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.ws_count = L.total ? reinterpret_cast<int*>(ws + L.count_off) : nullptr;
+    a.ws_lse = L.total ? reinterpret_cast<float*>(ws + L.lse_off) : nullptr;
+    a.ws_o = L.total ? reinterpret_cast<float*>(ws + L.o_off) : nullptr;
+    a.Hq = H_q;
+    a.Hkv = H_kv;
+    a.G = H_q / H_kv;
+    a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_splits = L.max_splits;
+    a.scale_log2 = scale * attn::kLog2e;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool bf16 = dtype == ATTN_BF16;
+    if (D == 64)
+        return bf16 ? launch_paged<64, true>(a, num_seqs, stream) : launch_paged<64, false>(a, num_seqs, stream);
+    return bf16 ? launch_paged<128, true>(a, num_seqs, stream) : launch_paged<128, false>(a, num_seqs, stream);
+}
+
+const char* attn_error_string(attn_status_t status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_MISALIGNED: return "misaligned pointer";
+        case ATTN_ERR_DEVICE: return "no supported device (compute capability 10.0 required)";
+        case ATTN_ERR_CUDA: return "CUDA call failed";
+        case ATTN_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case ATTN_ERR_BAD_INDEX: return "block-table entry or sequence length out of range";
+    }
+    return "unknown status";
+}
+
+attn_status_t attn_get_device_status(void* stream_) {
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int host = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&host, attn::g_attn_status, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(attn::g_attn_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return static_cast<attn_status_t>(host);
+}
+
+}  // extern "C"
