@@ -168,8 +168,10 @@ def run_ours(args, ws, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     ta.load()
-    copies = 4  # 4 x (96 MiB prefill inputs) and 4 x (67 MB decode pool): well past L2
+    copies = args.copies  # default 4: 4 x 96 MiB prefill inputs, 4 x 67 MB decode pool > L2
     w = Workload(device, copies)
+    do_pre = args.only in ("both", "prefill")
+    do_dec = args.only in ("both", "decode")
     stream = torch.cuda.current_stream()
     ws_buf = ta.paged_workspace(DECODE.num_seqs, DECODE.Hq, DECODE.Hkv, DECODE.D,
                                 DECODE.max_blocks, device)
@@ -179,13 +181,15 @@ def run_ours(args, ws, rank, local):
         d = w.dc[i % copies]
         if ev is not None:
             ev[0].record(stream)
-        ta.fwd(p["q"], p["k"], p["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
-               lse=w.p_lse, stream=stream)
+        if do_pre:
+            ta.fwd(p["q"], p["k"], p["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
+                   lse=w.p_lse, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        ta.fwd_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seq_lens"],
-                     scale=DECODE.scale, out=w.d_out, lse=w.d_lse, workspace=ws_buf,
-                     stream=stream)
+        if do_dec:
+            ta.fwd_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seq_lens"],
+                         scale=DECODE.scale, out=w.d_out, lse=w.d_lse, workspace=ws_buf,
+                         stream=stream)
         if ev is not None:
             ev[2].record(stream)
 
@@ -218,23 +222,36 @@ def run_ours(args, ws, rank, local):
     pre_avg = reduce_max(sum(pre_ms) / len(pre_ms), ws, device)
     dec_avg = reduce_max(sum(dec_ms) / len(dec_ms), ws, device)
 
-    e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)))
+    if args.e2e:
+        e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)))
+    else:
+        e2e = {"prefill_ms": float("nan"), "decode_ms": float("nan"), "h2d_bytes": 0,
+               "d2h_bytes": 0}
     e2e_pre = reduce_max(e2e["prefill_ms"], ws, device)
     e2e_dec = reduce_max(e2e["decode_ms"], ws, device)
 
     if rank != 0:
         return None
     peaks, peaks_src = load_peaks()
-    tflops = ws * w.prefill_flops / (pre_avg * 1e-3) / 1e12
-    gbs = ws * w.decode_bytes / (dec_avg * 1e-3) / 1e9
-    per_gpu_tflops = tflops / ws
-    per_gpu_gbs = gbs / ws
+
+    def rate(work, ms, scale_):
+        if not (ms == ms) or ms <= 0:  # NaN or nothing timed
+            return None
+        return work / (ms * 1e-3) / scale_
+
+    tflops = rate(ws * w.prefill_flops, pre_avg, 1e12) if do_pre else None
+    gbs = rate(ws * w.decode_bytes, dec_avg, 1e9) if do_dec else None
+    per_gpu_tflops = tflops / ws if tflops is not None else None
+    per_gpu_gbs = gbs / ws if gbs is not None else None
+    r2 = lambda x, n: None if x is None else round(x, n)  # noqa: E731
+    e2e_tf = rate(ws * w.prefill_flops, e2e_pre, 1e12) if do_pre else None
+    e2e_gb = rate(ws * w.decode_bytes, e2e_dec, 1e9) if do_dec else None
     traffic = profiled_traffic()
     pk_t = peaks["bf16_tflops_sustained"]
     pk_h = peaks["hbm_gbs"]
     line = {
         "metric": METRIC,
-        "value": round(tflops, 2),
+        "value": r2(tflops, 2),
         "unit": "TFLOP/s",
         "n_gpus": ws,
         "steps": args.steps,
@@ -260,37 +277,37 @@ def run_ours(args, ws, rank, local):
         "roofline": {
             "kernel": "prefill_fwd_kernel<128,bf16,causal>",
             "bound": "tensor",
-            "achieved": round(per_gpu_tflops, 2),
+            "achieved": r2(per_gpu_tflops, 2),
             "peak": pk_t,
             "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long loop)",
             "unit": "TFLOP/s",
-            "frac": round(per_gpu_tflops / pk_t, 4),
-            "frac_of_burst_peak": round(per_gpu_tflops / peaks["bf16_tflops"], 4),
+            "frac": r2(per_gpu_tflops and per_gpu_tflops / pk_t, 4),
+            "frac_of_burst_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops"], 4),
             "traffic": traffic.get("prefill"),
             "avg_launch_ms": round(pre_avg, 5),
         },
         "paged_decode": {
             "kernel": "paged_decode_kernel<128,bf16>",
-            "value": round(gbs, 1),
+            "value": r2(gbs, 1),
             "unit": "GB/s",
             "bound": "hbm",
-            "achieved": round(per_gpu_gbs, 1),
+            "achieved": r2(per_gpu_gbs, 1),
             "peak": pk_h,
             "peak_source": f"{peaks_src} hbm_gbs",
-            "frac": round(per_gpu_gbs / pk_h, 4),
+            "frac": r2(per_gpu_gbs and per_gpu_gbs / pk_h, 4),
             "traffic": traffic.get("decode"),
             "avg_launch_ms": round(dec_avg, 5),
         },
         "e2e": {
-            "value": round(ws * w.prefill_flops / (e2e_pre * 1e-3) / 1e12, 3),
+            "value": r2(e2e_tf, 3),
             "unit": "TFLOP/s",
             "h2d_bytes_per_step": e2e["h2d_bytes"],
             "d2h_bytes_per_step": e2e["d2h_bytes"],
-            "paged_decode_gbs": round(ws * w.decode_bytes / (e2e_dec * 1e-3) / 1e9, 2),
+            "paged_decode_gbs": r2(e2e_gb, 2),
             "how": "pinned host inputs copied to the device, the C-ABI call, outputs copied back, "
                    "all on one stream inside the timed region",
         },
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (int(do_pre) + int(do_dec)) * args.steps,
         "clocks": clocks.summary(),
     }
     if args.cpu_baseline and ws == 1:
@@ -432,6 +449,12 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU seconds for the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false",
+                    help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",
+                    help="run one kernel of the step only (profiling runs)")
+    ap.add_argument("--copies", type=int, default=4,
+                    help="device copies of the inputs the steps rotate over (4 > L2)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

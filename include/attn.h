@@ -86,8 +86,9 @@ typedef enum {
  *   scale multiplies Q K^T; pass 1/sqrt(D) for the textbook scaling. It must be
  *   finite and > 0.
  *
- *   D in {64, 128}. B, H_q, H_kv >= 1; Lq, Lk >= 0 (Lq == 0 or B == 0 is a
- *   no-op; Lk == 0 writes O = 0, lse = -inf). Lq, Lk <= 2^22.
+ *   D in {64, 128}. H_q, H_kv >= 1; B, Lq, Lk >= 0. B == 0 or Lq == 0 is a
+ *   no-op (every pointer may then be NULL). Lk == 0 writes O = 0, lse = -inf
+ *   (k and v may then be NULL). Lq, Lk <= 2^22.
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                        int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
@@ -119,7 +120,8 @@ size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D,
  *   block_table past ceil(seq_lens[s] / 16) are never read. An entry outside
  *   [0, num_blocks), or a seq_len past the table, is skipped on the device and
  *   reported as ATTN_ERR_BAD_INDEX by attn_get_device_status(). A sequence of
- *   length 0 gets O = 0 and lse = -inf.
+ *   length 0 gets O = 0 and lse = -inf. num_seqs == 0 is a no-op (every
+ *   pointer may then be NULL).
  *
  *   workspace: device memory of at least attn_paged_workspace_size(...) bytes,
  *   256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE (its first bytes are

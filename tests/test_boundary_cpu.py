@@ -60,6 +60,7 @@ def fwd_args(**kw):
 FWD_BAD = [
     ("null_q", dict(q=None), -1),
     ("null_out", dict(out=None), -1),
+    ("null_k_with_keys", dict(k=None), -1),
     ("neg_B", dict(B=-1), -1),
     ("zero_Hq", dict(Hq=0), -1),
     ("zero_Hkv", dict(Hkv=0), -1),
@@ -132,6 +133,16 @@ def test_valid_call_without_gpu_reports_device_error():
                             a["Lq"], a["Lk"], a["D"], a["scale"], a["causal"], a["dtype"], None)
     assert rc == -4
     assert ta.load().attn_get_device_status(None) == -4
+
+
+def test_empty_problems_are_noops_with_null_pointers():
+    lib = ta.load()
+    # B == 0 or Lq == 0: nothing to do, every pointer may be NULL (returns before any
+    # device access, so this is safe on any host)
+    assert lib.attn_fwd(None, None, None, None, None, 0, 2, 1, 8, 8, 64, 0.1, 1, 0, None) == 0
+    assert lib.attn_fwd(None, None, None, None, None, 1, 2, 1, 0, 8, 64, 0.1, 1, 0, None) == 0
+    assert lib.attn_fwd_paged(None, None, None, None, None, 16, None, None, 0, 12, 2, 128, 256,
+                              10, 0.1, 1, None, 0, None) == 0
 
 
 def test_workspace_size():

@@ -124,7 +124,6 @@ extern "C" {
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                        int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,
                        attn_dtype_t dtype, void* stream_) {
-    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID;
     if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
     if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -133,12 +132,15 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     if (Lq > kMaxSeq || Lk > kMaxSeq) return ATTN_ERR_UNSUPPORTED;
     const long long planes_q = static_cast<long long>(B) * H_q;
     if (planes_q > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || Lq == 0) return ATTN_OK;  // nothing to compute; pointers may be NULL
+    // k and v may be NULL (empty tensors) only when there are no keys
+    if (q == nullptr || out == nullptr || (Lk > 0 && (k == nullptr || v == nullptr)))
+        return ATTN_ERR_INVALID;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         (lse != nullptr && !aligned(lse, 4)))
         return ATTN_ERR_MISALIGNED;
     const attn_status_t dev = check_device();
     if (dev != ATTN_OK) return dev;
-    if (B == 0 || Lq == 0) return ATTN_OK;  // nothing to compute
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const bool bf16 = dtype == ATTN_BF16;
 
@@ -194,10 +196,11 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
                              int max_blocks_per_seq, int num_blocks, float scale,
                              attn_dtype_t dtype, void* workspace, size_t workspace_bytes,
                              void* stream_) {
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return ATTN_ERR_INVALID;
+    if (num_seqs == 0) return ATTN_OK;  // nothing to compute; pointers may be NULL
     if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
         seq_lens == nullptr || out == nullptr)
-        return ATTN_ERR_INVALID;
-    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
         return ATTN_ERR_INVALID;
     if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -216,7 +219,6 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
     if (workspace != nullptr && !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
     const attn_status_t dev = check_device();
     if (dev != ATTN_OK) return dev;
-    if (num_seqs == 0) return ATTN_OK;
 
     PagedArgs a{};
     a.q = static_cast<const uint16_t*>(q);
