@@ -343,25 +343,77 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     __syncthreads();
     if (!sm_last) return;
     __threadfence();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int r = idx / D, d = idx % D;
-        const size_t prow0 = unit * a.max_splits * G + r;
+    // Row statistics: one warp per head row reduces the chunks' log2-sum-exp values in
+    // parallel (32 loads in flight per warp, not a serial chain).
+    const size_t lse0 = unit * a.max_splits * G;  // + sp * G + r
+    for (int r = warp; r < G; r += kDecWarps) {
         float M = -INFINITY;
-        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(a.ws_lse + prow0 + sp * G));
-        float W = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-            for (int sp = 0; sp < nsplit; ++sp) {
-                const size_t prow = prow0 + sp * G;
-                const float f = ex2_approx(__ldcg(a.ws_lse + prow) - M);
-                W += f;
-                O += f * __ldcg(a.ws_o + prow * D + d);
+        for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, __ldcg(a.ws_lse + lse0 + sp * G + r));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float W = 0.f;
+        if (M != -INFINITY)
+            for (int sp = lane; sp < nsplit; sp += 32) W += ex2_approx(__ldcg(a.ws_lse + lse0 + sp * G + r) - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+        if (lane == 0) {
+            sm_m[0][r] = M;
+            sm_l[0][r] = W;
+        }
+    }
+    __syncthreads();
+    // Weighted sum of the chunks' normalised outputs, kCombineChunk chunks at a time
+    // with their weights staged in shared memory (reusing the warp-reduction buffer).
+    float* wbuf = &sm_o[0][0][0];
+    constexpr int kCombineChunk = (kDecWarps * kMaxGroup * D) / kMaxGroup;  // chunks per pass
+    float acc[(kMaxGroup * D + kDecWarps * 32 - 1) / (kDecWarps * 32)];
+#pragma unroll
+    for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) acc[e] = 0.f;
+    for (int c0 = 0; c0 < nsplit; c0 += kCombineChunk) {
+        const int cn = min(kCombineChunk, nsplit - c0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < cn * G; i += blockDim.x) {
+            const int sp = c0 + i / G, r = i % G;
+            const float M = sm_m[0][r], W = sm_l[0][r];
+            wbuf[i] = (M == -INFINITY) ? 0.f : ex2_approx(__ldcg(a.ws_lse + lse0 + sp * G + r) - M) / W;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) {
+            const int idx = threadIdx.x + e * blockDim.x;
+            if (idx < G * D) {
+                const int r = idx / D;
+                const float* src = a.ws_o + (lse0 + static_cast<size_t>(c0) * G) * D + idx;
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+                int i = 0;
+                for (; i + 4 <= cn; i += 4) {
+                    const float o0 = __ldcg(src + static_cast<size_t>(i) * G * D);
+                    const float o1 = __ldcg(src + static_cast<size_t>(i + 1) * G * D);
+                    const float o2 = __ldcg(src + static_cast<size_t>(i + 2) * G * D);
+                    const float o3 = __ldcg(src + static_cast<size_t>(i + 3) * G * D);
+                    s0 += wbuf[i * G + r] * o0;
+                    s1 += wbuf[(i + 1) * G + r] * o1;
+                    s2 += wbuf[(i + 2) * G + r] * o2;
+                    s3 += wbuf[(i + 3) * G + r] * o3;
+                }
+                for (; i < cn; ++i) s0 += wbuf[i * G + r] * __ldcg(src + static_cast<size_t>(i) * G * D);
+                acc[e] += (s0 + s1) + (s2 + s3);
             }
         }
-        const float on = W > 0.f ? O / W : 0.f;
-        const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
-        a.out[orow * D + d] = static_cast<uint16_t>(BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(on))
-                                                         : __half_as_ushort(__float2half_rn(on)));
-        if (d == 0 && a.lse != nullptr) a.lse[orow] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
+    }
+#pragma unroll
+    for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) {
+        const int idx = threadIdx.x + e * blockDim.x;
+        if (idx < G * D) {
+            const int r = idx / D, d = idx % D;
+            const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
+            a.out[orow * D + d] = static_cast<uint16_t>(BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[e]))
+                                                             : __half_as_ushort(__float2half_rn(acc[e])));
+            if (d == 0 && a.lse != nullptr) {
+                const float M = sm_m[0][r], W = sm_l[0][r];
+                a.lse[orow] = (M == -INFINITY || !(W > 0.f)) ? -INFINITY : (M + log2f(W)) * kLn2;
+            }
+        }
     }
     if (threadIdx.x == 0) a.ws_count[unit] = 0;  // leave the workspace as found
 }
