@@ -65,8 +65,10 @@ typedef enum {
     ATTN_ERR_TIMEOUT = -6,     /* from attn_get_device_status: a device-side
                                   bounded wait expired; the kernel gave up */
     ATTN_ERR_WORKSPACE = -7,   /* workspace NULL or smaller than required */
-    ATTN_ERR_BAD_INDEX = -8    /* from attn_get_device_status: a block-table entry
+    ATTN_ERR_BAD_INDEX = -8,   /* from attn_get_device_status: a block-table entry
                                   or sequence length out of range was skipped */
+    ATTN_ERR_SCRATCH_LIMIT = -9 /* attn_fwd_paged_noalloc: the problem needs more
+                                  scratch than the fixed 4 MiB buffer holds */
 } attn_status_t;
 
 /*
@@ -136,6 +138,43 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
                              int H_kv, int D, int max_blocks_per_seq, int num_blocks,
                              float scale, attn_dtype_t dtype, void* workspace,
                              size_t workspace_bytes, void* stream);
+
+/*
+ * attn_fwd_paged_noalloc -- attn_fwd_paged without a caller-supplied workspace.
+ * (The pages have no counterpart: this entry point is a property of this
+ * library, not of the attention method.)
+ *
+ * Some callers cannot allocate device memory. A plugin may be handed only its
+ * input and output buffers by a host framework that owns the allocator. A
+ * latency-critical path may not accept cudaMalloc's implicit device
+ * synchronisation. A deployment may have reserved all device memory up front.
+ * This entry point serves them: it allocates nothing and calls no allocating
+ * routine. Its scratch is one fixed array of 4 MiB (4,194,304 bytes) inside the
+ * library's device module, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ * Arguments, layouts, results and errors are those of attn_fwd_paged, without
+ * the workspace. A problem whose attn_paged_workspace_size() exceeds 4 MiB is
+ * rejected with ATTN_ERR_SCRATCH_LIMIT before anything is enqueued. The
+ * decode workload of 16 sequences, 12/2 heads, D = 128, 256 blocks per
+ * sequence needs 3,170,560 bytes.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress); make that first call before any
+ * stream capture. Each call clears the array's completion counters on `stream`
+ * before the kernel.
+ *
+ * Every call on a device shares the one array, which keeps the last call's
+ * contents: calls that overlap on the GPU (different streams, or different
+ * host threads without ordering) race and may produce wrong results. Order
+ * them on one stream, or use attn_fwd_paged with a workspace per stream.
+ */
+attn_status_t attn_fwd_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens,
+                                     int block_size, void* out, float* lse, int num_seqs,
+                                     int H_q, int H_kv, int D, int max_blocks_per_seq,
+                                     int num_blocks, float scale, attn_dtype_t dtype,
+                                     void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* attn_error_string(attn_status_t status);

@@ -25,7 +25,7 @@ ATTN_F16, ATTN_BF16 = 0, 1
 STATUS = {
     0: "ATTN_OK", -1: "ATTN_ERR_INVALID", -2: "ATTN_ERR_UNSUPPORTED", -3: "ATTN_ERR_MISALIGNED",
     -4: "ATTN_ERR_DEVICE", -5: "ATTN_ERR_CUDA", -6: "ATTN_ERR_TIMEOUT", -7: "ATTN_ERR_WORKSPACE",
-    -8: "ATTN_ERR_BAD_INDEX",
+    -8: "ATTN_ERR_BAD_INDEX", -9: "ATTN_ERR_SCRATCH_LIMIT",
 }
 # Every function include/attn.h declares, with its ctypes signature.
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -34,6 +34,8 @@ SIGNATURES = {
     "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                             _i, _vp, _sz, _vp]),
+    "attn_fwd_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i,
+                                    _i, _f, _i, _vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_get_device_status": (_i, [_vp]),
 }

@@ -246,6 +246,88 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
     return bf16 ? launch_paged<128, true>(a, num_seqs, stream) : launch_paged<128, false>(a, num_seqs, stream);
 }
 
+// ----------------------------------------------------------- no-allocation decode
+// Scratch for attn_fwd_paged_noalloc: a fixed 4 MiB array in this library's own device
+// module. Every GPU that loads the library holds it until the process exits. In host
+// code the name g_paged_scratch is only a host-side stand-in for the device array, so
+// it is never passed to a kernel; its device address is looked up once per device.
+}  // extern "C"
+namespace {
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(4) << 20;
+static __device__ __align__(256) uint8_t g_paged_scratch[kStaticScratchBytes];
+
+// Device address of g_paged_scratch on the current device; looked up on the first
+// call made with that device current (nullptr if the lookup fails).
+void* static_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_paged_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+}  // namespace
+extern "C" {
+
+attn_status_t attn_fwd_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens,
+                                     int block_size, void* out, float* lse, int num_seqs,
+                                     int H_q, int H_kv, int D, int max_blocks_per_seq,
+                                     int num_blocks, float scale, attn_dtype_t dtype,
+                                     void* stream_) {
+    // Same argument checks as attn_fwd_paged, done here first so that nothing is
+    // enqueued (not even the counter clear) when the call is rejected.
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return ATTN_ERR_INVALID;
+    if (num_seqs == 0) return ATTN_OK;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
+        seq_lens == nullptr || out == nullptr)
+        return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (H_q / H_kv > attn::kMaxGroup) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(max_blocks_per_seq) * attn::kPageSize > kMaxSeq || num_seqs > 65535 ||
+        H_kv > 65535)
+        return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    const attn::PagedLayout L = attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq);
+    if (L.total > kStaticScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    void* scratch = static_scratch_address();
+    if (scratch == nullptr) return ATTN_ERR_CUDA;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (L.total > 0) {
+        // The completion counters must start at zero; the partial results need not.
+        const size_t counters = static_cast<size_t>(num_seqs) * H_kv * sizeof(int);
+        if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + L.count_off, 0, counters, stream) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+    }
+    return attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, block_size, out, lse,
+                          num_seqs, H_q, H_kv, D, max_blocks_per_seq, num_blocks, scale, dtype,
+                          L.total > 0 ? scratch : nullptr, L.total > 0 ? kStaticScratchBytes : 0,
+                          stream_);
+}
+
 const char* attn_error_string(attn_status_t status) {
     switch (status) {
         case ATTN_OK: return "ok";
@@ -257,6 +339,8 @@ const char* attn_error_string(attn_status_t status) {
         case ATTN_ERR_TIMEOUT: return "device-side bounded wait expired";
         case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
         case ATTN_ERR_BAD_INDEX: return "block-table entry or sequence length out of range";
+        case ATTN_ERR_SCRATCH_LIMIT:
+            return "problem needs more scratch than the library's fixed 4 MiB device buffer";
     }
     return "unknown status";
 }
