@@ -96,7 +96,7 @@ attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
     if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-    const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_tiles));
+    const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_blocks));
     kern<<<grid, attn::kPrefillThreads, smem, stream>>>(tq, tk, tv, args);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -170,9 +170,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     args.group = H_q / H_kv;
     args.Lq = Lq;
     args.Lk = Lk;
-    args.n_q_tiles = (Lq + attn::kBM - 1) / attn::kBM;
+    args.n_q_blocks = (Lq + 2 * attn::kBM - 1) / (2 * attn::kBM);
     args.scale_log2 = scale * attn::kLog2e;
-    if (args.n_q_tiles > 65535) return ATTN_ERR_UNSUPPORTED;
     const int planes = static_cast<int>(planes_q);
     const bool c = causal != 0;
     if (D == 64)

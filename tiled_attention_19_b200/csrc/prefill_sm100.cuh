@@ -6,25 +6,36 @@
 // tracks the running maximum and normaliser and rescales partial outputs, and the
 // saved normalisation statistics). The score matrix lives only in tensor memory.
 //
-// One CTA owns one 128-row query tile of one (batch, head) and walks its 128-key
-// tiles. Roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t, which is TMEM lane t. It loads a
-//              row of S from TMEM, masks, updates the running max (log2 domain,
-//              scale folded into the exponent), forms P = 2^(S*c - m) in f16/bf16
-//              and stores it back into the same TMEM columns, corrects O when the
-//              reference max moved, and finally writes O / l and the lse.
-//   warp 4     producer: one lane issues TMA loads of Q once and of K_j, V_j into a
-//              ring of shared-memory stages (128-byte swizzle).
-//   warp 5     MMA issuer: one lane issues S_j = Q K_j^T (both operands in smem) and
-//              O += P_j V_j (P from TMEM, V from smem); it also owns TMEM allocation.
-// S/P use three 128-column TMEM buffers so S_{j+1} is computed while row j's
-// softmax runs; O uses 128 columns after them (512 columns in total).
+// One CTA owns two 128-row query tiles (Q0, Q1: 256 consecutive rows) of one
+// (batch, head); both walk the same 128-key tiles, so each K/V tile is loaded once
+// for 256 rows. Roles (384 threads, three warpgroups):
+//   warps 0-3  softmax of Q0, warps 4-7 softmax of Q1: thread t of a warpgroup owns
+//              query row t of its tile, which is TMEM lane t. Per key tile it loads its
+//              row of S from TMEM, masks, updates the running max (log2 domain, scale
+//              folded into the exponent), writes P = 2^(S*c - m) in f16/bf16 back over
+//              the same TMEM columns, corrects O when the reference max moved, and at
+//              the end writes O / l and the lse.
+//   warp 8     producer: one lane issues TMA loads of Q0, Q1 once and of K_j, V_j into
+//              two rings of shared-memory stages (128-byte swizzle).
+//   warp 9     MMA issuer: one lane issues, per key tile j,
+//                 PV0_{j-1}: O0 += P0_{j-1} V_{j-1}   (P from TMEM, V from smem)
+//                 S0_j     : S0  = Q0 K_j^T           (both from smem)
+//                 PV1_{j-1}, S1_j likewise,
+//              so each warpgroup's softmax of tile j overlaps the tensor core working
+//              for the other warpgroup. tcgen05 MMAs of one thread execute in issue
+//              order, so S0_j may overwrite the columns P0_{j-1} occupied once PV0_{j-1}
+//              was issued, and the commit that signals S0_j also covers PV0_{j-1}: the
+//              softmax may rescale O0 as soon as S0_j is ready.
+//   warps 10-11 idle.
+// Registers: launched at 168 per thread (384 x 168 = 64,512); the third warpgroup
+// drops to 72 and the two softmax warpgroups rise to 208 (2x128x208 + 128x72 = 62,464).
+// TMEM (512 columns): S0/P0 at 0, S1/P1 at 128, O0 at 256, O1 at 384.
 //
 // Causal masking (the "Flash Attention" skill page, Scenario 2 step 2: causal=True
 // for autoregressive models): key j is visible to query i iff j <= i + (Lk - Lq).
-// Key tiles entirely above the diagonal of the tile's last row are never loaded or
-// multiplied; the mask itself is applied only on tiles that cross the diagonal or
-// the ragged end of the keys.
+// Key tiles entirely above the diagonal of a query tile's last row are skipped for
+// that tile (never loaded if no tile of the CTA needs them); the mask itself is
+// applied only on tiles that cross the diagonal or the ragged end of the keys.
 //
 // Lazy rescaling: the reference max m of a row moves only when a tile's maximum
 // exceeds it by more than 8 (log2 units). Until then p = 2^(s*c - m) <= 2^8, which
@@ -37,10 +48,11 @@
 
 namespace attn {
 
-constexpr int kBM = 128;          // query rows per tile
+constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;          // keys per tile
-constexpr int kSBufs = 3;         // S/P buffers in TMEM
-constexpr int kPrefillThreads = 192;
+constexpr int kPrefillThreads = 384;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 72;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -48,13 +60,15 @@ struct PrefillCfg {
     static constexpr int kChunks = D / 64;             // 64-element (128-byte) column chunks
     static constexpr int kChunkBytes = kBM * 128;      // one chunk of a 128-row tile
     static constexpr int kTileBytes = kBM * D * 2;     // a whole Q, K or V tile
-    static constexpr int kStages = (D == 64) ? 4 : 3;  // K/V ring depth
-    static constexpr int kOCol = kSBufs * kBN;         // first TMEM column of O
+    static constexpr int kKStages = (D == 64) ? 5 : 3;
+    static constexpr int kVStages = (D == 64) ? 5 : 2;
+    static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 384;
     static constexpr int kTmemCols = 512;
-    static constexpr int kNumBars = 1 + 3 * kStages + 3 * kSBufs + 2;
-    static constexpr int kTileRegion = kTileBytes * (1 + 2 * kStages);
+    // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
+    // S_FULL[2], P_FULL[2], O_DONE[2], DRAIN
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 7;
+    static constexpr int kTileRegion = kTileBytes * (2 + kKStages + kVStages);
     static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTileRegion + kNumBars * 8 + 16;
-    static_assert(kOCol + D <= kTmemCols, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
 };
 
@@ -62,9 +76,21 @@ struct PrefillArgs {
     void* out;
     float* lse;
     int Hq, Hkv, group, Lq, Lk;
-    int n_q_tiles;
+    int n_q_blocks;    // ceil(Lq / 256): CTAs along the query axis
     float scale_log2;  // scale * log2(e)
 };
+
+// Number of key tiles query rows [row0, row0 + 128) need (0 if every row is fully masked).
+template <bool CAUSAL>
+__device__ __forceinline__ int key_tiles_for(int row0, int Lq, int Lk) {
+    int n = (Lk + kBN - 1) / kBN;
+    if (CAUSAL) {
+        const int last_row = min(row0 + kBM - 1, Lq - 1);
+        const int max_key = last_row + (Lk - Lq);
+        n = max_key < 0 ? 0 : min(n, max_key / kBN + 1);
+    }
+    return n;
+}
 
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -72,26 +98,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs args) {
     using Cfg = PrefillCfg<D>;
-    constexpr int NS = Cfg::kStages;
-    // barrier slots
+    constexpr int NK = Cfg::kKStages;
+    constexpr int NV = Cfg::kVStages;
     constexpr int Q_FULL = 0;
     constexpr int K_FULL = 1;
-    constexpr int V_FULL = K_FULL + NS;
-    constexpr int KV_EMPTY = V_FULL + NS;
-    constexpr int S_FULL = KV_EMPTY + NS;
-    constexpr int P_FULL = S_FULL + kSBufs;
-    constexpr int PV_BUF = P_FULL + kSBufs;
-    constexpr int PV_DONE = PV_BUF + kSBufs;
-    constexpr int DRAIN = PV_DONE + 1;
+    constexpr int K_EMPTY = K_FULL + NK;
+    constexpr int V_FULL = K_EMPTY + NK;
+    constexpr int V_EMPTY = V_FULL + NV;
+    constexpr int S_FULL = V_EMPTY + NV;  // [2]
+    constexpr int P_FULL = S_FULL + 2;    // [2]
+    constexpr int O_DONE = P_FULL + 2;    // [2]
+    constexpr int DRAIN = O_DONE + 2;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t sQ = s_base;
-    const uint32_t sK0 = s_base + Cfg::kTileBytes;
-    const uint32_t sV0 = sK0 + NS * Cfg::kTileBytes;
+    const uint32_t sQ0 = s_base;
+    const uint32_t sQ1 = s_base + Cfg::kTileBytes;
+    const uint32_t sK0 = s_base + 2 * Cfg::kTileBytes;
+    const uint32_t sV0 = sK0 + NK * Cfg::kTileBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kTileRegion);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -100,43 +127,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;                          // b * Hq + h
-    const int qt = args.n_q_tiles - 1 - blockIdx.y;     // longest causal tiles first
+    const int bh = blockIdx.x;                           // b * Hq + h
+    const int qb = args.n_q_blocks - 1 - blockIdx.y;     // longest causal blocks first
     const int h = bh % args.Hq;
     const int b = bh / args.Hq;
     const int kv_plane = b * args.Hkv + h / args.group;  // grouped-query head mapping
-    const int q0 = qt * kBM;
+    const int q0 = qb * 2 * kBM;
     const int diag = args.Lk - args.Lq;                  // causal: key j visible iff j <= i + diag
-
-    int n_kv = (args.Lk + kBN - 1) / kBN;
-    if (CAUSAL) {
-        const int last_row = min(q0 + kBM - 1, args.Lq - 1);
-        const int max_key = last_row + diag;
-        n_kv = max_key < 0 ? 0 : min(n_kv, max_key / kBN + 1);
-    }
+    const int n0 = key_tiles_for<CAUSAL>(q0, args.Lq, args.Lk);
+    const int n1 = key_tiles_for<CAUSAL>(q0 + kBM, args.Lq, args.Lk);  // n0 <= n1
 
     if (threadIdx.x == 0) {
         mbar_init(bar(Q_FULL), 1);
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NK; ++s) {
             mbar_init(bar(K_FULL + s), 1);
+            mbar_init(bar(K_EMPTY + s), 1);
+        }
+        for (int s = 0; s < NV; ++s) {
             mbar_init(bar(V_FULL + s), 1);
-            mbar_init(bar(KV_EMPTY + s), 1);
+            mbar_init(bar(V_EMPTY + s), 1);
         }
-        for (int s = 0; s < kSBufs; ++s) {
-            mbar_init(bar(S_FULL + s), 1);
-            mbar_init(bar(P_FULL + s), kBM);
-            mbar_init(bar(PV_BUF + s), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(S_FULL + t), 1);
+            mbar_init(bar(P_FULL + t), kBM);
+            mbar_init(bar(O_DONE + t), 1);
         }
-        mbar_init(bar(PV_DONE), 1);
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -146,103 +170,131 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int loads_issued = 0;  // producer: K/V tiles issued (for the abort drain)
+    int k_issued = 0, v_issued = 0;  // producer: tiles issued per ring (for the abort drain)
     bool mma_started = false;
 
-    if (warp == 4) {
+    if (warp >= 10) {
+        regs_decrease<kOtherRegs>();  // idle warps of the third warpgroup
+    } else if (warp == 8) {
         // ------------------------------------------------------------ producer
-        if (lane == 0 && n_kv > 0) {
-            mbar_arrive_expect_tx(bar(Q_FULL), Cfg::kTileBytes);
+        regs_decrease<kOtherRegs>();
+        if (lane == 0 && n1 > 0) {
+            mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
 #pragma unroll
-            for (int c = 0; c < Cfg::kChunks; ++c)
-                tma_load_3d(sQ + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, bh);
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % NS;
-                if (j >= NS && !wait_phase(bar(KV_EMPTY + s), ((j / NS) - 1) & 1, abort_flag))
-                    break;
-                mbar_arrive_expect_tx(bar(K_FULL + s), Cfg::kTileBytes);
-#pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sK0 + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
-                                bar(K_FULL + s), c * 64, j * kBN, kv_plane);
-                mbar_arrive_expect_tx(bar(V_FULL + s), Cfg::kTileBytes);
+            for (int c = 0; c < Cfg::kChunks; ++c) {
+                tma_load_3d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, bh);
+                tma_load_3d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, bh);
+            }
+            for (int j = 0; j < n1; ++j) {
+                const int sk = j % NK, sv = j % NV;
+                if (j >= NK && !wait_phase(bar(K_EMPTY + sk), ((j / NK) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sV0 + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
-                                bar(V_FULL + s), c * 64, j * kBN, kv_plane);
-                loads_issued = j + 1;
+                    tma_load_3d(sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
+                                bar(K_FULL + sk), c * 64, j * kBN, kv_plane);
+                k_issued = j + 1;
+                if (j >= NV && !wait_phase(bar(V_EMPTY + sv), ((j / NV) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(V_FULL + sv), Cfg::kTileBytes);
+#pragma unroll
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                    tma_load_3d(sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
+                                bar(V_FULL + sv), c * 64, j * kBN, kv_plane);
+                v_issued = j + 1;
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0 && n_kv > 0) {
+        regs_decrease<kOtherRegs>();
+        if (lane == 0 && n1 > 0) {
             constexpr uint32_t kIdescQK = idesc_f16(BF16, kBM, kBN, false, false);
             constexpr uint32_t kIdescPV = idesc_f16(BF16, kBM, D, false, true);
             mma_started = true;
-            if (wait_phase(bar(Q_FULL), 0, abort_flag)) {
-                tc_fence_after();
-                for (int j = 0; j <= n_kv; ++j) {
-                    if (j < n_kv) {
-                        const int s = j % NS, sb = j % kSBufs;
-                        if (!wait_phase(bar(K_FULL + s), (j / NS) & 1, abort_flag)) break;
-                        // The S buffer is free once the P·V that read it has completed.
-                        if (j >= kSBufs &&
-                            !wait_phase(bar(PV_BUF + sb), ((j / kSBufs) - 1) & 1, abort_flag))
-                            break;
-                        tc_fence_after();
-                        const uint32_t sK = sK0 + s * Cfg::kTileBytes;
+            // S_t = Q_t K_j^T into TMEM columns s_col (K-major operands: 16 elements =
+            // 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
+            auto issue_s = [&](uint32_t sQ, uint32_t s_col, int j) {
+                const uint32_t sK = sK0 + (j % NK) * Cfg::kTileBytes;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            // K-major operands: 16 elements (32 bytes) per step inside a
-                            // 128-byte swizzle row, then the next 64-column chunk.
-                            const uint32_t koff = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
-                            mma_ss(tmem + sb * kBN, sdesc_sw128(sQ + koff, 16, 1024),
-                                   sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(bar(S_FULL + sb));
-                    }
-                    if (j >= 1) {
-                        const int i = j - 1, s = i % NS, sb = i % kSBufs;
-                        if (!wait_phase(bar(P_FULL + sb), (i / kSBufs) & 1, abort_flag)) break;
-                        if (!wait_phase(bar(V_FULL + s), (i / NS) & 1, abort_flag)) break;
-                        tc_fence_after();
-                        const uint32_t sV = sV0 + s * Cfg::kTileBytes;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
+                    mma_ss(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
+                           sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_t += P_t V_j: P from TMEM (16 keys = 8 columns per step), V MN-major
+            // (16 keys = two 8-row swizzle atoms, 2048 bytes; D chunks 16 KiB apart).
+            auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int j) {
+                const uint32_t sV = sV0 + (j % NV) * Cfg::kTileBytes;
 #pragma unroll
-                        for (int ks = 0; ks < kBN / 16; ++ks) {
-                            // V is MN-major: 16 keys = two 8-row swizzle atoms (2048 bytes);
-                            // the 64-column chunks of D sit 16 KiB apart (leading offset).
-                            mma_ts(tmem + Cfg::kOCol, tmem + sb * kBN + ks * 8,
-                                   sdesc_sw128(sV + ks * 2048, Cfg::kChunkBytes, 1024), kIdescPV,
-                                   (i > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        mma_commit(bar(PV_DONE));
-                        mma_commit(bar(PV_BUF + sb));
-                        mma_commit(bar(KV_EMPTY + s));
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    mma_ts(tmem + o_col, tmem + p_col + ks * 8,
+                           sdesc_sw128(sV + ks * 2048, Cfg::kChunkBytes, 1024), kIdescPV,
+                           (j > 0 || ks > 0) ? 1u : 0u);
+            };
+            bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
+            for (int j = 0; ok && j <= n1; ++j) {
+                const int i = j - 1;  // the tile whose P·V is due
+                // PV0_{j-1}
+                if (i >= 0 && i < n0) {
+                    ok = wait_phase(bar(P_FULL + 0), i & 1, abort_flag) &&
+                         wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(Cfg::kSCol0, Cfg::kOCol0, i);
+                    if (i == n0 - 1) mma_commit(bar(O_DONE + 0));
+                }
+                if (j < n1) {
+                    ok = wait_phase(bar(K_FULL + j % NK), (j / NK) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (j < n0) {
+                        issue_s(sQ0, Cfg::kSCol0, j);
+                        mma_commit(bar(S_FULL + 0));
                     }
+                }
+                // PV1_{j-1}
+                if (i >= 0) {
+                    ok = wait_phase(bar(P_FULL + 1), i & 1, abort_flag) &&
+                         wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(Cfg::kSCol1, Cfg::kOCol1, i);
+                    mma_commit(bar(V_EMPTY + i % NV));
+                    if (i == n1 - 1) mma_commit(bar(O_DONE + 1));
+                }
+                if (j < n1) {
+                    issue_s(sQ1, Cfg::kSCol1, j);
+                    mma_commit(bar(S_FULL + 1));
+                    mma_commit(bar(K_EMPTY + j % NK));
                 }
             }
         }
     } else {
         // ------------------------------------------------------------- softmax
-        const int t = threadIdx.x;  // 0..127: query row within the tile == TMEM lane
-        const int row = q0 + t;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        regs_increase<kSoftmaxRegs>();
+        const int tile = warp >> 2;          // 0: Q0 (warps 0-3), 1: Q1 (warps 4-7)
+        const int t = threadIdx.x & 127;     // query row within the tile == TMEM lane
+        const int row = q0 + tile * kBM + t;
+        const int n_kv = tile == 0 ? n0 : n1;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t s_col = tile == 0 ? Cfg::kSCol0 : Cfg::kSCol1;
+        const uint32_t o_col = tile == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
         const float c = args.scale_log2;
         const int row_limit = CAUSAL ? min(args.Lk, row + diag + 1) : args.Lk;
+        const int tile_row0 = q0 + tile * kBM;
         float m_ref = -INFINITY;  // reference max, log2 units
         float l = 0.f;            // running sum of 2^(s*c - m_ref)
         bool ok = true;
 
         for (int j = 0; j < n_kv; ++j) {
-            const int sb = j % kSBufs;
-            const bool w = wait_phase(bar(S_FULL + sb), (j / kSBufs) & 1, abort_flag);
+            const bool w = wait_phase(bar(S_FULL + tile), j & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[kBN];
-            tmem_ld32(lane_base + sb * kBN + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(lane_base + sb * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld32(lane_base + sb * kBN + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-            tmem_ld32(lane_base + sb * kBN + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+            tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+            tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
             tmem_wait_ld();
             float s[kBN];
 #pragma unroll
@@ -250,7 +302,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
             const int kbase = j * kBN;
             const bool need_mask =
-                (kbase + kBN > args.Lk) || (CAUSAL && kbase + kBN - 1 > q0 + diag);
+                (kbase + kBN > args.Lk) || (CAUSAL && kbase + kBN - 1 > tile_row0 + diag);
             if (need_mask) {
                 const int lim = row_limit - kbase;
 #pragma unroll
@@ -280,33 +332,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 pk[x / 2] = pack2<BF16>(p0, p1);
             }
 
-            // Correct O when the reference max moved; the previous P·V must be done.
+            // P overwrites the first 64 columns of this tile's S buffer (16-bit pairs).
+            tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            // Correct O when the reference max moved. S_t(j) completing implies the
+            // P·V of tile j-1 (issued before it) has completed too.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                const bool w2 = wait_phase(bar(PV_DONE), (j - 1) & 1, abort_flag);
-                if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-                tc_fence_after();
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 32) {
                     uint32_t o[32];
-                    tmem_ld32(lane_base + Cfg::kOCol + d0, o);
+                    tmem_ld32(lane_base + o_col + d0, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-                    tmem_st32(lane_base + Cfg::kOCol + d0, o);
+                    tmem_st32(lane_base + o_col + d0, o);
                 }
             }
-            // P overwrites the first 64 columns of this S buffer (16-bit pairs).
-            tmem_st32(lane_base + sb * kBN + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_FULL + sb));
+            mbar_arrive(bar(P_FULL + tile));
             l = l * alpha + (rs0 + rs1);
             m_ref = m_new;
         }
 
         if (ok && n_kv > 0) {
-            const bool w = wait_phase(bar(PV_DONE), (n_kv - 1) & 1, abort_flag);
+            const bool w = wait_phase(bar(O_DONE + tile), 0, abort_flag);
             ok = __all_sync(0xffffffffu, w);
             if (ok) tc_fence_after();
         }
@@ -314,14 +364,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // ------------------------------------------------------------ epilogue
             const bool has = l > 0.f;
             const float inv_l = has ? 1.f / l : 0.f;
-            using T = uint16_t;
-            T* out_row = reinterpret_cast<T*>(args.out) +
-                         (static_cast<size_t>(bh) * args.Lq + row) * D;
+            uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) +
+                                (static_cast<size_t>(bh) * args.Lq + row) * D;
 #pragma unroll
             for (int d0 = 0; d0 < D; d0 += 32) {
                 uint32_t o[32];
                 if (n_kv > 0) {
-                    tmem_ld32(lane_base + Cfg::kOCol + d0, o);
+                    tmem_ld32(lane_base + o_col + d0, o);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
@@ -351,20 +400,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (*abort_flag) {
         // Nothing may still be writing into this CTA's shared or tensor memory when
         // it exits: wait for the loads already issued and for every MMA issued.
-        if (warp == 4 && lane == 0 && n_kv > 0) {
+        if (warp == 8 && lane == 0 && n1 > 0) {
             drain_phase(bar(Q_FULL), 0);
-            for (int j = max(0, loads_issued - NS); j < loads_issued; ++j) {
-                drain_phase(bar(K_FULL + j % NS), (j / NS) & 1);
-                drain_phase(bar(V_FULL + j % NS), (j / NS) & 1);
-            }
+            for (int j = max(0, k_issued - NK); j < k_issued; ++j)
+                drain_phase(bar(K_FULL + j % NK), (j / NK) & 1);
+            for (int j = max(0, v_issued - NV); j < v_issued; ++j)
+                drain_phase(bar(V_FULL + j % NV), (j / NV) & 1);
         }
-        if (warp == 5 && lane == 0 && mma_started) {
+        if (warp == 9 && lane == 0 && mma_started) {
             mma_commit(bar(DRAIN));
             drain_phase(bar(DRAIN), 0);
         }
         __syncthreads();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }

@@ -173,6 +173,16 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Register reallocation between warpgroups (all warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // --------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
