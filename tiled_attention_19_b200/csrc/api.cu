@@ -91,11 +91,27 @@ attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const
     auto kern = attn::prefill_fwd_kernel<D, BF16, CAUSAL>;
     constexpr int smem = PrefillCfg<D>::kSmemBytes;
     static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
+    static attn_status_t setup = ATTN_OK;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+            setup = ATTN_ERR_CUDA;
+            return;
+        }
+        // The kernel moves registers between warpgroups with setmaxnreg; refuse to
+        // launch unless the registers it is launched with cover the split.
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+            setup = ATTN_ERR_CUDA;
+            return;
+        }
+        if (static_cast<long long>(fa.numRegs) * attn::kPrefillThreads < attn::kRegBudget)
+            setup = ATTN_ERR_UNSUPPORTED;
     });
-    if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+    if (setup != ATTN_OK) {
+        cudaGetLastError();
+        return setup;
+    }
     const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_blocks));
     kern<<<grid, attn::kPrefillThreads, smem, stream>>>(tq, tk, tv, args);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -27,8 +27,9 @@
 //              was issued, and the commit that signals S0_j also covers PV0_{j-1}: the
 //              softmax may rescale O0 as soon as S0_j is ready.
 //   warps 10-11 idle.
-// Registers: launched at 168 per thread (384 x 168 = 64,512); the third warpgroup
-// drops to 72 and the two softmax warpgroups rise to 208 (2x128x208 + 128x72 = 62,464).
+// Registers: the third warpgroup releases registers (setmaxnreg.dec to 80) and the two
+// softmax warpgroups take them (setmaxnreg.inc to 200): 2x128x200 + 128x80 = 61,440 of
+// the 384 x 168 = 64,512 the CTA is launched with.
 // TMEM (512 columns): S0/P0 at 0, S1/P1 at 128, O0 at 256, O1 at 384.
 //
 // Causal masking (the "Flash Attention" skill page, Scenario 2 step 2: causal=True
@@ -51,8 +52,13 @@ namespace attn {
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;          // keys per tile
 constexpr int kPrefillThreads = 384;
-constexpr int kSoftmaxRegs = 208;
-constexpr int kOtherRegs = 72;
+// Register split between warpgroups (setmaxnreg). It only works if the registers the
+// CTA was launched with cover it; the launcher checks 384 x (registers per thread at
+// launch) >= kRegBudget before the first launch and refuses otherwise, because a
+// setmaxnreg.inc that cannot be satisfied waits forever.
+constexpr int kSoftmaxRegs = 200;
+constexpr int kOtherRegs = 80;
+constexpr int kRegBudget = 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs;  // 61,440
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
