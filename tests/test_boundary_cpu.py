@@ -147,12 +147,14 @@ def test_empty_problems_are_noops_with_null_pointers():
 
 def test_workspace_size():
     ws = ta.paged_workspace_size
-    assert ws(16, 12, 2, 128, 8) == 0          # one chunk per sequence: no split, no workspace
-    n = ws(16, 12, 2, 128, 256)
-    # counters + per-chunk lse + per-chunk O, each region 256-byte aligned
-    splits = 256 // 8
-    expect = 256 + (16 * 2 * splits * 6 * 4 + 255) // 256 * 256 + 16 * 2 * splits * 6 * 128 * 4
-    assert n == expect
+    assert ws(16, 12, 2, 128, 1) == 0          # one block per sequence: never split, no workspace
+    # 32 units -> 296 CTAs (chunks); counters + per-chunk lse + per-chunk O, each 256-B aligned
+    grid, G = 296, 6
+    expect = 256 + (grid * G * 4 + 255) // 256 * 256 + (grid * G * 128 * 4 + 255) // 256 * 256
+    assert ws(16, 12, 2, 128, 256) == expect
+    # more units than half the default grid: two chunks per unit on average
+    assert ws(320, 32, 2, 128, 256) > ws(16, 32, 2, 128, 256)
     assert ws(16, 12, 2, 128, 256, 32) == 0    # unsupported block size -> 0
     assert ws(0, 12, 2, 128, 256) == 0
     assert ws(1, 4, 4, 64, 9) > 0
+    assert ws(1024, 8, 2, 128, 256) == 0       # > 1024 units: one CTA per unit, no split

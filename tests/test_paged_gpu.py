@@ -106,3 +106,30 @@ def test_bad_seq_len_is_reported_not_faulted():
     x["seq_lens"][1] = 10 ** 6  # past the table
     run_paged(x, s.scale)
     assert ta.device_status() == -8
+
+
+def test_decode_skewed_lengths_balanced_schedule():
+    # one long sequence among many short and empty ones: the long one is cut into many
+    # chunks merged through the workspace, the short ones finish in one chunk
+    lens = (4096,) + (0, 1, 3, 16, 17) * 6 + (31,)
+    s = inputs.PagedSpec("t", len(lens), 8, 2, 128, 16, 4096, torch.bfloat16, 1 / math.sqrt(128),
+                         seed=31, fixed_lens=lens)
+    x = inputs.make(s)
+    out, lse = run_paged(x, s.scale, guard=True)
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out, lse, ro, rl, s.dtype, "skewed")
+
+
+def test_decode_many_units_one_cta_each():
+    # more than 1024 (sequence, K/V head) units: each CTA takes a whole unit, no split
+    s = inputs.PagedSpec("t", 520, 4, 2, 64, 16, 160, torch.float16, 0.125, seed=32, min_len=0)
+    assert s.num_seqs * s.Hkv > 1024
+    assert ta.paged_workspace_size(s.num_seqs, s.Hq, s.Hkv, s.D, s.max_blocks) == 0
+    x = inputs.make(s)
+    out, lse = run_paged(x, s.scale, guard=True)
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out, lse, ro, rl, s.dtype, "many units")

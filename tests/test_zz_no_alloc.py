@@ -65,9 +65,9 @@ def test_noalloc_matches_workspace_entry_point(name):
 
 
 def test_noalloc_refuses_problems_past_the_scratch_limit():
-    # 64 sequences of up to 4096 tokens need about 12.7 MB of scratch: refused before
-    # anything is enqueued (no kernel runs, so the pointers are never touched).
-    s = inputs.PagedSpec("big", 64, 12, 2, 128, 16, 4096, torch.bfloat16, 0.088, seed=22)
+    # 160 sequences with 32 query heads over 2 K/V heads need about 5.3 MB of scratch:
+    # refused before anything is enqueued (no kernel runs, so the pointers are never read).
+    s = inputs.PagedSpec("big", 160, 32, 2, 128, 16, 4096, torch.bfloat16, 0.088, seed=22)
     assert ta.paged_workspace_size(s.num_seqs, s.Hq, s.Hkv, s.D, s.max_blocks) > SCRATCH_LIMIT
     q = torch.empty(s.num_seqs, s.Hq, s.D, dtype=s.dtype, device=DEV)
     cache = torch.empty(16, s.Hkv, 16, s.D, dtype=s.dtype, device=DEV)

@@ -125,11 +125,33 @@ attn_status_t dispatch_causal(bool causal, const CUtensorMap& tq, const CUtensor
                   : launch_prefill<D, BF16, false>(tq, tk, tv, args, planes, stream);
 }
 
+// 2-D view (D, rows) of a paged cache [num_blocks, H_kv, 16, D]: one row per token of
+// each (block, head); box 64 x 16 (one block's rows, 64 columns) with 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* tm, const void* base, bool bf16, int D, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(attn::kPageSize)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, bool BF16>
-attn_status_t launch_paged(const PagedArgs& a, int num_seqs, cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>(a.max_splits), static_cast<unsigned>(a.Hkv),
-                    static_cast<unsigned>(num_seqs));
-    attn::paged_decode_kernel<D, BF16><<<grid, attn::kDecWarps * 32, 0, stream>>>(a);
+attn_status_t launch_paged(const CUtensorMap& tk, const CUtensorMap& tv, const PagedArgs& a,
+                           int grid, cudaStream_t stream) {
+    auto kern = attn::paged_decode_kernel<D, BF16>;
+    constexpr int smem = attn::DecodeCfg<D>::kSmemBytes;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+    kern<<<static_cast<unsigned>(grid), attn::kDecThreads, smem, stream>>>(tk, tv, a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -235,10 +257,16 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
     const attn_status_t dev = check_device();
     if (dev != ATTN_OK) return dev;
 
+    const long long rows = static_cast<long long>(num_blocks) * H_kv * attn::kPageSize;
+    if (rows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const bool bf16 = dtype == ATTN_BF16;
+    alignas(64) CUtensorMap tk, tv;
+    if (!encode_cache_map(&tk, k_cache, bf16, D, rows > 0 ? rows : 1) ||
+        !encode_cache_map(&tv, v_cache, bf16, D, rows > 0 ? rows : 1))
+        return ATTN_ERR_CUDA;
+
     PagedArgs a{};
     a.q = static_cast<const uint16_t*>(q);
-    a.kc = static_cast<const uint16_t*>(k_cache);
-    a.vc = static_cast<const uint16_t*>(v_cache);
     a.block_table = block_table;
     a.seq_lens = seq_lens;
     a.out = static_cast<uint16_t*>(out);
@@ -247,18 +275,20 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
     a.ws_count = L.total ? reinterpret_cast<int*>(ws + L.count_off) : nullptr;
     a.ws_lse = L.total ? reinterpret_cast<float*>(ws + L.lse_off) : nullptr;
     a.ws_o = L.total ? reinterpret_cast<float*>(ws + L.o_off) : nullptr;
+    a.num_seqs = num_seqs;
     a.Hq = H_q;
     a.Hkv = H_kv;
     a.G = H_q / H_kv;
     a.max_blocks = max_blocks_per_seq;
     a.num_blocks = num_blocks;
-    a.max_splits = L.max_splits;
+    a.balanced = L.balanced;
     a.scale_log2 = scale * attn::kLog2e;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const bool bf16 = dtype == ATTN_BF16;
     if (D == 64)
-        return bf16 ? launch_paged<64, true>(a, num_seqs, stream) : launch_paged<64, false>(a, num_seqs, stream);
-    return bf16 ? launch_paged<128, true>(a, num_seqs, stream) : launch_paged<128, false>(a, num_seqs, stream);
+        return bf16 ? launch_paged<64, true>(tk, tv, a, L.grid, stream)
+                    : launch_paged<64, false>(tk, tv, a, L.grid, stream);
+    return bf16 ? launch_paged<128, true>(tk, tv, a, L.grid, stream)
+                : launch_paged<128, false>(tk, tv, a, L.grid, stream);
 }
 
 // ----------------------------------------------------------- no-allocation decode

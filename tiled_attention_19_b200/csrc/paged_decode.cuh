@@ -5,58 +5,79 @@
 // sequence's logical block to a physical one; the kernel resolves every position
 // through the table ("Fast attention kernels and operator fusion", the-ai.news,
 // section on FlashAttention-style and paged attention; block_size = 16 as in its
-// vLLM example). The softmax is exact: per K/V chunk an online softmax, then the
-// chunks are merged with log-sum-exp weights.
+// vLLM example). The softmax is exact: an online softmax per chunk of blocks, then the
+// chunks of a sequence are merged with log-sum-exp weights.
 //
-// Work unit = (sequence s, K/V head, chunk of kBlocksPerCta blocks). One CTA of
-// kDecWarps warps; each warp owns kBlocksPerWarp whole blocks. All G = H_q / H_kv
-// query heads of the K/V head are processed together as the 16 rows of an
-// m16n8k16 tensor-core tile (rows >= G are zero), so every K/V byte is read once.
+// Work split. A unit is one (sequence, K/V head); its G = H_q / H_kv query heads are
+// the rows of one m16n8k16 tensor-core tile (rows >= G are zero), so every K/V byte is
+// read once. The grid has P = max(kDecCtas, 2U) CTAs for U units. Every CTA reads the
+// sequence lengths and derives the same schedule: the blocks of all units (T in total)
+// are cut into chunks of at most C = ceil(T / (P - U)) blocks, each unit into
+// ceil(blocks / C) near-equal chunks (at least one), which gives at most P chunks; CTA
+// c takes chunk c. One wave of CTAs with equal shares of the bytes: the kernel is bound
+// by HBM bandwidth, not by its longest sequence. (With more than kDecMaxUnits units
+// each CTA takes one whole unit instead.)
 //
-// Fragments come straight from global memory into registers with 16-byte loads:
-//  - Scores: the dot product over D may take the D positions in any order, so the
-//    query and key fragments use the same permutation: mma thread (g, t) holds the
-//    D/4 contiguous dims [t*D/4, (t+1)*D/4) of its token row, slab s taking dims
-//    t*D/4 + 4s .. 4s+3. Each thread loads two 64-byte runs of K per block.
-//  - P·V: output dims are permuted so thread (g, t) holds V columns
-//    g*D/8 .. g*D/8 + D/8 - 1 for its four token rows 2t, 2t+1, 2t+8, 2t+9; the
-//    accumulator of thread (g, t) then covers output dims [2t*D/8, (2t+2)*D/8).
-// The P fragment is the score accumulator itself (the usual register reuse).
-//
-// Split-KV combine: each CTA reduces its warps in shared memory. A sequence that
-// fits one CTA writes O and lse directly. Otherwise each CTA writes its normalised
-// partial O and its log2-sum-exp to the workspace, fences, and bumps a per-(s, head)
-// counter; the CTA that brings the counter to the number of chunks merges all
-// partials and resets the counter to 0.
+// Per CTA: a producer warp reads the chunk's block-table entries and issues 2-D TMA
+// loads (128-byte swizzle) of each block's K and V rows into a ring of shared-memory
+// stages; four consumer warps take the blocks in turn and read their fragments with
+// ldmatrix (.trans for V), so the swizzle keeps the reads free of bank conflicts. Each
+// warp keeps its own running max, sum and output; the CTA merges its warps in shared
+// memory. A unit with one chunk writes O and lse directly; otherwise every chunk writes
+// its normalised output and log2-sum-exp to the workspace, fences and bumps the unit's
+// counter, and the CTA that completes the count merges the chunks and resets the
+// counter to zero.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace attn {
 
-constexpr int kDecWarps = 4;
-constexpr int kBlocksPerWarp = 2;
-constexpr int kBlocksPerCta = kDecWarps * kBlocksPerWarp;
 constexpr int kPageSize = 16;
 constexpr int kMaxGroup = 16;
+constexpr int kDecConsumers = 4;                      // consumer warps
+constexpr int kDecThreads = (kDecConsumers + 1) * 32;  // + the producer warp
+constexpr int kDecStages = 12;                        // blocks in flight per CTA
+constexpr int kDecCtas = 296;                         // two per SM on a 148-SM B200
+constexpr int kDecMaxUnits = 1024;                    // balanced schedule up to this many units
+
+template <int D>
+struct DecodeCfg {
+    static constexpr int kTileBytes = kPageSize * 128;          // one 16-row x 64-column swizzled tile
+    static constexpr int kKBytes = kPageSize * D * 2;           // one block's K rows (D/64 tiles)
+    static constexpr int kStageBytes = 2 * kKBytes;             // K and V
+    // merge buffers, reusing the ring: per-warp O with padded rows plus the factors, or
+    // the chunk weights of one unit. A unit has at most (P - U) + 1 <= kDecMaxUnits + 1
+    // chunks, since P = max(kDecCtas, 2U) and U <= kDecMaxUnits.
+    static constexpr int kMergeBytes = kDecConsumers * kMaxGroup * (D + 8) * 4 + kDecConsumers * kMaxGroup * 4;
+    static constexpr int kWeightBytes = (kDecMaxUnits + 1) * kMaxGroup * 4;
+    static constexpr int kRingBytes = kDecStages * kStageBytes;
+    static constexpr int kBufBytes = kRingBytes > kMergeBytes
+                                         ? (kRingBytes > kWeightBytes ? kRingBytes : kWeightBytes)
+                                         : (kMergeBytes > kWeightBytes ? kMergeBytes : kWeightBytes);
+    static_assert(kDecCtas - 1 <= kDecMaxUnits, "chunks of one unit bounded by kDecMaxUnits + 1");
+    static constexpr int kSmemBytes = 1024 + kBufBytes;         // + alignment slack
+};
 
 struct PagedArgs {
     const uint16_t* q;
-    const uint16_t* kc;
-    const uint16_t* vc;
     const int32_t* block_table;
     const int32_t* seq_lens;
     uint16_t* out;
     float* lse;
-    float* ws_o;      // [S][Hkv][max_splits][G][D]
-    float* ws_lse;    // [S][Hkv][max_splits][G], log2 units
-    int* ws_count;    // [S][Hkv]
-    int Hq, Hkv, G, max_blocks, num_blocks, max_splits;
+    float* ws_o;      // [P][G][D]   normalised chunk outputs
+    float* ws_lse;    // [P][G]      chunk log2-sum-exp
+    int* ws_count;    // [U]         completed chunks per unit
+    int num_seqs, Hq, Hkv, G, max_blocks, num_blocks;
+    int balanced;     // 1: chunked schedule over P CTAs; 0: one CTA per unit
     float scale_log2;
 };
 
-// Workspace layout shared by the size query and the launcher.
+// Grid and workspace layout, shared by the size query and the launcher.
 struct PagedLayout {
-    int max_splits;
+    int grid;
+    int balanced;
     size_t count_off, lse_off, o_off, total;
 };
 
@@ -64,26 +85,43 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline PagedLayout paged_layout(int num_seqs, int Hq, int Hkv, int D, int max_blocks) {
     PagedLayout L{};
-    L.max_splits = max_blocks <= 0 ? 1 : (max_blocks + kBlocksPerCta - 1) / kBlocksPerCta;
-    if (L.max_splits <= 1 || num_seqs <= 0) {
-        L.max_splits = 1;
+    const long long U = static_cast<long long>(num_seqs) * Hkv;
+    if (U <= 0) return L;
+    if (U > kDecMaxUnits) {  // one CTA per unit, no split, no workspace
+        L.grid = static_cast<int>(U);
+        L.balanced = 0;
         return L;
     }
-    const size_t units = static_cast<size_t>(num_seqs) * Hkv;
+    L.balanced = 1;
+    L.grid = static_cast<int>(U * 2 > kDecCtas ? U * 2 : kDecCtas);
+    if (max_blocks <= 1) return L;  // every unit fits one chunk: nothing is ever merged
     const size_t G = Hq / Hkv;
     L.count_off = 0;
-    L.lse_off = align_up(units * sizeof(int), 256);
-    L.o_off = L.lse_off + align_up(units * L.max_splits * G * sizeof(float), 256);
-    L.total = L.o_off + align_up(units * L.max_splits * G * D * sizeof(float), 256);
+    L.lse_off = align_up(static_cast<size_t>(U) * sizeof(int), 256);
+    L.o_off = L.lse_off + align_up(static_cast<size_t>(L.grid) * G * sizeof(float), 256);
+    L.total = L.o_off + align_up(static_cast<size_t>(L.grid) * G * D * sizeof(float), 256);
     return L;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+// 2-D TMA load (x = column, y = row) into shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x,
+                                            int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(tmap), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
 
 template <bool BF16>
@@ -104,318 +142,485 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
     }
 }
 
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+// Byte offset of 16-byte chunk `ch` (of the row's D/8) of token row `row` in a block
+// stored as D/64 swizzled 16 x 64 tiles (the chunk index is XORed with row % 8).
+template <int D>
+__device__ __forceinline__ uint32_t swz(int row, int ch) {
+    return (ch >> 3) * DecodeCfg<D>::kTileBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint16_t to_bits(float x) {
+    if constexpr (BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+    else return __half_as_ushort(__float2half_rn(x));
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kDecWarps * 32)
-    paged_decode_kernel(const PagedArgs a) {
-    constexpr int KU = D / 32;   // 16-byte K loads per token run (D/4 elements)
-    constexpr int VU = D / 64;   // 16-byte V loads per token run (D/8 elements)
-    constexpr int NT = D / 8;    // P·V n-tiles
-    constexpr int SL = D / 16;   // score k-slabs
-    __shared__ float sm_m[kDecWarps][kMaxGroup];
-    __shared__ float sm_l[kDecWarps][kMaxGroup];
-    __shared__ __align__(16) float sm_o[kDecWarps][kMaxGroup][D];
-    __shared__ int sm_last;
+__global__ void __launch_bounds__(kDecThreads, 2)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const PagedArgs a) {
+    using Cfg = DecodeCfg<D>;
+    constexpr int SL = D / 16;  // score k-slabs
+    constexpr int NT = D / 8;   // output n-tiles
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
+    __shared__ int stage_skip[kDecStages];
+    __shared__ int s_nb[kDecMaxUnits];   // blocks per unit
+    __shared__ int s_pre[kDecMaxUnits];  // first chunk index of each unit
+    __shared__ int s_red[8];
+    __shared__ float sm_m[kDecConsumers][kMaxGroup], sm_l[kDecConsumers][kMaxGroup];
+    __shared__ int s_last;
+    __shared__ int s_abort;  // raised by a bounded wait that ran out
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t ring = smem_u32(smem);
 
-    const int split = blockIdx.x;
-    const int hkv = blockIdx.y;
-    const int sq = blockIdx.z;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2;  // mma group id: head row g (and g + 8), or token row
-    const int t = lane & 3;   // thread in group
-
-    int len = a.seq_lens[sq];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int Hkv = a.Hkv, G = a.G;
+    const int U = a.num_seqs * Hkv;
     const int cap = a.max_blocks * kPageSize;
+
+    // The block table is read only after the schedule is known: start pulling it into
+    // L2 now (the CTAs split its 128-byte lines between them).
+    {
+        const size_t tbl_bytes = static_cast<size_t>(a.num_seqs) * a.max_blocks * sizeof(int32_t);
+        const char* tbl = reinterpret_cast<const char*>(a.block_table);
+        for (size_t off = (static_cast<size_t>(blockIdx.x) * blockDim.x + tid) * 128; off < tbl_bytes;
+             off += static_cast<size_t>(gridDim.x) * blockDim.x * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(tbl + off));
+    }
+    // ------------------------------------------------------------ the schedule
+    int unit = -1, b0 = 0, b1 = 0, chunk0 = 0, nchunk = 1;
+    if (a.balanced && U <= 32) {
+        // One warp derives the schedule for up to 32 units with shuffles only.
+        if (warp == 0) {
+            int nbu = 0;
+            if (lane < U) {
+                int len = a.seq_lens[lane / Hkv];
+                if (len < 0 || len > cap) len = len < 0 ? 0 : cap;
+                nbu = (len + kPageSize - 1) / kPageSize;
+            }
+            int T = nbu;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
+            const int P = gridDim.x;
+            const int C = max(1, (T + (P - U) - 1) / (P - U));
+            const int v = lane < U ? max(1, (nbu + C - 1) / C) : 0;
+            int x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            const int start = x - v;  // exclusive prefix
+            const int cta = blockIdx.x;
+            const bool mine = lane < U && cta >= start && cta < start + v;
+            const unsigned who = __ballot_sync(0xffffffffu, mine);
+            if (lane == 0) s_red[0] = who ? (__ffs(who) - 1) : -1;
+            if (mine) {
+                const int k = cta - start;
+                s_red[1] = static_cast<int>(static_cast<long long>(k) * nbu / v);
+                s_red[2] = static_cast<int>(static_cast<long long>(k + 1) * nbu / v);
+                s_red[3] = start;
+                s_red[4] = v;
+            }
+        }
+        __syncthreads();
+        unit = s_red[0];
+        if (unit < 0) return;  // more CTAs than chunks (CTA-uniform)
+        b0 = s_red[1];
+        b1 = s_red[2];
+        chunk0 = s_red[3];
+        nchunk = s_red[4];
+    } else if (a.balanced) {
+        // pass 1: blocks per unit, and their total T
+        int part = 0;
+        for (int u = tid; u < U; u += blockDim.x) {
+            int len = a.seq_lens[u / Hkv];
+            if (len < 0 || len > cap) len = len < 0 ? 0 : cap;  // reported by the unit's CTA
+            const int nbu = (len + kPageSize - 1) / kPageSize;
+            s_nb[u] = nbu;
+            part += nbu;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) s_red[warp] = part;
+        __syncthreads();
+        long long T = 0;
+#pragma unroll
+        for (int w = 0; w < kDecThreads / 32; ++w) T += s_red[w];
+        __syncthreads();
+        const int P = gridDim.x;  // P >= 2U, so P - U >= U >= 1
+        const int C = static_cast<int>(max(1LL, (T + (P - U) - 1) / (P - U)));
+        // pass 2: exclusive prefix over units of the chunk counts max(1, ceil(blocks / C))
+        int carry = 0;
+        for (int base = 0; base < U; base += blockDim.x) {
+            const int u = base + tid;
+            const int v = (u < U) ? max(1, (s_nb[u] + C - 1) / C) : 0;
+            int x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) s_red[warp] = x;
+            __syncthreads();
+            int before = carry, total = 0;
+#pragma unroll
+            for (int w = 0; w < kDecThreads / 32; ++w) {
+                if (w < warp) before += s_red[w];
+                total += s_red[w];
+            }
+            if (u < U) s_pre[u] = before + x - v;
+            carry += total;
+            __syncthreads();
+        }
+        // this CTA's chunk: the last unit whose prefix is <= blockIdx.x
+        const int cta = blockIdx.x;
+        int lo = 0, hi = U - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_pre[mid] <= cta) lo = mid;
+            else hi = mid - 1;
+        }
+        const int nbu = s_nb[lo];
+        const int n = max(1, (nbu + C - 1) / C);
+        if (cta >= s_pre[lo] + n) return;  // more CTAs than chunks (CTA-uniform)
+        unit = lo;
+        const int k = cta - s_pre[lo];
+        b0 = static_cast<int>(static_cast<long long>(k) * nbu / n);
+        b1 = static_cast<int>(static_cast<long long>(k + 1) * nbu / n);
+        chunk0 = s_pre[lo];
+        nchunk = n;
+    } else {
+        unit = blockIdx.x;
+        int len = a.seq_lens[unit / Hkv];
+        if (len < 0 || len > cap) len = len < 0 ? 0 : cap;
+        b1 = (len + kPageSize - 1) / kPageSize;
+    }
+    const int sq = unit / Hkv;
+    const int hkv = unit % Hkv;
+    int len = a.seq_lens[sq];
     if (len < 0 || len > cap) {
-        report_status(ATTN_ERR_BAD_INDEX);
+        if (tid == 0 && b0 == 0) report_status(ATTN_ERR_BAD_INDEX);
         len = len < 0 ? 0 : cap;
     }
-    const int nblk = (len + kPageSize - 1) / kPageSize;
-    const int nsplit = nblk == 0 ? 1 : (nblk + kBlocksPerCta - 1) / kBlocksPerCta;
-    if (split >= nsplit) return;
-    const int G = a.G;
+    const int nb = b1 - b0;
 
-    // ---- query fragments (rows = the G heads of this K/V head, zero-padded to 16)
-    uint32_t qa[SL][4];
-    {
-        const uint16_t* qbase = a.q + (static_cast<size_t>(sq) * a.Hq + hkv * G) * D + t * (D / 4);
-        uint4 q0[KU], q1[KU];
-#pragma unroll
-        for (int u = 0; u < KU; ++u) {
-            q0[u] = g < G ? *reinterpret_cast<const uint4*>(qbase + static_cast<size_t>(g) * D + u * 8)
-                          : make_uint4(0, 0, 0, 0);
-            q1[u] = g + 8 < G
-                        ? *reinterpret_cast<const uint4*>(qbase + static_cast<size_t>(g + 8) * D + u * 8)
-                        : make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
         }
-#pragma unroll
-        for (int s = 0; s < SL; ++s) {
-            const int u = s >> 1, w = (s & 1) * 2;
-            qa[s][0] = word_of(q0[u], w);      // row g,   dims 4s+0,1 of the run
-            qa[s][1] = word_of(q1[u], w);      // row g+8
-            qa[s][2] = word_of(q0[u], w + 1);  // row g,   dims 4s+2,3
-            qa[s][3] = word_of(q1[u], w + 1);  // row g+8
-        }
-    }
-
-    // ---- issue every K/V load of this warp's blocks up front
-    const int blk_first = split * kBlocksPerCta + warp * kBlocksPerWarp;
-    uint4 kr[kBlocksPerWarp][2][KU];
-    uint4 vr[kBlocksPerWarp][4][VU];
-    bool valid[kBlocksPerWarp];
-#pragma unroll
-    for (int i = 0; i < kBlocksPerWarp; ++i) {
-        const int blk = blk_first + i;
-        int phys = -1;
-        if (blk < nblk) {
-            phys = a.block_table[static_cast<size_t>(sq) * a.max_blocks + blk];
-            if (phys < 0 || phys >= a.num_blocks) {
-                report_status(ATTN_ERR_BAD_INDEX);
-                phys = -1;
-            }
-        }
-        valid[i] = phys >= 0;
-        if (valid[i]) {
-            const size_t base = (static_cast<size_t>(phys) * a.Hkv + hkv) * kPageSize * D;
-            const uint16_t* kb = a.kc + base;
-            const uint16_t* vb = a.vc + base;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int u = 0; u < KU; ++u)
-                    kr[i][nt][u] = ldg_stream(kb + (nt * 8 + g) * D + t * (D / 4) + u * 8);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int tok = 2 * t + (r & 1) + (r >> 1) * 8;
-#pragma unroll
-                for (int u = 0; u < VU; ++u)
-                    vr[i][r][u] = ldg_stream(vb + tok * D + g * (D / 8) + u * 8);
-            }
-        } else {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int u = 0; u < KU; ++u) kr[i][nt][u] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int u = 0; u < VU; ++u) vr[i][r][u] = make_uint4(0, 0, 0, 0);
-        }
-    }
-
-    // ---- online softmax over this warp's blocks (rows g and g+8)
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float oacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
-    const float c = a.scale_log2;
-
-#pragma unroll
-    for (int i = 0; i < kBlocksPerWarp; ++i) {
-        if (!valid[i]) continue;  // warp-uniform
-        const int tok0 = (blk_first + i) * kPageSize;
-        float sc[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-            for (int s = 0; s < SL; ++s) {
-                const int u = s >> 1, w = (s & 1) * 2;
-                mma16816<BF16>(sc[nt], qa[s], word_of(kr[i][nt][u], w), word_of(kr[i][nt][u], w + 1));
-            }
-        }
-        // columns of the score tile: token tok0 + nt*8 + 2t + e
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const bool in = tok0 + nt * 8 + 2 * t + e < len;
-                sc[nt][e] = in ? sc[nt][e] : -INFINITY;
-                sc[nt][2 + e] = in ? sc[nt][2 + e] : -INFINITY;
-                mx0 = fmaxf(mx0, sc[nt][e]);
-                mx1 = fmaxf(mx1, sc[nt][2 + e]);
-            }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0 * c), mn1 = fmaxf(m1, mx1 * c);
-        const float al0 = (mn0 == m0) ? 1.f : ex2_approx(m0 - mn0);
-        const float al1 = (mn1 == m1) ? 1.f : ex2_approx(m1 - mn1);
-        const float nm0 = (mn0 == -INFINITY) ? 0.f : -mn0;
-        const float nm1 = (mn1 == -INFINITY) ? 0.f : -mn1;
-        float p[2][4];
-        float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            p[nt][0] = ex2_approx(fmaf(sc[nt][0], c, nm0));
-            p[nt][1] = ex2_approx(fmaf(sc[nt][1], c, nm0));
-            p[nt][2] = ex2_approx(fmaf(sc[nt][2], c, nm1));
-            p[nt][3] = ex2_approx(fmaf(sc[nt][3], c, nm1));
-            rs0 += p[nt][0] + p[nt][1];
-            rs1 += p[nt][2] + p[nt][3];
-        }
-        l0 = l0 * al0 + rs0;
-        l1 = l1 * al1 + rs1;
-        m0 = mn0;
-        m1 = mn1;
-        const uint32_t pa[4] = {pack2<BF16>(p[0][0], p[0][1]), pack2<BF16>(p[0][2], p[0][3]),
-                                pack2<BF16>(p[1][0], p[1][1]), pack2<BF16>(p[1][2], p[1][3])};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            oacc[nt][0] *= al0;
-            oacc[nt][1] *= al0;
-            oacc[nt][2] *= al1;
-            oacc[nt][3] *= al1;
-            // column g of this n-tile is output dim g*D/8 + nt: element nt of each token run
-            const int u = nt >> 3, wsel = (nt & 7) >> 1;
-            const uint32_t sel = (nt & 1) ? 0x7632u : 0x5410u;
-            const uint32_t b0 = __byte_perm(word_of(vr[i][0][u], wsel), word_of(vr[i][1][u], wsel), sel);
-            const uint32_t b1 = __byte_perm(word_of(vr[i][2][u], wsel), word_of(vr[i][3][u], wsel), sel);
-            mma16816<BF16>(oacc[nt], pa, b0, b1);
-        }
-    }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-
-    // ---- reduce the warps of this CTA in shared memory
-    if (t == 0) {
-        sm_m[warp][g] = m0;
-        sm_l[warp][g] = l0;
-        sm_m[warp][g + 8] = m1;
-        sm_l[warp][g + 8] = l1;
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        // accumulator columns 2t, 2t+1 are output dims 2t*D/8 + nt and (2t+1)*D/8 + nt
-        sm_o[warp][g][(2 * t) * (D / 8) + nt] = oacc[nt][0];
-        sm_o[warp][g][(2 * t + 1) * (D / 8) + nt] = oacc[nt][1];
-        sm_o[warp][g + 8][(2 * t) * (D / 8) + nt] = oacc[nt][2];
-        sm_o[warp][g + 8][(2 * t + 1) * (D / 8) + nt] = oacc[nt][3];
+        s_abort = 0;
+        fence_barrier_init();
     }
     __syncthreads();
 
-    const bool direct = nsplit == 1;
-    const size_t unit = static_cast<size_t>(sq) * a.Hkv + hkv;
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int r = idx / D, d = idx % D;
-        float M = -INFINITY;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g + 8
+    float oacc[NT][4];
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][r]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
+    for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+    const int g = lane >> 2, t = lane & 3;
+    volatile int* abort_flag = &s_abort;
+    int issued = 0;  // producer: blocks whose loads were issued
+
+    if (warp == kDecConsumers) {
+        // ---------------------------------------------------------------- producer
+        for (int base = 0; base < nb; base += 32) {
+            int phys = -1;
+            if (base + lane < nb) {
+                phys = a.block_table[static_cast<size_t>(sq) * a.max_blocks + b0 + base + lane];
+                if (phys < 0 || phys >= a.num_blocks) {
+                    report_status(ATTN_ERR_BAD_INDEX);
+                    phys = -1;
+                }
+            }
+            const int n_here = min(32, nb - base);
+            bool ok = true;
+            for (int k = 0; k < n_here; ++k) {
+                const int i = base + k;
+                const int p = __shfl_sync(0xffffffffu, phys, k);
+                if (lane == 0) {
+                    const int s = i % kDecStages;
+                    if (i >= kDecStages &&
+                        !wait_phase(smem_u32(&empty_bar[s]), ((i / kDecStages) - 1) & 1, abort_flag))
+                        ok = false;
+                    const uint32_t fb = smem_u32(&full_bar[s]);
+                    if (!ok) {
+                        // gave up: issue nothing more
+                    } else
+                    if (p < 0) {
+                        stage_skip[s] = 1;
+                        mbar_arrive(fb);
+                    } else {
+                        stage_skip[s] = 0;
+                        mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+                        const int row = (p * Hkv + hkv) * kPageSize;
+                        const uint32_t dst = ring + s * Cfg::kStageBytes;
 #pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) {
-                const float f = ex2_approx(sm_m[w][r] - M);
-                L += f * sm_l[w][r];
-                O += f * sm_o[w][r][d];
+                        for (int c = 0; c < D / 64; ++c) {
+                            tma_load_2d(dst + c * Cfg::kTileBytes, &tm_k, fb, c * 64, row);
+                            tma_load_2d(dst + Cfg::kKBytes + c * Cfg::kTileBytes, &tm_v, fb, c * 64, row);
+                        }
+                    }
+                    if (ok) issued = i + 1;
+                }
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            }
+            if (*abort_flag) break;
+        }
+    } else {
+        // ---------------------------------------------------------------- consumers
+        // query fragments (A operand, natural order): rows g, g + 8 = heads of the group
+        uint32_t qa[SL][4];
+        {
+            const uint16_t* qb = a.q + (static_cast<size_t>(sq) * a.Hq + hkv * G) * D;
+#pragma unroll
+            for (int s = 0; s < SL; ++s) {
+                const int d = 16 * s + 2 * t;
+                qa[s][0] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * D + d) : 0u;
+                qa[s][1] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d) : 0u;
+                qa[s][2] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * D + d + 8) : 0u;
+                qa[s][3] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d + 8) : 0u;
             }
         }
-        const float on = L > 0.f ? O / L : 0.f;
-        const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
+        const float c = a.scale_log2;
+        // ldmatrix lane roles: K (x4): token (lane>>4)*8 + lane%8, chunk 2s + (lane>>3)%2;
+        // V (x4.trans): token ((lane>>3)&1)*8 + lane%8, chunk 2p + (lane>>4).
+        const int k_tok = ((lane >> 4) << 3) + (lane & 7), k_sub = (lane >> 3) & 1;
+        const int v_tok = (((lane >> 3) & 1) << 3) + (lane & 7), v_sub = lane >> 4;
+        for (int i = warp; i < nb; i += kDecConsumers) {
+            const int s = i % kDecStages;
+            const bool ready = __all_sync(
+                0xffffffffu, wait_phase(smem_u32(&full_bar[s]), (i / kDecStages) & 1, abort_flag));
+            if (!ready) break;
+            if (!stage_skip[s]) {
+                const uint32_t kb = ring + s * Cfg::kStageBytes;
+                const uint32_t vb = kb + Cfg::kKBytes;
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int sl = 0; sl < SL; ++sl) {
+                    uint32_t kf[4];
+                    ldsm_x4(kb + swz<D>(k_tok, 2 * sl + k_sub), kf);
+                    mma16816<BF16>(sc[0], qa[sl], kf[0], kf[1]);
+                    mma16816<BF16>(sc[1], qa[sl], kf[2], kf[3]);
+                }
+                const int tok0 = (b0 + i) * kPageSize;
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool in = tok0 + nt * 8 + 2 * t + e < len;
+                        sc[nt][e] = in ? sc[nt][e] : -INFINITY;
+                        sc[nt][2 + e] = in ? sc[nt][2 + e] : -INFINITY;
+                        mx0 = fmaxf(mx0, sc[nt][e]);
+                        mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                    }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0 * c), mn1 = fmaxf(m1, mx1 * c);
+                const float al0 = (mn0 == m0) ? 1.f : ex2_approx(m0 - mn0);
+                const float al1 = (mn1 == m1) ? 1.f : ex2_approx(m1 - mn1);
+                const float nm0 = (mn0 == -INFINITY) ? 0.f : -mn0;
+                const float nm1 = (mn1 == -INFINITY) ? 0.f : -mn1;
+                float p[2][4];
+                float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    p[nt][0] = ex2_approx(fmaf(sc[nt][0], c, nm0));
+                    p[nt][1] = ex2_approx(fmaf(sc[nt][1], c, nm0));
+                    p[nt][2] = ex2_approx(fmaf(sc[nt][2], c, nm1));
+                    p[nt][3] = ex2_approx(fmaf(sc[nt][3], c, nm1));
+                    rs0 += p[nt][0] + p[nt][1];
+                    rs1 += p[nt][2] + p[nt][3];
+                }
+                l0 = l0 * al0 + rs0;
+                l1 = l1 * al1 + rs1;
+                m0 = mn0;
+                m1 = mn1;
+                const uint32_t pa[4] = {pack2<BF16>(p[0][0], p[0][1]), pack2<BF16>(p[0][2], p[0][3]),
+                                        pack2<BF16>(p[1][0], p[1][1]), pack2<BF16>(p[1][2], p[1][3])};
+#pragma unroll
+                for (int pp = 0; pp < NT / 2; ++pp) {
+                    uint32_t vf[4];
+                    ldsm_x4_t(vb + swz<D>(v_tok, 2 * pp + v_sub), vf);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        float* o = oacc[2 * pp + h2];
+                        o[0] *= al0;
+                        o[1] *= al0;
+                        o[2] *= al1;
+                        o[3] *= al1;
+                        mma16816<BF16>(oacc[2 * pp + h2], pa, vf[2 * h2], vf[2 * h2 + 1]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+        }
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    }
+    __syncthreads();  // every stage consumed: the ring is free for the merge buffers
+    if (*abort_flag) {
+        // A wait ran out (reported as ATTN_ERR_TIMEOUT): let the loads already issued
+        // land before this CTA's shared memory is reused or released, then stop.
+        if (warp == kDecConsumers && lane == 0)
+            for (int i = max(0, issued - kDecStages); i < issued; ++i)
+                drain_phase(smem_u32(&full_bar[i % kDecStages]), (i / kDecStages) & 1);
+        return;
+    }
+
+    // ---------------------------------------------------- merge this CTA's warps
+    // Per-warp outputs in shared memory (row stride D + 8 floats keeps the fragment
+    // stores at most two-way bank conflicted), then one scale factor per (warp, row).
+    constexpr int kRow = D + 8;
+    float* sm_o = reinterpret_cast<float*>(smem);  // [kDecConsumers][16][kRow]
+    float* sm_f = sm_o + kDecConsumers * kMaxGroup * kRow;  // [kDecConsumers][16] factors
+    if (warp < kDecConsumers) {
+        if (t == 0) {
+            sm_m[warp][g] = m0;
+            sm_l[warp][g] = l0;
+            sm_m[warp][g + 8] = m1;
+            sm_l[warp][g + 8] = l1;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float* r0 = sm_o + (warp * kMaxGroup + g) * kRow + nt * 8 + 2 * t;
+            float* r1 = sm_o + (warp * kMaxGroup + g + 8) * kRow + nt * 8 + 2 * t;
+            r0[0] = oacc[nt][0];
+            r0[1] = oacc[nt][1];
+            r1[0] = oacc[nt][2];
+            r1[1] = oacc[nt][3];
+        }
+    }
+    __syncthreads();
+    __shared__ float s_rowM[kMaxGroup], s_rowL[kMaxGroup];
+    if (tid < G) {
+        const int r = tid;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) M = fmaxf(M, sm_m[w][r]);
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) {
+            const float f = (M == -INFINITY) ? 0.f : ex2_approx(sm_m[w][r] - M);
+            sm_f[w * kMaxGroup + r] = f;
+            L += f * sm_l[w][r];
+        }
+        s_rowM[r] = M;
+        s_rowL[r] = L;
+    }
+    __syncthreads();
+
+    const bool direct = nchunk == 1;
+    const int cidx = blockIdx.x;  // chunk index (balanced schedule; unused when direct)
+    for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
+        const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
+        const float L = s_rowL[r];
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) {
+            const float f = sm_f[w * kMaxGroup + r] * inv;
+            const float4 v = *reinterpret_cast<const float4*>(sm_o + (w * kMaxGroup + r) * kRow + d);
+            o.x += f * v.x;
+            o.y += f * v.y;
+            o.z += f * v.z;
+            o.w += f * v.w;
+        }
+        const float lse2 = L > 0.f ? s_rowM[r] + log2f(L) : -INFINITY;
         if (direct) {
             const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
-            a.out[orow * D + d] = static_cast<uint16_t>(BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(on))
-                                                             : __half_as_ushort(__float2half_rn(on)));
+            uint2 pk;
+            pk.x = pack2<BF16>(o.x, o.y);
+            pk.y = pack2<BF16>(o.z, o.w);
+            *reinterpret_cast<uint2*>(a.out + orow * D + d) = pk;
             if (d == 0 && a.lse != nullptr) a.lse[orow] = lse2 * kLn2;
         } else {
-            const size_t prow = (unit * a.max_splits + split) * G + r;
-            a.ws_o[prow * D + d] = on;
+            const size_t prow = static_cast<size_t>(cidx) * G + r;
+            *reinterpret_cast<float4*>(a.ws_o + prow * D + d) = o;
             if (d == 0) a.ws_lse[prow] = lse2;
         }
     }
     if (direct) return;
 
-    // ---- last CTA of this (sequence, head) merges the chunks
+    // ---------------------------------------------- the last chunk merges the unit
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const int prev = atomicAdd(&a.ws_count[unit], 1);
-        sm_last = prev == nsplit - 1;
-    }
+    if (tid == 0) s_last = atomicAdd(&a.ws_count[unit], 1) == nchunk - 1;
     __syncthreads();
-    if (!sm_last) return;
+    if (!s_last) return;
     __threadfence();
-    // Row statistics: one warp per head row reduces the chunks' log2-sum-exp values in
-    // parallel (32 loads in flight per warp, not a serial chain).
-    const size_t lse0 = unit * a.max_splits * G;  // + sp * G + r
-    for (int r = warp; r < G; r += kDecWarps) {
+    // All chunks' log2-sum-exp in shared memory at once (one round of parallel loads),
+    // then per row the maximum, the total weight and each chunk's normalised weight.
+    float* s_w = sm_o;  // [nchunk][G], reused
+    const int nw = nchunk * G;
+    for (int i = tid; i < nw; i += blockDim.x)
+        s_w[i] = __ldcg(a.ws_lse + static_cast<size_t>(chunk0) * G + i);
+    __syncthreads();
+    for (int r = warp; r < G; r += kDecThreads / 32) {
         float M = -INFINITY;
-        for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, __ldcg(a.ws_lse + lse0 + sp * G + r));
+        for (int k = lane; k < nchunk; k += 32) M = fmaxf(M, s_w[k * G + r]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float W = 0.f;
         if (M != -INFINITY)
-            for (int sp = lane; sp < nsplit; sp += 32) W += ex2_approx(__ldcg(a.ws_lse + lse0 + sp * G + r) - M);
+            for (int k = lane; k < nchunk; k += 32) W += ex2_approx(s_w[k * G + r] - M);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
         if (lane == 0) {
-            sm_m[0][r] = M;
-            sm_l[0][r] = W;
+            s_rowM[r] = M;
+            s_rowL[r] = W;
         }
     }
     __syncthreads();
-    // Weighted sum of the chunks' normalised outputs, kCombineChunk chunks at a time
-    // with their weights staged in shared memory (reusing the warp-reduction buffer).
-    float* wbuf = &sm_o[0][0][0];
-    constexpr int kCombineChunk = (kDecWarps * kMaxGroup * D) / kMaxGroup;  // chunks per pass
-    float acc[(kMaxGroup * D + kDecWarps * 32 - 1) / (kDecWarps * 32)];
+    for (int i = tid; i < nw; i += blockDim.x) {
+        const int r = i % G;
+        const float M = s_rowM[r], W = s_rowL[r];
+        s_w[i] = (M == -INFINITY || !(W > 0.f)) ? 0.f : ex2_approx(s_w[i] - M) / W;
+    }
+    __syncthreads();
+    // Each thread owns one 4-float slice of the output and sums it over the chunks,
+    // eight independent loads in flight at a time.
+    for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
+        const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
+        const float4* src = reinterpret_cast<const float4*>(a.ws_o + (static_cast<size_t>(chunk0) * G + r) * D + d);
+        const size_t step = static_cast<size_t>(G) * D / 4;  // float4 stride between chunks
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < nchunk; k += 8) {
+            float4 v[8];
 #pragma unroll
-    for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) acc[e] = 0.f;
-    for (int c0 = 0; c0 < nsplit; c0 += kCombineChunk) {
-        const int cn = min(kCombineChunk, nsplit - c0);
-        __syncthreads();
-        for (int i = threadIdx.x; i < cn * G; i += blockDim.x) {
-            const int sp = c0 + i / G, r = i % G;
-            const float M = sm_m[0][r], W = sm_l[0][r];
-            wbuf[i] = (M == -INFINITY) ? 0.f : ex2_approx(__ldcg(a.ws_lse + lse0 + sp * G + r) - M) / W;
-        }
-        __syncthreads();
+            for (int u = 0; u < 8; ++u)
+                v[u] = (k + u < nchunk) ? __ldcg(src + (k + u) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) {
-            const int idx = threadIdx.x + e * blockDim.x;
-            if (idx < G * D) {
-                const int r = idx / D;
-                const float* src = a.ws_o + (lse0 + static_cast<size_t>(c0) * G) * D + idx;
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-                int i = 0;
-                for (; i + 4 <= cn; i += 4) {
-                    const float o0 = __ldcg(src + static_cast<size_t>(i) * G * D);
-                    const float o1 = __ldcg(src + static_cast<size_t>(i + 1) * G * D);
-                    const float o2 = __ldcg(src + static_cast<size_t>(i + 2) * G * D);
-                    const float o3 = __ldcg(src + static_cast<size_t>(i + 3) * G * D);
-                    s0 += wbuf[i * G + r] * o0;
-                    s1 += wbuf[(i + 1) * G + r] * o1;
-                    s2 += wbuf[(i + 2) * G + r] * o2;
-                    s3 += wbuf[(i + 3) * G + r] * o3;
-                }
-                for (; i < cn; ++i) s0 += wbuf[i * G + r] * __ldcg(src + static_cast<size_t>(i) * G * D);
-                acc[e] += (s0 + s1) + (s2 + s3);
+            for (int u = 0; u < 8; ++u) {
+                const float w = (k + u < nchunk) ? s_w[(k + u) * G + r] : 0.f;
+                acc.x += w * v[u].x;
+                acc.y += w * v[u].y;
+                acc.z += w * v[u].z;
+                acc.w += w * v[u].w;
             }
         }
-    }
-#pragma unroll
-    for (int e = 0; e < (int)(sizeof(acc) / sizeof(float)); ++e) {
-        const int idx = threadIdx.x + e * blockDim.x;
-        if (idx < G * D) {
-            const int r = idx / D, d = idx % D;
-            const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
-            a.out[orow * D + d] = static_cast<uint16_t>(BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[e]))
-                                                             : __half_as_ushort(__float2half_rn(acc[e])));
-            if (d == 0 && a.lse != nullptr) {
-                const float M = sm_m[0][r], W = sm_l[0][r];
-                a.lse[orow] = (M == -INFINITY || !(W > 0.f)) ? -INFINITY : (M + log2f(W)) * kLn2;
-            }
+        const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
+        uint2 pk;
+        pk.x = pack2<BF16>(acc.x, acc.y);
+        pk.y = pack2<BF16>(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(a.out + orow * D + d) = pk;
+        if (d == 0 && a.lse != nullptr) {
+            const float M = s_rowM[r], W = s_rowL[r];
+            a.lse[orow] = (M == -INFINITY || !(W > 0.f)) ? -INFINITY : (M + log2f(W)) * kLn2;
         }
     }
-    if (threadIdx.x == 0) a.ws_count[unit] = 0;  // leave the workspace as found
+    if (tid == 0) a.ws_count[unit] = 0;  // leave the workspace as found
 }
 
 }  // namespace attn
