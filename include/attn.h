@@ -98,9 +98,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
 
 /*
  * attn_paged_workspace_size -- bytes of device workspace attn_fwd_paged needs
- * for these sizes (0 when no split is ever needed). The workspace holds the
- * partial results of the split-KV chunks and one completion counter per
- * (sequence, K/V head).
+ * for these sizes (0 when no sequence is ever split). The workspace holds the
+ * partial results of the split-KV chunks (one per CTA of the balanced
+ * schedule) and one completion counter per (sequence, K/V head).
  */
 size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D,
                                  int max_blocks_per_seq, int block_size);
@@ -157,7 +157,7 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
  * the workspace. A problem whose attn_paged_workspace_size() exceeds 4 MiB is
  * rejected with ATTN_ERR_SCRATCH_LIMIT before anything is enqueued. The
  * decode workload of 16 sequences, 12/2 heads, D = 128, 256 blocks per
- * sequence needs 3,170,560 bytes.
+ * sequence needs 916,736 bytes.
  *
  * The first call on a device looks up the array's device address with that
  * device current (cudaGetSymbolAddress); make that first call before any
