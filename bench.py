@@ -35,8 +35,10 @@ sys.path.insert(0, ROOT)
 from tiled_attention_19_b200 import inputs  # noqa: E402
 
 PREFILL = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
+PREFILL_DEFAULT = PREFILL.name
 DECODE = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
 METRIC = "fwd attention TFLOP/s & % of FP16 tensor peak; paged decode HBM GB/s"
+L2_BYTES = 126 * 1000 * 1000
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["tiled_attention_19_b200/csrc/" + f for f in
                   ("api.cu", "common.cuh", "ptx.cuh", "prefill_sm100.cuh", "paged_decode.cuh")]
@@ -143,6 +145,14 @@ def barrier(ws: int):
         dist.barrier()
 
 
+def job_rate(work_per_rank: float, ms_max_over_ranks: float, ws: int, unit_scale: float):
+    """Whole-job throughput of weak-scaled replicas: every rank processes the same
+    amount of work, and the job takes as long as the slowest rank."""
+    if not (ms_max_over_ranks == ms_max_over_ranks) or ms_max_over_ranks <= 0:
+        return None
+    return ws * work_per_rank / (ms_max_over_ranks * 1e-3) / unit_scale
+
+
 # ----------------------------------------------------------------- our GPU arm
 class Workload:
     """Device copies of the step's inputs (rotated) and its outputs."""
@@ -152,11 +162,15 @@ class Workload:
         xp = inputs.make(PREFILL)
         xd = inputs.make(DECODE)
         self.xp_host, self.xd_host = xp, xd
-        self.pf = [{k: v.to(device) for k, v in xp.items()} for _ in range(copies)]
+        # enough prefill copies that one rotation spans more than twice the 126 MB L2
+        per_copy = sum(v.numel() * v.element_size() for v in xp.values())
+        self.p_copies = max(copies, -(-2 * L2_BYTES // per_copy)) if copies > 1 else 1
+        self.pf = [{k: v.to(device) for k, v in xp.items()} for _ in range(self.p_copies)]
         self.dc = [{k: v.to(device) for k, v in xd.items()} for _ in range(copies)]
         self.copies = copies
         self.p_out = torch.empty_like(self.pf[0]["q"])
         self.p_lse = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Lq, device=device)
+        self.prefill_bytes = inputs.dense_bytes(PREFILL)
         self.d_out = torch.empty_like(self.dc[0]["q"])
         self.d_lse = torch.empty(DECODE.num_seqs, DECODE.Hq, device=device)
         self.prefill_flops = PREFILL.flops()
@@ -177,12 +191,12 @@ def run_ours(args, ws, rank, local):
                                 DECODE.max_blocks, device)
 
     def step(i, ev=None):
-        p = w.pf[i % copies]
+        p = w.pf[i % w.p_copies]
         d = w.dc[i % copies]
         if ev is not None:
             ev[0].record(stream)
         if do_pre:
-            ta.fwd(p["q"], p["k"], p["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
+            ta.fwd(p["q"], p["k"], p["v"], causal=PREFILL.causal, scale=PREFILL.scale, out=w.p_out,
                    lse=w.p_lse, stream=stream)
         if ev is not None:
             ev[1].record(stream)
@@ -234,18 +248,13 @@ def run_ours(args, ws, rank, local):
         return None
     peaks, peaks_src = load_peaks()
 
-    def rate(work, ms, scale_):
-        if not (ms == ms) or ms <= 0:  # NaN or nothing timed
-            return None
-        return work / (ms * 1e-3) / scale_
-
-    tflops = rate(ws * w.prefill_flops, pre_avg, 1e12) if do_pre else None
-    gbs = rate(ws * w.decode_bytes, dec_avg, 1e9) if do_dec else None
+    tflops = job_rate(w.prefill_flops, pre_avg, ws, 1e12) if do_pre else None
+    gbs = job_rate(w.decode_bytes, dec_avg, ws, 1e9) if do_dec else None
     per_gpu_tflops = tflops / ws if tflops is not None else None
     per_gpu_gbs = gbs / ws if gbs is not None else None
     r2 = lambda x, n: None if x is None else round(x, n)  # noqa: E731
-    e2e_tf = rate(ws * w.prefill_flops, e2e_pre, 1e12) if do_pre else None
-    e2e_gb = rate(ws * w.decode_bytes, e2e_dec, 1e9) if do_dec else None
+    e2e_tf = job_rate(w.prefill_flops, e2e_pre, ws, 1e12) if do_pre else None
+    e2e_gb = job_rate(w.decode_bytes, e2e_dec, ws, 1e9) if do_dec else None
     traffic = profiled_traffic()
     pk_t = peaks["bf16_tflops_sustained"]
     pk_h = peaks["hbm_gbs"]
@@ -264,18 +273,22 @@ def run_ours(args, ws, rank, local):
         "data": "synthetic (seeded N(0,1) inputs shaped like the pages' workloads)",
         "config": {
             "workload": f"{PREFILL.name} + {DECODE.name}",
-            "prefill": {"B": PREFILL.B, "H": PREFILL.Hq, "L": PREFILL.Lq, "D": PREFILL.D,
-                        "causal": True, "dtype": "bf16", "flops": w.prefill_flops},
+            "prefill": {"B": PREFILL.B, "H": PREFILL.Hq, "Lq": PREFILL.Lq, "Lk": PREFILL.Lk,
+                        "D": PREFILL.D, "causal": PREFILL.causal,
+                        "dtype": "bf16" if PREFILL.dtype == torch.bfloat16 else "f16",
+                        "flops": w.prefill_flops},
             "decode": {"seqs": DECODE.num_seqs, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv,
                        "D": DECODE.D, "block_size": DECODE.block_size,
                        "tokens": int(w.xd_host["seq_lens"].sum()),
                        "bytes": w.decode_bytes},
-            "l2": "inputs rotate over 4 device copies (prefill 4 x 96 MiB, decode pool 4 x 67 MB), "
-                  "larger than the 126 MB L2",
+            "l2": f"inputs rotate over device copies larger than the 126 MB L2: prefill "
+                  f"{w.p_copies} x {sum(v.numel() * v.element_size() for v in w.xp_host.values()) / 1e6:.1f} MB, "
+                  f"decode pool {copies} x 67 MB",
             "parallelism": f"replicas x{ws} (independent problems per GPU)",
         },
         "roofline": {
-            "kernel": "prefill_fwd_kernel<128,bf16,causal>",
+            "kernel": f"prefill_fwd_kernel<{PREFILL.D},{'bf16' if PREFILL.dtype == torch.bfloat16 else 'f16'},"
+                      f"{'causal' if PREFILL.causal else 'full'}>",
             "bound": "tensor",
             "achieved": r2(per_gpu_tflops, 2),
             "peak": pk_t,
@@ -336,7 +349,7 @@ def measure_e2e(w, ta, stream, device, steps: int):
         e[0].record(stream)
         for k in dp:
             dp[k].copy_(hp[k], non_blocking=True)
-        ta.fwd(dp["q"], dp["k"], dp["v"], causal=True, scale=PREFILL.scale, out=w.p_out,
+        ta.fwd(dp["q"], dp["k"], dp["v"], causal=PREFILL.causal, scale=PREFILL.scale, out=w.p_out,
                lse=w.p_lse, stream=stream)
         op.copy_(w.p_out, non_blocking=True)
         lp.copy_(w.p_lse, non_blocking=True)
@@ -455,7 +468,12 @@ def main(argv=None):
                     help="run one kernel of the step only (profiling runs)")
     ap.add_argument("--copies", type=int, default=4,
                     help="device copies of the inputs the steps rotate over (4 > L2)")
+    ap.add_argument("--prefill-workload", default=PREFILL_DEFAULT,
+                    choices=[n for n, w in inputs.WORKLOADS.items() if w.kind == "dense"],
+                    help="dense workload of the prefill call (default: the long causal prefill)")
     args = ap.parse_args(argv)
+    global PREFILL
+    PREFILL = inputs.WORKLOADS[args.prefill_workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()

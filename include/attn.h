@@ -188,6 +188,16 @@ const char* attn_error_string(attn_status_t status);
  */
 attn_status_t attn_get_device_status(void* stream);
 
+/*
+ * attn_selftest_bounded_wait -- exercise the kernels' failure detection without a
+ * fault. Launches one CTA that waits, through the same bounded wait the attention
+ * kernels use, on a barrier that nothing completes. The wait gives up after about a
+ * second, sets ATTN_ERR_TIMEOUT in the device status word and the kernel returns; the
+ * context stays usable. Returns ATTN_OK once enqueued (ATTN_ERR_DEVICE without an
+ * sm_100 device); read the outcome with attn_get_device_status().
+ */
+attn_status_t attn_selftest_bounded_wait(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,66 @@
+"""The multi-GPU bench path on CPU: two gloo ranks on 127.0.0.1.
+
+bench.py runs independent replicas (the hot path shards with no exchange): each rank
+times its own step, the job time is the slowest rank's (max over ranks), and the job
+throughput is all ranks' work over that time. These tests run that host-side logic
+with world_size 2 on the gloo backend.
+"""
+from __future__ import annotations
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, ws: int, port: int, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        got_ws, got_rank, got_local = bench.dist_env()
+        bench.barrier(ws)
+        mine = 10.0 + 5.0 * rank            # this rank's step time (ms)
+        mx = bench.reduce_max(mine, ws, "cpu")
+        rate = bench.job_rate(2.0e12, mx, ws, 1e12)  # 2 TFLOP per rank per step
+        bench.barrier(ws)
+        out[rank] = (got_ws, got_rank, got_local, mx, rate)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_take_the_slowest_rank_and_sum_the_work():
+    ws = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(ws, _free_port(), out), nprocs=ws, join=True)
+        res = dict(out)
+    for rank in range(ws):
+        got_ws, got_rank, got_local, mx, rate = res[rank]
+        assert (got_ws, got_rank, got_local) == (2, rank, rank)
+        assert mx == 15.0                       # max over ranks, not the rank's own
+        assert rate == pytest.approx(2 * 2.0e12 / 15e-3 / 1e12)
+
+
+def test_job_rate_single_rank_and_degenerate_times():
+    assert bench.job_rate(1e12, 1.0, 1, 1e12) == pytest.approx(1000.0)
+    assert bench.job_rate(1e12, 0.0, 1, 1e12) is None
+    assert bench.job_rate(1e12, float("nan"), 1, 1e12) is None
+
+
+def test_reference_arm_prints_only_on_rank_zero(monkeypatch):
+    class A:
+        steps, warmup, cpu_seconds = 1, 3, 0.1
+    assert bench.run_reference(A(), 2, 1) is None   # rank 1: no work, exits quietly

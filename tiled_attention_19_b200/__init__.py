@@ -38,6 +38,7 @@ SIGNATURES = {
                                     _i, _f, _i, _vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_get_device_status": (_i, [_vp]),
+    "attn_selftest_bounded_wait": (_i, [_vp]),
 }
 
 _lib = None

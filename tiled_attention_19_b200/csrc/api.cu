@@ -291,6 +291,31 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
                 : launch_paged<128, false>(tk, tv, a, L.grid, stream);
 }
 
+// ------------------------------------------------------------ failure detection
+namespace attn {
+// One CTA waits on an mbarrier that nothing ever completes, through the same bounded
+// wait the attention kernels use: the wait must give up, report ATTN_ERR_TIMEOUT in the
+// device status word and let the kernel return.
+__global__ void selftest_wait_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wait_phase(smem_u32(&bar), 0, &abort_flag);
+}
+}  // namespace attn
+
+extern "C" attn_status_t attn_selftest_bounded_wait(void* stream_) {
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    attn::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>();
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // ----------------------------------------------------------- no-allocation decode
 // Scratch for attn_fwd_paged_noalloc: a fixed 4 MiB array in this library's own device
 // module. Every GPU that loads the library holds it until the process exits. In host
