@@ -52,6 +52,9 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(key)
         lib.oracle_attn_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
                                         _i64, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_fwd_window.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                               _i64, _i64, ctypes.c_double, ctypes.c_int, _i64,
+                                               _i64, ctypes.c_int]
         lib.oracle_attn_fwd_rows.argtypes = [_dp, _dp, _dp, _i64p, _i64, _dp, _dp, _i64, _i64,
                                              _i64, _i64, _i64, _i64, ctypes.c_double,
                                              ctypes.c_int, ctypes.c_int]
@@ -61,7 +64,7 @@ def load(path: str | None = None):
                                           _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                           ctypes.c_int]
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_probs,
-                  lib.oracle_attn_paged):
+                  lib.oracle_attn_paged, lib.oracle_attn_fwd_window):
             f.restype = ctypes.c_int
         _libs[key] = lib
     return _libs[key]
@@ -99,6 +102,22 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, threads: int | None = 
                                  Lq, Lk, D, float(scale), int(bool(causal)),
                                  threads or default_threads())
     _check(rc, "attn_fwd")
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def attn_fwd_window(q, k, v, scale: float, causal: bool = False, window=(-1, -1),
+                    threads: int | None = None, lib=None):
+    """Sliding-window attention, window = (left, right) with -1 = unbounded on that side."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    out = np.zeros((B, Hq, Lq, D), np.float64)
+    lse = np.zeros((B, Hq, Lq), np.float64)
+    rc = (lib or load()).oracle_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                                B, Hq, Hkv, Lq, Lk, D, float(scale),
+                                                int(bool(causal)), int(window[0]), int(window[1]),
+                                                threads or default_threads())
+    _check(rc, "attn_fwd_window")
     return torch.from_numpy(out), torch.from_numpy(lse)
 
 

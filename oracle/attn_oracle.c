@@ -20,6 +20,11 @@
  *    (hermes-agent-app.ru), Scenario 2, step 2. Reading taken: key j is
  *    visible to query i iff j <= i + (Lk - Lq) (bottom-right alignment; the
  *    same as top-left when Lq == Lk, and a single decode query sees all keys).
+ *  - Sliding-window (local) attention, window_size = (left, right): same page,
+ *    Scenario 2, step 3 ("attention only to a window of tokens before/after").
+ *    Reading taken: with i' = i + (Lk - Lq), key j is visible iff
+ *    i' - left <= j <= i' + right, a negative bound meaning unbounded on that
+ *    side; causal=True caps the right side at i' (right = 0).
  *  - Fewer K/V heads than query heads (multi-query / grouped-query): same
  *    page, Scenario 2, step 3. Reading taken: consecutive query heads share a
  *    K/V head, h_kv = h_q / (H_q / H_kv).
@@ -54,19 +59,19 @@
  * One query row of attention.
  *   qi      : the query row, D values
  *   K, V    : Lk rows of D values each
- *   n_vis   : keys 0 .. n_vis-1 are visible (the causal mask is a prefix)
+ *   lo, hi  : keys lo .. hi-1 are visible (the mask is one contiguous range)
  *   s       : scratch for the Lk scores
  *   o       : output row, D values
  *   lse     : output log-sum-exp of the row (may be NULL)
  *   p_out   : if not NULL, receives the Lk softmax probabilities
  */
 static void attention_row(const double* qi, const double* K, const double* V,
-                          int64_t Lk, int64_t n_vis, int64_t D, double scale,
+                          int64_t Lk, int64_t lo, int64_t hi, int64_t D, double scale,
                           double* s, double* o, double* lse, double* p_out) {
     int64_t j, d;
     /* Scores: scale * (q_i . k_j); masked keys get -inf. */
     for (j = 0; j < Lk; ++j) {
-        if (j < n_vis) {
+        if (j >= lo && j < hi) {
             double dot = 0.0;
             for (d = 0; d < D; ++d) dot += qi[d] * K[j * D + d];
             s[j] = scale * dot;
@@ -97,13 +102,21 @@ static void attention_row(const double* qi, const double* K, const double* V,
     if (lse) *lse = m + log(l);
 }
 
-/* Number of keys visible to query row i (keys form a prefix). */
-static int64_t visible_keys(int64_t i, int64_t Lq, int64_t Lk, int causal) {
-    if (!causal) return Lk;
-    int64_t last = i + (Lk - Lq); /* highest visible key index */
-    if (last < 0) return 0;
-    if (last >= Lk) return Lk;
-    return last + 1;
+/*
+ * Keys visible to query row i: [*lo, *hi). With i' = i + (Lk - Lq) (bottom-right
+ * alignment), key j is visible iff i' - left <= j <= i' + right; a negative left or
+ * right leaves that side unbounded, and causal sets right = 0.
+ */
+static void visible_range(int64_t i, int64_t Lq, int64_t Lk, int causal, int64_t left,
+                          int64_t right, int64_t* lo, int64_t* hi) {
+    int64_t last = i + (Lk - Lq); /* i' */
+    int64_t a = 0, b = Lk;
+    if (causal) right = 0;
+    if (left >= 0 && last - left > a) a = last - left;
+    if (right >= 0 && last + right + 1 < b) b = last + right + 1;
+    if (b < a) b = a;
+    *lo = a;
+    *hi = b;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -116,6 +129,7 @@ typedef struct {
     int64_t B, Hq, Hkv, Lq, Lk, D;
     double scale;
     int causal;
+    int64_t win_left, win_right; /* -1: unbounded */
     const int64_t* rows; /* NULL: every row, in order */
     int64_t n_rows;
     int64_t next; /* shared work counter */
@@ -146,8 +160,9 @@ static void* dense_worker(void* arg) {
         double* o = J->out + r * J->D;
         double* lse = J->lse ? J->lse + r : NULL;
         double* p = J->probs ? J->probs + r * J->Lk : NULL;
-        attention_row(qi, K, V, J->Lk, visible_keys(i, J->Lq, J->Lk, J->causal), J->D,
-                      J->scale, s, o, lse, p);
+        int64_t lo, hi;
+        visible_range(i, J->Lq, J->Lk, J->causal, J->win_left, J->win_right, &lo, &hi);
+        attention_row(qi, K, V, J->Lk, lo, hi, J->D, J->scale, s, o, lse, p);
     }
     free(s);
     return NULL;
@@ -182,7 +197,20 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o
                     int64_t D, double scale, int causal, int nthreads) {
     int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
     if (rc) return rc;
-    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal, -1, -1,
+                   NULL, B * Hq * Lq, 0, ORACLE_OK};
+    return run_dense(&J, nthreads);
+}
+
+/* Sliding-window attention: as oracle_attn_fwd with window (left, right), -1 = unbounded. */
+int oracle_attn_fwd_window(const double* q, const double* k, const double* v, double* out,
+                           double* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq,
+                           int64_t Lk, int64_t D, double scale, int causal, int64_t left,
+                           int64_t right, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    if (left < -1 || right < -1) return ORACLE_ERR_ARG;
+    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal, left, right,
                    NULL, B * Hq * Lq, 0, ORACLE_OK};
     return run_dense(&J, nthreads);
 }
@@ -199,7 +227,7 @@ int oracle_attn_fwd_rows(const double* q, const double* k, const double* v,
     if (rc) return rc;
     for (int64_t r = 0; r < n_rows; ++r)
         if (rows[r] < 0 || rows[r] >= B * Hq * Lq) return ORACLE_ERR_INDEX;
-    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+    dense_job J = {q, k, v, out, lse, NULL, B, Hq, Hkv, Lq, Lk, D, scale, causal, -1, -1,
                    rows, n_rows, 0, ORACLE_OK};
     return run_dense(&J, nthreads);
 }
@@ -212,7 +240,7 @@ int oracle_attn_probs(const double* q, const double* k, const double* v, double*
     if (rc) return rc;
     double* out = (double*)malloc(sizeof(double) * (size_t)(B * Hq * Lq * D + 1));
     if (!out) return ORACLE_ERR_NOMEM;
-    dense_job J = {q, k, v, out, NULL, probs, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+    dense_job J = {q, k, v, out, NULL, probs, B, Hq, Hkv, Lq, Lk, D, scale, causal, -1, -1,
                    NULL, B * Hq * Lq, 0, ORACLE_OK};
     rc = run_dense(&J, 1);
     free(out);
@@ -266,7 +294,7 @@ static void* paged_worker(void* arg) {
         for (int64_t g = 0; g < group; ++g) {
             int64_t h = hkv * group + g;
             const double* qi = J->q + (sq * J->Hq + h) * J->D;
-            attention_row(qi, Kd, Vd, len, len, J->D, J->scale, s,
+            attention_row(qi, Kd, Vd, len, 0, len, J->D, J->scale, s,
                           J->out + (sq * J->Hq + h) * J->D,
                           J->lse ? J->lse + sq * J->Hq + h : NULL, NULL);
         }

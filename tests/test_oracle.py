@@ -35,9 +35,11 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_examples
 
 
 # --------------------------------------------------------------------------- helpers
-def brute_attention(q, k, v, scale, causal):
+def brute_attention(q, k, v, scale, causal, window=(-1, -1)):
     """Independent brute force: exact decimal products, Decimal exp/ln at 60 digits,
-    no max subtraction. Returns (out, lse) as float64 arrays."""
+    no max subtraction. Returns (out, lse) as float64 arrays. window = (left, right):
+    query i (shifted to i + Lk - Lq) sees keys within left before and right after it,
+    -1 meaning unbounded; causal caps the right side at 0."""
     q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
@@ -51,7 +53,10 @@ def brute_attention(q, k, v, scale, causal):
             for h in range(Hq):
                 hk = h // G
                 for i in range(Lq):
-                    vis = [j for j in range(Lk) if (not causal) or j <= i + Lk - Lq]
+                    ii = i + Lk - Lq
+                    right = 0 if causal else window[1]
+                    vis = [j for j in range(Lk)
+                           if (right < 0 or j <= ii + right) and (window[0] < 0 or j >= ii - window[0])]
                     if not vis:
                         lse[b, h, i] = -math.inf
                         continue
@@ -322,10 +327,44 @@ def pin_split_combine(lib=None):
         close(lse, l)
 
 
+def pin_window(lib=None):
+    # brute force with windows, GQA, Lq != Lk
+    cases = [
+        (1, 2, 1, 6, 6, 4, False, (1, 1), 0.6),
+        (1, 2, 2, 5, 9, 3, True, (2, -1), 0.8),     # causal + left window
+        (2, 2, 1, 7, 4, 2, False, (0, 2), 1.1),     # Lq > Lk: some rows see nothing
+        (1, 1, 1, 8, 8, 5, False, (-1, 1), 0.4),
+    ]
+    for n, (B, Hq, Hkv, Lq, Lk, D, causal, win, scale) in enumerate(cases):
+        q = rand((B, Hq, Lq, D), 400 + n)
+        k = rand((B, Hkv, Lk, D), 410 + n)
+        v = rand((B, Hkv, Lk, D), 420 + n)
+        o_ref, l_ref = brute_attention(q, k, v, scale, causal, win)
+        o, l = oracle.attn_fwd_window(q, k, v, scale, causal, win, lib=lib)
+        close(o, o_ref)
+        close(l, l_ref)
+    # exact equivalences with the unwindowed definition
+    q = rand((1, 2, 9, 4), 430)
+    k = rand((1, 2, 13, 4), 431)
+    v = rand((1, 2, 13, 4), 432)
+    full = oracle.attn_fwd(q, k, v, 0.5, False, lib=lib)
+    causal = oracle.attn_fwd(q, k, v, 0.5, True, lib=lib)
+    for got, want in [(oracle.attn_fwd_window(q, k, v, 0.5, False, (-1, -1), lib=lib), full),
+                      (oracle.attn_fwd_window(q, k, v, 0.5, False, (-1, 0), lib=lib), causal),
+                      (oracle.attn_fwd_window(q, k, v, 0.5, True, (-1, 7), lib=lib), causal),
+                      (oracle.attn_fwd_window(q, k, v, 0.5, False, (50, 50), lib=lib), full)]:
+        assert torch.equal(got[0], want[0]) and torch.equal(got[1], want[1])
+    # window (0, 0): row i attends to key i + (Lk - Lq) alone
+    o, l = oracle.attn_fwd_window(q, k, v, 0.5, False, (0, 0), lib=lib)
+    for i in range(9):
+        close(o[0, :, i], v[0, :, i + 4])
+        close(l[0, :, i], 0.5 * np.einsum("hd,hd->h", q[0, :, i], k[0, :, i + 4]))
+
+
 PINS = [pin_brute_force, pin_golden, pin_probability_rows, pin_constant_values,
         pin_identical_keys, pin_argmax_limit, pin_causal_row0, pin_shift_invariance,
         pin_permutation_equivariance, pin_gqa_equals_repeat, pin_paged_equals_dense,
-        pin_fully_masked_rows, pin_online_softmax, pin_split_combine]
+        pin_fully_masked_rows, pin_online_softmax, pin_split_combine, pin_window]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -373,6 +412,10 @@ MUTANTS = {
     "paged_row_index": ("t % J->block_size) * J->D;", "t / J->block_size) * J->D;"),
     "paged_head_index": ("((phys * J->Hkv + hkv) * J->block_size", "((phys * J->Hkv) * J->block_size"),
     "paged_len_plus_one": ("int64_t len = J->seq_lens[sq];", "int64_t len = J->seq_lens[sq] + 1;"),
+    "window_left_off_by_one": ("if (left >= 0 && last - left > a) a = last - left;",
+                               "if (left >= 0 && last - left + 1 > a) a = last - left + 1;"),
+    "window_right_off_by_one": ("if (right >= 0 && last + right + 1 < b) b = last + right + 1;",
+                                "if (right >= 0 && last + right < b) b = last + right;"),
     "masked_row_nan": ("if (m == -INFINITY) { /* no visible key */",
                        "if (0) { /* no visible key */"),
 }
