@@ -97,6 +97,22 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
                        int causal, attn_dtype_t dtype, void* stream);
 
 /*
+ * attn_fwd_window -- attn_fwd with a sliding window (local attention): the
+ * window_size = (left, right) of the "Flash Attention" skill page (hermes-agent-app.ru),
+ * Scenario 2, step 3. With i' = i + (Lk - Lq), key j is visible to query i iff
+ * i' - window_left <= j <= i' + window_right; -1 leaves that side unbounded, and
+ * causal != 0 caps the right side at i' (window_right is then ignored). Key tiles
+ * outside every row's window are never loaded. (-1, -1) without causal is attn_fwd's
+ * full attention; (-1, -1) with causal is attn_fwd's causal attention. Rows that see no
+ * key get O = 0 and lse = -inf. Returns ATTN_ERR_INVALID for a bound below -1; all
+ * other arguments as attn_fwd.
+ */
+attn_status_t attn_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse,
+                              int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                              int causal, int window_left, int window_right, attn_dtype_t dtype,
+                              void* stream);
+
+/*
  * attn_paged_workspace_size -- bytes of device workspace attn_fwd_paged needs
  * for these sizes (0 when no sequence is ever split). The workspace holds the
  * partial results of the split-KV chunks (one per CTA of the balanced

@@ -31,8 +31,8 @@ def declared_functions():
 
 def test_header_declares_expected_entry_points():
     names = declared_functions()
-    for n in ("attn_fwd", "attn_fwd_paged", "attn_paged_workspace_size", "attn_error_string",
-              "attn_get_device_status"):
+    for n in ("attn_fwd", "attn_fwd_window", "attn_fwd_paged", "attn_paged_workspace_size",
+              "attn_error_string", "attn_get_device_status"):
         assert n in names
 
 
@@ -122,6 +122,18 @@ def test_attn_fwd_paged_validation(name, kw, code):
                                   a["lse"], a["S"], a["Hq"], a["Hkv"], a["D"], a["MB"], a["NB"],
                                   a["scale"], a["dtype"], a["ws"], a["ws_n"], a["stream"])
     assert rc == code, (rc, ta.STATUS.get(rc))
+
+
+def test_attn_fwd_window_validation():
+    lib = ta.load()
+    a = fwd_args()
+    base = (a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"],
+            a["D"], a["scale"], 0)
+    assert lib.attn_fwd_window(*base, -2, 5, 0, None) == -1       # bound below -1
+    assert lib.attn_fwd_window(*base, 5, -3, 0, None) == -1
+    bad = list(base)
+    bad[10] = 96                                                   # D: unsupported
+    assert lib.attn_fwd_window(*bad, 4, 4, 0, None) == -2
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")

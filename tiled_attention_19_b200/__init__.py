@@ -31,6 +31,8 @@ STATUS = {
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _i,
+                             _vp]),
     "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                             _i, _vp, _sz, _vp]),
@@ -101,9 +103,12 @@ def _check(rc: int, what: str) -> None:
 
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: float | None = None, out: torch.Tensor | None = None,
-        lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
-    """softmax(q k^T * scale [+ causal mask]) v.  q [B,Hq,Lq,D]; k, v [B,Hkv,Lk,D].
-    Returns (out [B,Hq,Lq,D], lse [B,Hq,Lq] fp32 or None). scale defaults to 1/sqrt(D)."""
+        lse: torch.Tensor | None = None, return_lse: bool = True, stream=None,
+        window: tuple | None = None):
+    """softmax(q k^T * scale [+ causal / window mask]) v.  q [B,Hq,Lq,D]; k, v [B,Hkv,Lk,D].
+    window = (left, right) restricts query i to keys i'-left..i'+right (i' = i + Lk - Lq,
+    -1 = unbounded). Returns (out [B,Hq,Lq,D], lse [B,Hq,Lq] fp32 or None). scale defaults
+    to 1/sqrt(D)."""
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
@@ -116,10 +121,16 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    rc = load().attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
-                         _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv, Lq, Lk, D,
-                         float(scale), int(bool(causal)), _dtype_code(q.dtype), _stream(stream))
-    _check(rc, "attn_fwd")
+    args = (_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+            _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv, Lq, Lk, D, float(scale),
+            int(bool(causal)))
+    if window is None:
+        rc = load().attn_fwd(*args, _dtype_code(q.dtype), _stream(stream))
+        _check(rc, "attn_fwd")
+    else:
+        rc = load().attn_fwd_window(*args, int(window[0]), int(window[1]), _dtype_code(q.dtype),
+                                    _stream(stream))
+        _check(rc, "attn_fwd_window")
     return out, lse
 
 

@@ -85,10 +85,10 @@ bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L,
 }
 
 // ------------------------------------------------------------------ launchers
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool MASKED>
 attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const PrefillArgs& args, int planes, cudaStream_t stream) {
-    auto kern = attn::prefill_fwd_kernel<D, BF16, CAUSAL>;
+    auto kern = attn::prefill_fwd_kernel<D, BF16, MASKED>;
     constexpr int smem = PrefillCfg<D>::kSmemBytes;
     static std::once_flag once;
     static attn_status_t setup = ATTN_OK;
@@ -118,10 +118,10 @@ attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const
 }
 
 template <int D, bool BF16>
-attn_status_t dispatch_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+attn_status_t dispatch_masked(bool masked, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv, const PrefillArgs& args, int planes,
                               cudaStream_t stream) {
-    return causal ? launch_prefill<D, BF16, true>(tq, tk, tv, args, planes, stream)
+    return masked ? launch_prefill<D, BF16, true>(tq, tk, tv, args, planes, stream)
                   : launch_prefill<D, BF16, false>(tq, tk, tv, args, planes, stream);
 }
 
@@ -155,13 +155,11 @@ attn_status_t launch_paged(const CUtensorMap& tk, const CUtensorMap& tv, const P
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-}  // namespace
-
-extern "C" {
-
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
-                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,
-                       attn_dtype_t dtype, void* stream_) {
+// Dense forward with a band of visible keys: key j is visible to query i iff
+// i' - left <= j <= i' + right with i' = i + (Lk - Lq); -1 leaves a side unbounded.
+attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int left,
+                       int right, attn_dtype_t dtype, void* stream_) {
     if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
     if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -209,14 +207,36 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     args.Lq = Lq;
     args.Lk = Lk;
     args.n_q_blocks = (Lq + 2 * attn::kBM - 1) / (2 * attn::kBM);
+    args.win_left = left;
+    args.win_right = right;
     args.scale_log2 = scale * attn::kLog2e;
     const int planes = static_cast<int>(planes_q);
-    const bool c = causal != 0;
+    const bool m = left >= 0 || right >= 0;
     if (D == 64)
-        return bf16 ? dispatch_causal<64, true>(c, tq, tk, tv, args, planes, stream)
-                    : dispatch_causal<64, false>(c, tq, tk, tv, args, planes, stream);
-    return bf16 ? dispatch_causal<128, true>(c, tq, tk, tv, args, planes, stream)
-                : dispatch_causal<128, false>(c, tq, tk, tv, args, planes, stream);
+        return bf16 ? dispatch_masked<64, true>(m, tq, tk, tv, args, planes, stream)
+                    : dispatch_masked<64, false>(m, tq, tk, tv, args, planes, stream);
+    return bf16 ? dispatch_masked<128, true>(m, tq, tk, tv, args, planes, stream)
+                : dispatch_masked<128, false>(m, tq, tk, tv, args, planes, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,
+                       attn_dtype_t dtype, void* stream) {
+    return fwd_band(q, k, v, out, lse, B, H_q, H_kv, Lq, Lk, D, scale, -1, causal ? 0 : -1, dtype,
+                    stream);
+}
+
+attn_status_t attn_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse,
+                              int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                              int causal, int window_left, int window_right, attn_dtype_t dtype,
+                              void* stream) {
+    if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID;
+    return fwd_band(q, k, v, out, lse, B, H_q, H_kv, Lq, Lk, D, scale, window_left,
+                    causal ? 0 : window_right, dtype, stream);
 }
 
 size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D, int max_blocks_per_seq,

@@ -32,11 +32,13 @@
 // the 384 x 168 = 64,512 the CTA is launched with.
 // TMEM (512 columns): S0/P0 at 0, S1/P1 at 128, O0 at 256, O1 at 384.
 //
-// Causal masking (the "Flash Attention" skill page, Scenario 2 step 2: causal=True
-// for autoregressive models): key j is visible to query i iff j <= i + (Lk - Lq).
-// Key tiles entirely above the diagonal of a query tile's last row are skipped for
-// that tile (never loaded if no tile of the CTA needs them); the mask itself is
-// applied only on tiles that cross the diagonal or the ragged end of the keys.
+// Band masks (the "Flash Attention" skill page, Scenario 2: causal=True for
+// autoregressive models, step 2, and sliding-window attention window_size=(left,
+// right), step 3): with i' = i + (Lk - Lq), key j is visible to query i iff
+// i' - left <= j <= i' + right (a negative bound is unbounded; causal is right = 0).
+// Each query tile walks only the key tiles that hold a visible key of one of its rows;
+// the element mask is applied only on tiles that cross a band edge or the ragged end
+// of the keys. Without a band (MASKED = false) only the ragged end is masked.
 //
 // Lazy rescaling: the reference max m of a row moves only when a tile's maximum
 // exceeds it by more than 8 (log2 units). Until then p = 2^(s*c - m) <= 2^8, which
@@ -83,22 +85,44 @@ struct PrefillArgs {
     float* lse;
     int Hq, Hkv, group, Lq, Lk;
     int n_q_blocks;    // ceil(Lq / 256): CTAs along the query axis
+    int win_left;      // band: keys >= i' - win_left visible (-1: unbounded)
+    int win_right;     // band: keys <= i' + win_right visible (-1: unbounded; causal: 0)
     float scale_log2;  // scale * log2(e)
 };
 
-// Number of key tiles query rows [row0, row0 + 128) need (0 if every row is fully masked).
-template <bool CAUSAL>
-__device__ __forceinline__ int key_tiles_for(int row0, int Lq, int Lk) {
-    int n = (Lk + kBN - 1) / kBN;
-    if (CAUSAL) {
-        const int last_row = min(row0 + kBM - 1, Lq - 1);
-        const int max_key = last_row + (Lk - Lq);
-        n = max_key < 0 ? 0 : min(n, max_key / kBN + 1);
+// First and one-past-last visible key of query row i (empty if hi <= lo).
+template <bool MASKED>
+__device__ __forceinline__ void row_keys(int i, const PrefillArgs& a, int& lo, int& hi) {
+    lo = 0;
+    hi = a.Lk;
+    if (MASKED) {
+        const int ii = i + (a.Lk - a.Lq);
+        if (a.win_left >= 0) lo = max(0, ii - a.win_left);
+        if (a.win_right >= 0) hi = min(a.Lk, ii + a.win_right + 1);
     }
-    return n;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+// Key tiles [t0, t1) holding a visible key of some row in [row0, row0 + 128).
+template <bool MASKED>
+__device__ __forceinline__ void key_tiles_for(int row0, const PrefillArgs& a, int& t0, int& t1) {
+    const int r1 = min(row0 + kBM - 1, a.Lq - 1);
+    if (r1 < row0) {  // no real rows (past Lq)
+        t0 = t1 = 0;
+        return;
+    }
+    int lo0, hi0, lo1, hi1;
+    row_keys<MASKED>(row0, a, lo0, hi0);  // band edges grow with the row
+    row_keys<MASKED>(r1, a, lo1, hi1);
+    const int first = lo0, last = hi1 - 1;
+    if (last < first || last < 0 || first >= a.Lk) {
+        t0 = t1 = 0;
+        return;
+    }
+    t0 = first / kBN;
+    t1 = last / kBN + 1;
+}
+
+template <int D, bool BF16, bool MASKED>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -139,9 +163,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int b = bh / args.Hq;
     const int kv_plane = b * args.Hkv + h / args.group;  // grouped-query head mapping
     const int q0 = qb * 2 * kBM;
-    const int diag = args.Lk - args.Lq;                  // causal: key j visible iff j <= i + diag
-    const int n0 = key_tiles_for<CAUSAL>(q0, args.Lq, args.Lk);
-    const int n1 = key_tiles_for<CAUSAL>(q0 + kBM, args.Lq, args.Lk);  // n0 <= n1
+    // key-tile ranges of the two query tiles and of the CTA (their union, no gaps:
+    // the band edges are monotone in the row)
+    int a0, b0, a1, b1;
+    key_tiles_for<MASKED>(q0, args, a0, b0);
+    key_tiles_for<MASKED>(q0 + kBM, args, a1, b1);
+    const int jlo = (b0 > a0) ? a0 : a1;
+    const int jhi = max(b0, b1);
+    const int n_all = (b1 > a1 || b0 > a0) ? jhi - jlo : 0;  // key tiles this CTA loads
 
     if (threadIdx.x == 0) {
         mbar_init(bar(Q_FULL), 1);
@@ -184,42 +213,43 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     } else if (warp == 8) {
         // ------------------------------------------------------------ producer
         regs_decrease<kOtherRegs>();
-        if (lane == 0 && n1 > 0) {
+        if (lane == 0 && n_all > 0) {
             mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
                 tma_load_3d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, bh);
                 tma_load_3d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, bh);
             }
-            for (int j = 0; j < n1; ++j) {
-                const int sk = j % NK, sv = j % NV;
-                if (j >= NK && !wait_phase(bar(K_EMPTY + sk), ((j / NK) - 1) & 1, abort_flag)) break;
+            for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile jlo + n
+                const int j = jlo + n;
+                const int sk = n % NK, sv = n % NV;
+                if (n >= NK && !wait_phase(bar(K_EMPTY + sk), ((n / NK) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
                     tma_load_3d(sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
                                 bar(K_FULL + sk), c * 64, j * kBN, kv_plane);
-                k_issued = j + 1;
-                if (j >= NV && !wait_phase(bar(V_EMPTY + sv), ((j / NV) - 1) & 1, abort_flag)) break;
+                k_issued = n + 1;
+                if (n >= NV && !wait_phase(bar(V_EMPTY + sv), ((n / NV) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(V_FULL + sv), Cfg::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
                     tma_load_3d(sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
                                 bar(V_FULL + sv), c * 64, j * kBN, kv_plane);
-                v_issued = j + 1;
+                v_issued = n + 1;
             }
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
         regs_decrease<kOtherRegs>();
-        if (lane == 0 && n1 > 0) {
+        if (lane == 0 && n_all > 0) {
             constexpr uint32_t kIdescQK = idesc_f16(BF16, kBM, kBN, false, false);
             constexpr uint32_t kIdescPV = idesc_f16(BF16, kBM, D, false, true);
             mma_started = true;
             // S_t = Q_t K_j^T into TMEM columns s_col (K-major operands: 16 elements =
             // 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
-            auto issue_s = [&](uint32_t sQ, uint32_t s_col, int j) {
-                const uint32_t sK = sK0 + (j % NK) * Cfg::kTileBytes;
+            auto issue_s = [&](uint32_t sQ, uint32_t s_col, int n) {
+                const uint32_t sK = sK0 + (n % NK) * Cfg::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
@@ -229,49 +259,55 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             };
             // O_t += P_t V_j: P from TMEM (16 keys = 8 columns per step), V MN-major
             // (16 keys = two 8-row swizzle atoms, 2048 bytes; D chunks 16 KiB apart).
-            auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int j) {
-                const uint32_t sV = sV0 + (j % NV) * Cfg::kTileBytes;
+            // `first` starts the accumulator (the query tile's first key tile).
+            auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int n, bool first) {
+                const uint32_t sV = sV0 + (n % NV) * Cfg::kTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
                     mma_ts(tmem + o_col, tmem + p_col + ks * 8,
                            sdesc_sw128(sV + ks * 2048, Cfg::kChunkBytes, 1024), kIdescPV,
-                           (j > 0 || ks > 0) ? 1u : 0u);
+                           (!first || ks > 0) ? 1u : 0u);
             };
             bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
-            for (int j = 0; ok && j <= n1; ++j) {
-                const int i = j - 1;  // the tile whose P·V is due
+            for (int n = 0; ok && n <= n_all; ++n) {
+                const int j = jlo + n;  // the key tile whose S is due
+                const int i = j - 1;    // the key tile whose P·V is due
                 // PV0_{j-1}
-                if (i >= 0 && i < n0) {
-                    ok = wait_phase(bar(P_FULL + 0), i & 1, abort_flag) &&
-                         wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                if (n >= 1 && i >= a0 && i < b0) {
+                    ok = wait_phase(bar(P_FULL + 0), (i - a0) & 1, abort_flag) &&
+                         wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(Cfg::kSCol0, Cfg::kOCol0, i);
-                    if (i == n0 - 1) mma_commit(bar(O_DONE + 0));
+                    issue_pv(Cfg::kSCol0, Cfg::kOCol0, n - 1, i == a0);
+                    if (i == b0 - 1) mma_commit(bar(O_DONE + 0));
                 }
-                if (j < n1) {
-                    ok = wait_phase(bar(K_FULL + j % NK), (j / NK) & 1, abort_flag);
+                if (n < n_all) {
+                    ok = wait_phase(bar(K_FULL + n % NK), (n / NK) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    if (j < n0) {
-                        issue_s(sQ0, Cfg::kSCol0, j);
+                    if (j >= a0 && j < b0) {
+                        issue_s(sQ0, Cfg::kSCol0, n);
                         mma_commit(bar(S_FULL + 0));
                     }
                 }
                 // PV1_{j-1}
-                if (i >= 0) {
-                    ok = wait_phase(bar(P_FULL + 1), i & 1, abort_flag) &&
-                         wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(Cfg::kSCol1, Cfg::kOCol1, i);
-                    mma_commit(bar(V_EMPTY + i % NV));
-                    if (i == n1 - 1) mma_commit(bar(O_DONE + 1));
+                if (n >= 1) {
+                    if (i >= a1 && i < b1) {
+                        ok = wait_phase(bar(P_FULL + 1), (i - a1) & 1, abort_flag) &&
+                             wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(Cfg::kSCol1, Cfg::kOCol1, n - 1, i == a1);
+                        if (i == b1 - 1) mma_commit(bar(O_DONE + 1));
+                    }
+                    mma_commit(bar(V_EMPTY + (n - 1) % NV));  // V_{j-1} is no longer needed
                 }
-                if (j < n1) {
-                    issue_s(sQ1, Cfg::kSCol1, j);
-                    mma_commit(bar(S_FULL + 1));
-                    mma_commit(bar(K_EMPTY + j % NK));
+                if (n < n_all) {
+                    if (j >= a1 && j < b1) {
+                        issue_s(sQ1, Cfg::kSCol1, n);
+                        mma_commit(bar(S_FULL + 1));
+                    }
+                    mma_commit(bar(K_EMPTY + n % NK));  // K_j is no longer needed
                 }
             }
         }
@@ -281,19 +317,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int tile = warp >> 2;          // 0: Q0 (warps 0-3), 1: Q1 (warps 4-7)
         const int t = threadIdx.x & 127;     // query row within the tile == TMEM lane
         const int row = q0 + tile * kBM + t;
-        const int n_kv = tile == 0 ? n0 : n1;
+        const int ta = tile == 0 ? a0 : a1;  // this query tile's key tiles [ta, tb)
+        const int tb = tile == 0 ? b0 : b1;
+        const int n_kv = tb > ta ? tb - ta : 0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t s_col = tile == 0 ? Cfg::kSCol0 : Cfg::kSCol1;
         const uint32_t o_col = tile == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
         const float c = args.scale_log2;
-        const int row_limit = CAUSAL ? min(args.Lk, row + diag + 1) : args.Lk;
+        int row_lo, row_hi;  // this row's visible keys [row_lo, row_hi)
+        row_keys<MASKED>(row, args, row_lo, row_hi);
+        // band edges of the tile: the largest first key and the smallest end
         const int tile_row0 = q0 + tile * kBM;
+        int edge_lo, edge_hi, unused;
+        row_keys<MASKED>(min(tile_row0 + kBM - 1, args.Lq - 1), args, edge_lo, unused);
+        row_keys<MASKED>(tile_row0, args, unused, edge_hi);
         float m_ref = -INFINITY;  // reference max, log2 units
         float l = 0.f;            // running sum of 2^(s*c - m_ref)
         bool ok = true;
 
-        for (int j = 0; j < n_kv; ++j) {
-            const bool w = wait_phase(bar(S_FULL + tile), j & 1, abort_flag);
+        for (int jj = 0; jj < n_kv; ++jj) {
+            const int j = ta + jj;  // key tile
+            const bool w = wait_phase(bar(S_FULL + tile), jj & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[kBN];
@@ -307,12 +351,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int x = 0; x < kBN; ++x) s[x] = __uint_as_float(sr[x]);
 
             const int kbase = j * kBN;
-            const bool need_mask =
-                (kbase + kBN > args.Lk) || (CAUSAL && kbase + kBN - 1 > tile_row0 + diag);
+            const bool need_mask = (kbase + kBN > args.Lk) ||
+                                   (MASKED && (kbase < edge_lo || kbase + kBN > edge_hi));
             if (need_mask) {
-                const int lim = row_limit - kbase;
+                const int lo = row_lo - kbase, hi = row_hi - kbase;
 #pragma unroll
-                for (int x = 0; x < kBN; ++x) s[x] = (x < lim) ? s[x] : -INFINITY;
+                for (int x = 0; x < kBN; ++x) s[x] = (x >= lo && x < hi) ? s[x] : -INFINITY;
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
@@ -343,7 +387,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             // Correct O when the reference max moved. S_t(j) completing implies the
             // P·V of tile j-1 (issued before it) has completed too.
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 32) {
                     uint32_t o[32];
@@ -406,7 +450,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (*abort_flag) {
         // Nothing may still be writing into this CTA's shared or tensor memory when
         // it exits: wait for the loads already issued and for every MMA issued.
-        if (warp == 8 && lane == 0 && n1 > 0) {
+        if (warp == 8 && lane == 0 && n_all > 0) {
             drain_phase(bar(Q_FULL), 0);
             for (int j = max(0, k_issued - NK); j < k_issued; ++j)
                 drain_phase(bar(K_FULL + j % NK), (j / NK) & 1);
