@@ -157,7 +157,7 @@ def job_rate(work_per_rank: float, ms_max_over_ranks: float, ws: int, unit_scale
 class Workload:
     """Device copies of the step's inputs (rotated) and its outputs."""
 
-    def __init__(self, device, copies: int):
+    def __init__(self, device, copies: int, window=None):
         self.device = device
         xp = inputs.make(PREFILL)
         xd = inputs.make(DECODE)
@@ -173,8 +173,21 @@ class Workload:
         self.prefill_bytes = inputs.dense_bytes(PREFILL)
         self.d_out = torch.empty_like(self.dc[0]["q"])
         self.d_lse = torch.empty(DECODE.num_seqs, DECODE.Hq, device=device)
-        self.prefill_flops = PREFILL.flops()
+        self.prefill_flops = PREFILL.flops() if window is None else windowed_flops(PREFILL, window)
         self.decode_bytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
+
+
+def windowed_flops(spec, window) -> float:
+    """4 * D FLOPs per visible (query row, key) pair, counted exactly for a band:
+    row i (i' = i + Lk - Lq) sees keys max(0, i'-left) .. min(Lk-1, i'+right)."""
+    left, right = window
+    if spec.causal:
+        right = 0
+    i = torch.arange(spec.Lq, dtype=torch.int64) + (spec.Lk - spec.Lq)
+    lo = torch.clamp(i - left, min=0) if left >= 0 else torch.zeros_like(i)
+    hi = torch.clamp(i + right, max=spec.Lk - 1) if right >= 0 else torch.full_like(i, spec.Lk - 1)
+    pairs = int(torch.clamp(hi - lo + 1, min=0).sum())
+    return 4.0 * spec.D * spec.B * spec.Hq * pairs
 
 
 def run_ours(args, ws, rank, local):
@@ -183,7 +196,7 @@ def run_ours(args, ws, rank, local):
     torch.cuda.set_device(device)
     ta.load()
     copies = args.copies  # default 4: 4 x 96 MiB prefill inputs, 4 x 67 MB decode pool > L2
-    w = Workload(device, copies)
+    w = Workload(device, copies, args.window)
     do_pre = args.only in ("both", "prefill")
     do_dec = args.only in ("both", "decode")
     stream = torch.cuda.current_stream()
@@ -197,7 +210,7 @@ def run_ours(args, ws, rank, local):
             ev[0].record(stream)
         if do_pre:
             ta.fwd(p["q"], p["k"], p["v"], causal=PREFILL.causal, scale=PREFILL.scale, out=w.p_out,
-                   lse=w.p_lse, stream=stream)
+                   lse=w.p_lse, stream=stream, window=args.window)
         if ev is not None:
             ev[1].record(stream)
         if do_dec:
@@ -237,7 +250,7 @@ def run_ours(args, ws, rank, local):
     dec_avg = reduce_max(sum(dec_ms) / len(dec_ms), ws, device)
 
     if args.e2e:
-        e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)))
+        e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)), window=args.window)
     else:
         e2e = {"prefill_ms": float("nan"), "decode_ms": float("nan"), "h2d_bytes": 0,
                "d2h_bytes": 0}
@@ -285,6 +298,7 @@ def run_ours(args, ws, rank, local):
                   f"{w.p_copies} x {sum(v.numel() * v.element_size() for v in w.xp_host.values()) / 1e6:.1f} MB, "
                   f"decode pool {copies} x 67 MB",
             "parallelism": f"replicas x{ws} (independent problems per GPU)",
+            "window": args.window,
         },
         "roofline": {
             "kernel": f"prefill_fwd_kernel<{PREFILL.D},{'bf16' if PREFILL.dtype == torch.bfloat16 else 'f16'},"
@@ -328,7 +342,7 @@ def run_ours(args, ws, rank, local):
     return line
 
 
-def measure_e2e(w, ta, stream, device, steps: int):
+def measure_e2e(w, ta, stream, device, steps: int, window=None):
     """Same metric through the public API with host buffers: H2D of the step's inputs
     from pinned memory, the call, D2H of its outputs, all inside the timed region."""
     hp = {k: v.pin_memory() for k, v in w.xp_host.items()}
@@ -350,7 +364,7 @@ def measure_e2e(w, ta, stream, device, steps: int):
         for k in dp:
             dp[k].copy_(hp[k], non_blocking=True)
         ta.fwd(dp["q"], dp["k"], dp["v"], causal=PREFILL.causal, scale=PREFILL.scale, out=w.p_out,
-               lse=w.p_lse, stream=stream)
+               lse=w.p_lse, stream=stream, window=window)
         op.copy_(w.p_out, non_blocking=True)
         lp.copy_(w.p_lse, non_blocking=True)
         e[1].record(stream)
@@ -468,6 +482,8 @@ def main(argv=None):
                     help="run one kernel of the step only (profiling runs)")
     ap.add_argument("--copies", type=int, default=4,
                     help="device copies of the inputs the steps rotate over (4 > L2)")
+    ap.add_argument("--window", type=int, nargs=2, metavar=("LEFT", "RIGHT"), default=None,
+                    help="sliding window of the prefill call (-1 = unbounded side)")
     ap.add_argument("--prefill-workload", default=PREFILL_DEFAULT,
                     choices=[n for n, w in inputs.WORKLOADS.items() if w.kind == "dense"],
                     help="dense workload of the prefill call (default: the long causal prefill)")

@@ -85,10 +85,10 @@ bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L,
 }
 
 // ------------------------------------------------------------------ launchers
-template <int D, bool BF16, bool MASKED>
+template <int D, bool BF16, int MASK>
 attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const PrefillArgs& args, int planes, cudaStream_t stream) {
-    auto kern = attn::prefill_fwd_kernel<D, BF16, MASKED>;
+    auto kern = attn::prefill_fwd_kernel<D, BF16, MASK>;
     constexpr int smem = PrefillCfg<D>::kSmemBytes;
     static std::once_flag once;
     static attn_status_t setup = ATTN_OK;
@@ -118,11 +118,14 @@ attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const
 }
 
 template <int D, bool BF16>
-attn_status_t dispatch_masked(bool masked, const CUtensorMap& tq, const CUtensorMap& tk,
-                              const CUtensorMap& tv, const PrefillArgs& args, int planes,
-                              cudaStream_t stream) {
-    return masked ? launch_prefill<D, BF16, true>(tq, tk, tv, args, planes, stream)
-                  : launch_prefill<D, BF16, false>(tq, tk, tv, args, planes, stream);
+attn_status_t dispatch_mask(int mask, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const PrefillArgs& args, int planes,
+                            cudaStream_t stream) {
+    if (mask == attn::kMaskCausal)
+        return launch_prefill<D, BF16, attn::kMaskCausal>(tq, tk, tv, args, planes, stream);
+    if (mask == attn::kMaskWindow)
+        return launch_prefill<D, BF16, attn::kMaskWindow>(tq, tk, tv, args, planes, stream);
+    return launch_prefill<D, BF16, attn::kMaskNone>(tq, tk, tv, args, planes, stream);
 }
 
 // 2-D view (D, rows) of a paged cache [num_blocks, H_kv, 16, D]: one row per token of
@@ -211,12 +214,14 @@ attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, f
     args.win_right = right;
     args.scale_log2 = scale * attn::kLog2e;
     const int planes = static_cast<int>(planes_q);
-    const bool m = left >= 0 || right >= 0;
+    const int m = (left < 0 && right < 0) ? attn::kMaskNone
+                  : (left < 0 && right == 0) ? attn::kMaskCausal
+                                             : attn::kMaskWindow;
     if (D == 64)
-        return bf16 ? dispatch_masked<64, true>(m, tq, tk, tv, args, planes, stream)
-                    : dispatch_masked<64, false>(m, tq, tk, tv, args, planes, stream);
-    return bf16 ? dispatch_masked<128, true>(m, tq, tk, tv, args, planes, stream)
-                : dispatch_masked<128, false>(m, tq, tk, tv, args, planes, stream);
+        return bf16 ? dispatch_mask<64, true>(m, tq, tk, tv, args, planes, stream)
+                    : dispatch_mask<64, false>(m, tq, tk, tv, args, planes, stream);
+    return bf16 ? dispatch_mask<128, true>(m, tq, tk, tv, args, planes, stream)
+                : dispatch_mask<128, false>(m, tq, tk, tv, args, planes, stream);
 }
 
 }  // namespace

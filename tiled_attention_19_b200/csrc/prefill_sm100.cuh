@@ -38,7 +38,8 @@
 // i' - left <= j <= i' + right (a negative bound is unbounded; causal is right = 0).
 // Each query tile walks only the key tiles that hold a visible key of one of its rows;
 // the element mask is applied only on tiles that cross a band edge or the ragged end
-// of the keys. Without a band (MASKED = false) only the ragged end is masked.
+// of the keys. Without a band (kMaskNone) only the ragged end is masked; causal and
+// general windows are separate instantiations (kMaskCausal, kMaskWindow).
 //
 // Lazy rescaling: the reference max m of a row moves only when a tile's maximum
 // exceeds it by more than 8 (log2 units). Until then p = 2^(s*c - m) <= 2^8, which
@@ -90,29 +91,44 @@ struct PrefillArgs {
     float scale_log2;  // scale * log2(e)
 };
 
+// Mask modes, fixed at compile time so the common cases carry no window arithmetic.
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
+
 // First and one-past-last visible key of query row i (empty if hi <= lo).
-template <bool MASKED>
+template <int MASK>
 __device__ __forceinline__ void row_keys(int i, const PrefillArgs& a, int& lo, int& hi) {
     lo = 0;
     hi = a.Lk;
-    if (MASKED) {
+    if (MASK == kMaskCausal) {
+        hi = min(a.Lk, i + (a.Lk - a.Lq) + 1);
+    } else if (MASK == kMaskWindow) {
         const int ii = i + (a.Lk - a.Lq);
         if (a.win_left >= 0) lo = max(0, ii - a.win_left);
         if (a.win_right >= 0) hi = min(a.Lk, ii + a.win_right + 1);
     }
 }
 
-// Key tiles [t0, t1) holding a visible key of some row in [row0, row0 + 128).
-template <bool MASKED>
+// Key tiles [t0, t1) holding a visible key of some row in [row0, row0 + 128). Without
+// a window a tile past Lq takes the tiles of the last real row (t0 = 0 and t1 never
+// below the previous tile's), which the two-tile issue loop relies on; with a window it
+// is empty.
+template <int MASK>
 __device__ __forceinline__ void key_tiles_for(int row0, const PrefillArgs& a, int& t0, int& t1) {
     const int r1 = min(row0 + kBM - 1, a.Lq - 1);
+    if (MASK != kMaskWindow) {
+        int lo, hi;
+        row_keys<MASK>(r1, a, lo, hi);
+        t0 = 0;
+        t1 = hi <= 0 ? 0 : (hi - 1) / kBN + 1;
+        return;
+    }
     if (r1 < row0) {  // no real rows (past Lq)
         t0 = t1 = 0;
         return;
     }
     int lo0, hi0, lo1, hi1;
-    row_keys<MASKED>(row0, a, lo0, hi0);  // band edges grow with the row
-    row_keys<MASKED>(r1, a, lo1, hi1);
+    row_keys<MASK>(row0, a, lo0, hi0);  // band edges grow with the row
+    row_keys<MASK>(r1, a, lo1, hi1);
     const int first = lo0, last = hi1 - 1;
     if (last < first || last < 0 || first >= a.Lk) {
         t0 = t1 = 0;
@@ -122,7 +138,7 @@ __device__ __forceinline__ void key_tiles_for(int row0, const PrefillArgs& a, in
     t1 = last / kBN + 1;
 }
 
-template <int D, bool BF16, bool MASKED>
+template <int D, bool BF16, int MASK>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -165,10 +181,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int q0 = qb * 2 * kBM;
     // key-tile ranges of the two query tiles and of the CTA (their union, no gaps:
     // the band edges are monotone in the row)
-    int a0, b0, a1, b1;
-    key_tiles_for<MASKED>(q0, args, a0, b0);
-    key_tiles_for<MASKED>(q0 + kBM, args, a1, b1);
-    const int jlo = (b0 > a0) ? a0 : a1;
+    int a0 = 0, b0, a1 = 0, b1;
+    if constexpr (MASK == kMaskWindow) {
+        key_tiles_for<MASK>(q0, args, a0, b0);
+        key_tiles_for<MASK>(q0 + kBM, args, a1, b1);
+    } else {  // every query tile starts at key tile 0
+        int unused;
+        key_tiles_for<MASK>(q0, args, unused, b0);
+        key_tiles_for<MASK>(q0 + kBM, args, unused, b1);
+    }
+    const int jlo = (MASK != kMaskWindow) ? 0 : ((b0 > a0) ? a0 : a1);
     const int jhi = max(b0, b1);
     const int n_all = (b1 > a1 || b0 > a0) ? jhi - jlo : 0;  // key tiles this CTA loads
 
@@ -269,45 +291,86 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                            (!first || ks > 0) ? 1u : 0u);
             };
             bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
-            for (int n = 0; ok && n <= n_all; ++n) {
-                const int j = jlo + n;  // the key tile whose S is due
-                const int i = j - 1;    // the key tile whose P·V is due
-                // PV0_{j-1}
-                if (n >= 1 && i >= a0 && i < b0) {
-                    ok = wait_phase(bar(P_FULL + 0), (i - a0) & 1, abort_flag) &&
-                         wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(Cfg::kSCol0, Cfg::kOCol0, n - 1, i == a0);
-                    if (i == b0 - 1) mma_commit(bar(O_DONE + 0));
-                }
-                if (n < n_all) {
-                    ok = wait_phase(bar(K_FULL + n % NK), (n / NK) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (j >= a0 && j < b0) {
-                        issue_s(sQ0, Cfg::kSCol0, n);
-                        mma_commit(bar(S_FULL + 0));
+            if constexpr (MASK != kMaskWindow) {
+                // Query tiles both start at key tile 0: n0 = b0 <= n1 = b1.
+                const int n0 = b0, n1 = b1;
+                for (int j = 0; ok && j <= n1; ++j) {
+                    const int i = j - 1;  // the key tile whose P·V is due
+                    // PV0_{j-1}
+                    if (i >= 0 && i < n0) {
+                        ok = wait_phase(bar(P_FULL + 0), i & 1, abort_flag) &&
+                             wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(Cfg::kSCol0, Cfg::kOCol0, i, i == 0);
+                        if (i == n0 - 1) mma_commit(bar(O_DONE + 0));
+                    }
+                    if (j < n1) {
+                        ok = wait_phase(bar(K_FULL + j % NK), (j / NK) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (j < n0) {
+                            issue_s(sQ0, Cfg::kSCol0, j);
+                            mma_commit(bar(S_FULL + 0));
+                        }
+                    }
+                    // PV1_{j-1}
+                    if (i >= 0) {
+                        ok = wait_phase(bar(P_FULL + 1), i & 1, abort_flag) &&
+                             wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(Cfg::kSCol1, Cfg::kOCol1, i, i == 0);
+                        mma_commit(bar(V_EMPTY + i % NV));
+                        if (i == n1 - 1) mma_commit(bar(O_DONE + 1));
+                    }
+                    if (j < n1) {
+                        issue_s(sQ1, Cfg::kSCol1, j);
+                        mma_commit(bar(S_FULL + 1));
+                        mma_commit(bar(K_EMPTY + j % NK));
                     }
                 }
-                // PV1_{j-1}
-                if (n >= 1) {
-                    if (i >= a1 && i < b1) {
-                        ok = wait_phase(bar(P_FULL + 1), (i - a1) & 1, abort_flag) &&
+            } else {
+                for (int n = 0; ok && n <= n_all; ++n) {
+                    const int j = jlo + n;  // the key tile whose S is due
+                    const int i = j - 1;    // the key tile whose P·V is due
+                    // PV0_{j-1}
+                    if (n >= 1 && i >= a0 && i < b0) {
+                        ok = wait_phase(bar(P_FULL + 0), (i - a0) & 1, abort_flag) &&
                              wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_pv(Cfg::kSCol1, Cfg::kOCol1, n - 1, i == a1);
-                        if (i == b1 - 1) mma_commit(bar(O_DONE + 1));
+                        issue_pv(Cfg::kSCol0, Cfg::kOCol0, n - 1, i == a0);
+                        if (i == b0 - 1) mma_commit(bar(O_DONE + 0));
                     }
-                    mma_commit(bar(V_EMPTY + (n - 1) % NV));  // V_{j-1} is no longer needed
-                }
-                if (n < n_all) {
-                    if (j >= a1 && j < b1) {
-                        issue_s(sQ1, Cfg::kSCol1, n);
-                        mma_commit(bar(S_FULL + 1));
+                    if (n < n_all) {
+                        ok = wait_phase(bar(K_FULL + n % NK), (n / NK) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (j >= a0 && j < b0) {
+                            issue_s(sQ0, Cfg::kSCol0, n);
+                            mma_commit(bar(S_FULL + 0));
+                        }
                     }
-                    mma_commit(bar(K_EMPTY + n % NK));  // K_j is no longer needed
+                    // PV1_{j-1}
+                    if (n >= 1) {
+                        if (i >= a1 && i < b1) {
+                            ok = wait_phase(bar(P_FULL + 1), (i - a1) & 1, abort_flag) &&
+                                 wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(Cfg::kSCol1, Cfg::kOCol1, n - 1, i == a1);
+                            if (i == b1 - 1) mma_commit(bar(O_DONE + 1));
+                        }
+                        mma_commit(bar(V_EMPTY + (n - 1) % NV));  // V_{j-1} is no longer needed
+                    }
+                    if (n < n_all) {
+                        if (j >= a1 && j < b1) {
+                            issue_s(sQ1, Cfg::kSCol1, n);
+                            mma_commit(bar(S_FULL + 1));
+                        }
+                        mma_commit(bar(K_EMPTY + n % NK));  // K_j is no longer needed
+                    }
                 }
             }
         }
@@ -325,12 +388,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t o_col = tile == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
         const float c = args.scale_log2;
         int row_lo, row_hi;  // this row's visible keys [row_lo, row_hi)
-        row_keys<MASKED>(row, args, row_lo, row_hi);
+        row_keys<MASK>(row, args, row_lo, row_hi);
         // band edges of the tile: the largest first key and the smallest end
         const int tile_row0 = q0 + tile * kBM;
         int edge_lo, edge_hi, unused;
-        row_keys<MASKED>(min(tile_row0 + kBM - 1, args.Lq - 1), args, edge_lo, unused);
-        row_keys<MASKED>(tile_row0, args, unused, edge_hi);
+        row_keys<MASK>(min(tile_row0 + kBM - 1, args.Lq - 1), args, edge_lo, unused);
+        row_keys<MASK>(tile_row0, args, unused, edge_hi);
         float m_ref = -INFINITY;  // reference max, log2 units
         float l = 0.f;            // running sum of 2^(s*c - m_ref)
         bool ok = true;
@@ -352,11 +415,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
             const int kbase = j * kBN;
             const bool need_mask = (kbase + kBN > args.Lk) ||
-                                   (MASKED && (kbase < edge_lo || kbase + kBN > edge_hi));
+                                   (MASK != kMaskNone && (kbase < edge_lo || kbase + kBN > edge_hi));
             if (need_mask) {
                 const int lo = row_lo - kbase, hi = row_hi - kbase;
+                if (MASK == kMaskWindow) {
 #pragma unroll
-                for (int x = 0; x < kBN; ++x) s[x] = (x >= lo && x < hi) ? s[x] : -INFINITY;
+                    for (int x = 0; x < kBN; ++x) s[x] = (x >= lo && x < hi) ? s[x] : -INFINITY;
+                } else {
+#pragma unroll
+                    for (int x = 0; x < kBN; ++x) s[x] = (x < hi) ? s[x] : -INFINITY;
+                }
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
