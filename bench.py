@@ -63,8 +63,8 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    kernel sources as they are now (else None)."""
+    """DRAM bytes per launch from the committed ncu summary, keyed by workload name, if
+    it was taken on the kernel sources as they are now (else empty)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return {}
@@ -310,7 +310,7 @@ def run_ours(args, ws, rank, local):
             "unit": "TFLOP/s",
             "frac": r2(per_gpu_tflops and per_gpu_tflops / pk_t, 4),
             "frac_of_burst_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops"], 4),
-            "traffic": traffic.get("prefill"),
+            "traffic": None if args.window else traffic.get(PREFILL.name),
             "avg_launch_ms": round(pre_avg, 5),
         },
         "paged_decode": {
@@ -322,7 +322,7 @@ def run_ours(args, ws, rank, local):
             "peak": pk_h,
             "peak_source": f"{peaks_src} hbm_gbs",
             "frac": r2(per_gpu_gbs and per_gpu_gbs / pk_h, 4),
-            "traffic": traffic.get("decode"),
+            "traffic": traffic.get(DECODE.name),
             "avg_launch_ms": round(dec_avg, 5),
         },
         "e2e": {
