@@ -3,8 +3,9 @@
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
 import this package. The library under ``tiled_attention_19_b200`` never does, and the
 two share no code. The arithmetic lives in ``attn_oracle.c``: a literal, row-by-row
-statement of softmax(Q K^T * scale [+ causal mask]) V in double precision (see that
-file's header for the definition each step follows). This module only builds the
+statement of softmax(Q K^T * scale [+ causal mask]) V in double precision, and of
+its gradients by the chain rule (see that file's header for the definition each step
+follows). This module only builds the
 shared object and marshals arrays into it.
 
 Inputs may be any floating torch tensor (or numpy array); they are widened to fp64
@@ -63,8 +64,18 @@ def load(path: str | None = None):
         lib.oracle_attn_paged.argtypes = [_dp, _dp, _dp, _i32p, _i32p, _i64, _dp, _dp, _i64,
                                           _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                           ctypes.c_int]
+        lib.oracle_attn_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64,
+                                        _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64,
+                                        _i64, ctypes.c_int]
+        lib.oracle_attn_bwd_dq_rows.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _i64, _i64,
+                                                _i64, _i64, _i64, _i64, ctypes.c_double,
+                                                ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_bwd_dkv_keys.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _dp, _i64,
+                                                 _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                                 ctypes.c_int, ctypes.c_int]
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_probs,
-                  lib.oracle_attn_paged, lib.oracle_attn_fwd_window):
+                  lib.oracle_attn_paged, lib.oracle_attn_fwd_window, lib.oracle_attn_bwd,
+                  lib.oracle_attn_bwd_dq_rows, lib.oracle_attn_bwd_dkv_keys):
             f.restype = ctypes.c_int
         _libs[key] = lib
     return _libs[key]
@@ -168,3 +179,55 @@ def attn_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float,
                                    MB, NB, float(scale), threads or default_threads())
     _check(rc, "attn_paged")
     return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def attn_bwd(q, k, v, dout, scale: float, causal: bool = False, window=(-1, -1),
+             threads: int | None = None, lib=None):
+    """Gradients of attention given dout = dLoss/dO: (dq[B,Hq,Lq,D], dk[B,Hkv,Lk,D],
+    dv[B,Hkv,Lk,D]) in fp64. window = (left, right) as in attn_fwd_window."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    assert k.shape == (B, Hkv, Lk, D) and v.shape == k.shape and do.shape == q.shape
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    rc = (lib or load()).oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
+                                         _ptr(dv), B, Hq, Hkv, Lq, Lk, D, float(scale),
+                                         int(bool(causal)), int(window[0]), int(window[1]),
+                                         threads or default_threads())
+    _check(rc, "attn_bwd")
+    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+
+
+def attn_bwd_dq_rows(q, k, v, dout, rows, scale: float, causal: bool = False,
+                     threads: int | None = None, lib=None):
+    """dq of selected query rows, ids (b*Hq + h)*Lq + i -> dq[n, D] fp64."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+    dq = np.zeros((rows.shape[0], D), np.float64)
+    rc = (lib or load()).oracle_attn_bwd_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do),
+                                                 _ptr(rows, _i64p), rows.shape[0], _ptr(dq), B,
+                                                 Hq, Hkv, Lq, Lk, D, float(scale),
+                                                 int(bool(causal)), threads or default_threads())
+    _check(rc, "attn_bwd_dq_rows")
+    return torch.from_numpy(dq)
+
+
+def attn_bwd_dkv_keys(q, k, v, dout, keys, scale: float, causal: bool = False,
+                      threads: int | None = None, lib=None):
+    """dk, dv of selected keys, ids (b*Hkv + h_kv)*Lk + j -> (dk[n, D], dv[n, D]) fp64."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64).reshape(-1))
+    dk = np.zeros((keys.shape[0], D), np.float64)
+    dv = np.zeros((keys.shape[0], D), np.float64)
+    rc = (lib or load()).oracle_attn_bwd_dkv_keys(_ptr(q), _ptr(k), _ptr(v), _ptr(do),
+                                                  _ptr(keys, _i64p), keys.shape[0], _ptr(dk),
+                                                  _ptr(dv), B, Hq, Hkv, Lq, Lk, D, float(scale),
+                                                  int(bool(causal)), threads or default_threads())
+    _check(rc, "attn_bwd_dkv_keys")
+    return torch.from_numpy(dk), torch.from_numpy(dv)

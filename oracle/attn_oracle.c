@@ -34,6 +34,17 @@
  *    masked scores of the row.
  *  - A row with no visible key has no softmax. Reading taken: O = 0 and
  *    lse = -inf.
+ *  - Backward pass: only the normalisation statistics are kept from the forward
+ *    pass, and the attention tiles are recomputed during backpropagation: "Self-
+ *    attention, CUDA kernels and FlashAttention", section 3 (recomputation). The
+ *    pages print no gradient formulas. What the backward pass computes is the
+ *    gradient of a scalar loss through the section 1 definition, given dO =
+ *    dLoss/dO. Here it is written out by the chain rule for one query row i:
+ *    P_ij are the row's probabilities, dV_j += P_ij dO_i, dP_ij = dO_i . v_j,
+ *    delta_i = sum_j P_ij dP_ij (the softmax Jacobian applied to the row of dP),
+ *    dS_ij = P_ij (dP_ij - delta_i), dQ_i = scale sum_j dS_ij k_j and dK_j +=
+ *    scale dS_ij q_i. Masked keys have P_ij = 0 and so take no part. Grouped K/V
+ *    heads collect the gradients of every query head that reads them.
  *  - Paged KV cache: storage in fixed-size blocks plus a table from logical
  *    position to physical block, resolved for every position inside the
  *    attention: "Fast attention kernels and operator fusion" (the-ai.news),
@@ -331,4 +342,311 @@ int oracle_attn_paged(const double* q, const double* k_cache, const double* v_ca
     paged_worker(&J);
     for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
     return J.status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass: gradients of a scalar loss through dense attention.       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One query row of the backward pass. Recomputes the row's probabilities p (with
+ * attention_row), then the row of dP_ij = do_i . v_j over the visible keys, the
+ * row's delta = sum_j P_ij dP_ij, and dS_ij = P_ij (dP_ij - delta).
+ *   dqi      : receives dQ_i = scale sum_j dS_ij k_j (may be NULL)
+ *   dK, dV   : Lk rows each, accumulated into (may be NULL):
+ *              dV_j += P_ij do_i and dK_j += scale dS_ij q_i
+ *   s, p, ds : scratch of Lk values; o : scratch of D values
+ * Returns the row's delta (0 for a row with no visible key).
+ */
+static double backward_row(const double* qi, const double* doi, const double* K,
+                           const double* V, int64_t Lk, int64_t lo, int64_t hi, int64_t D,
+                           double scale, double* s, double* p, double* ds, double* o,
+                           double* dqi, double* dK, double* dV) {
+    int64_t j, d;
+    attention_row(qi, K, V, Lk, lo, hi, D, scale, s, o, NULL, p);
+    /* dP_ij = do_i . v_j (kept in ds for now) and delta = sum_j P_ij dP_ij. */
+    double delta = 0.0;
+    for (j = lo; j < hi; ++j) {
+        double dot = 0.0;
+        for (d = 0; d < D; ++d) dot += doi[d] * V[j * D + d];
+        ds[j] = dot;
+        delta += p[j] * dot;
+    }
+    /* dS_ij = P_ij (dP_ij - delta). */
+    for (j = lo; j < hi; ++j) ds[j] = p[j] * (ds[j] - delta);
+    if (dqi) {
+        for (d = 0; d < D; ++d) dqi[d] = 0.0;
+        for (j = lo; j < hi; ++j)
+            for (d = 0; d < D; ++d) dqi[d] += ds[j] * K[j * D + d];
+        for (d = 0; d < D; ++d) dqi[d] *= scale;
+    }
+    for (j = lo; j < hi; ++j) {
+        if (dV)
+            for (d = 0; d < D; ++d) dV[j * D + d] += p[j] * doi[d];
+        if (dK)
+            for (d = 0; d < D; ++d) dK[j * D + d] += scale * ds[j] * qi[d];
+    }
+    return delta;
+}
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *dq, *dk, *dv;
+    int64_t B, Hq, Hkv, Lq, Lk, D;
+    double scale;
+    int causal;
+    int64_t win_left, win_right;
+    int64_t next; /* shared work counter over (b, h_kv) units */
+    int status;
+} bwd_job;
+
+/* One unit = one (batch, K/V head): every query row of every query head that reads it,
+ * so the unit's dK and dV rows are written by this worker alone. */
+static void* bwd_worker(void* arg) {
+    bwd_job* J = (bwd_job*)arg;
+    const size_t n = (size_t)(J->Lk > 0 ? J->Lk : 1);
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* p = (double*)malloc(sizeof(double) * n);
+    double* ds = (double*)malloc(sizeof(double) * n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !p || !ds || !o) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        free(s); free(p); free(ds); free(o);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    for (;;) {
+        int64_t u = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (u >= J->B * J->Hkv) break;
+        const int64_t b = u / J->Hkv, hkv = u % J->Hkv;
+        const double* K = J->k + u * J->Lk * J->D;
+        const double* V = J->v + u * J->Lk * J->D;
+        double* dK = J->dk + u * J->Lk * J->D;
+        double* dV = J->dv + u * J->Lk * J->D;
+        for (int64_t x = 0; x < J->Lk * J->D; ++x) dK[x] = dV[x] = 0.0;
+        for (int64_t g = 0; g < group; ++g) {
+            const int64_t h = hkv * group + g;
+            for (int64_t i = 0; i < J->Lq; ++i) {
+                const int64_t id = (b * J->Hq + h) * J->Lq + i;
+                int64_t lo, hi;
+                visible_range(i, J->Lq, J->Lk, J->causal, J->win_left, J->win_right, &lo, &hi);
+                backward_row(J->q + id * J->D, J->dout + id * J->D, K, V, J->Lk, lo, hi, J->D,
+                             J->scale, s, p, ds, o, J->dq + id * J->D, dK, dV);
+            }
+        }
+    }
+    free(s); free(p); free(ds); free(o);
+    return NULL;
+}
+
+/*
+ * Gradients of attention: dq[B,Hq,Lq,D], dk[B,Hkv,Lk,D], dv[B,Hkv,Lk,D] from
+ * q[B,Hq,Lq,D], k/v[B,Hkv,Lk,D] and dout[B,Hq,Lq,D] = dLoss/dO, with the mask of
+ * oracle_attn_fwd_window (left = right = -1 and causal = 0: no mask).
+ */
+int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
+                    double* dq, double* dk, double* dv, int64_t B, int64_t Hq, int64_t Hkv,
+                    int64_t Lq, int64_t Lk, int64_t D, double scale, int causal, int64_t left,
+                    int64_t right, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    if (left < -1 || right < -1) return ORACLE_ERR_ARG;
+    bwd_job J = {q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Lq, Lk, D, scale, causal, left, right,
+                 0, ORACLE_OK};
+    int64_t units = B * Hkv;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (units < nthreads) nthreads = (int)(units > 0 ? units : 1);
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&tid[started], NULL, bwd_worker, &J) == 0) ++started;
+    bwd_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return J.status;
+}
+
+/* Selected outputs of the backward pass, for problems too large to run whole. */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    int64_t B, Hq, Hkv, Lq, Lk, D;
+    double scale;
+    int causal;
+    const int64_t* ids; /* query rows (dq) or keys (dk, dv), flattened */
+    int64_t n;
+    double *dq, *dk, *dv;  /* n rows of D each */
+    int64_t unit;          /* keys: the (b * Hkv + h_kv) unit the row statistics are for */
+    double *lse, *delta;   /* keys: per query row of the unit's group, [group * Lq] */
+    int64_t next;
+    int status;
+} sel_job;
+
+/* dQ of selected query rows: each row by backward_row on its own. */
+static void* dq_rows_worker(void* arg) {
+    sel_job* J = (sel_job*)arg;
+    const size_t n = (size_t)(J->Lk > 0 ? J->Lk : 1);
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* p = (double*)malloc(sizeof(double) * n);
+    double* ds = (double*)malloc(sizeof(double) * n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !p || !ds || !o) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        free(s); free(p); free(ds); free(o);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    for (;;) {
+        int64_t r = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (r >= J->n) break;
+        const int64_t id = J->ids[r];
+        const int64_t i = id % J->Lq, bh = id / J->Lq;
+        const int64_t h = bh % J->Hq, b = bh / J->Hq;
+        const int64_t u = b * J->Hkv + h / group;
+        int64_t lo, hi;
+        visible_range(i, J->Lq, J->Lk, J->causal, -1, -1, &lo, &hi);
+        backward_row(J->q + id * J->D, J->dout + id * J->D, J->k + u * J->Lk * J->D,
+                     J->v + u * J->Lk * J->D, J->Lk, lo, hi, J->D, J->scale, s, p, ds, o,
+                     J->dq + r * J->D, NULL, NULL);
+    }
+    free(s); free(p); free(ds); free(o);
+    return NULL;
+}
+
+/* Row statistics of one unit's query rows: lse_i (attention_row) and delta_i. */
+static void* unit_stats_worker(void* arg) {
+    sel_job* J = (sel_job*)arg;
+    const size_t n = (size_t)(J->Lk > 0 ? J->Lk : 1);
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* p = (double*)malloc(sizeof(double) * n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !p || !o) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        free(s); free(p); free(o);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    const int64_t b = J->unit / J->Hkv, hkv = J->unit % J->Hkv;
+    const double* K = J->k + J->unit * J->Lk * J->D;
+    const double* V = J->v + J->unit * J->Lk * J->D;
+    for (;;) {
+        int64_t r = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (r >= group * J->Lq) break;
+        const int64_t g = r / J->Lq, i = r % J->Lq;
+        const int64_t id = (b * J->Hq + hkv * group + g) * J->Lq + i;
+        const double* doi = J->dout + id * J->D;
+        int64_t lo, hi;
+        visible_range(i, J->Lq, J->Lk, J->causal, -1, -1, &lo, &hi);
+        attention_row(J->q + id * J->D, K, V, J->Lk, lo, hi, J->D, J->scale, s, o, &J->lse[r], p);
+        double delta = 0.0;
+        for (int64_t j = lo; j < hi; ++j) {
+            double dot = 0.0;
+            for (int64_t d = 0; d < J->D; ++d) dot += doi[d] * V[j * J->D + d];
+            delta += p[j] * dot;
+        }
+        J->delta[r] = delta;
+    }
+    free(s); free(p); free(o);
+    return NULL;
+}
+
+/* dK_j, dV_j of the selected keys of the current unit, as sums over the query rows
+ * that see key j: P_ij = exp(s_ij - lse_i), dS_ij = P_ij (do_i . v_j - delta_i). */
+static void* dkv_keys_worker(void* arg) {
+    sel_job* J = (sel_job*)arg;
+    const int64_t group = J->Hq / J->Hkv;
+    const int64_t b = J->unit / J->Hkv, hkv = J->unit % J->Hkv;
+    const double* K = J->k + J->unit * J->Lk * J->D;
+    const double* V = J->v + J->unit * J->Lk * J->D;
+    for (;;) {
+        int64_t r = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (r >= J->n) break;
+        if (J->ids[r] / J->Lk != J->unit) continue;
+        const int64_t j = J->ids[r] % J->Lk;
+        double* dk = J->dk + r * J->D;
+        double* dv = J->dv + r * J->D;
+        for (int64_t d = 0; d < J->D; ++d) dk[d] = dv[d] = 0.0;
+        for (int64_t g = 0; g < group; ++g) {
+            for (int64_t i = 0; i < J->Lq; ++i) {
+                int64_t lo, hi;
+                visible_range(i, J->Lq, J->Lk, J->causal, -1, -1, &lo, &hi);
+                if (j < lo || j >= hi) continue;
+                const int64_t id = (b * J->Hq + hkv * group + g) * J->Lq + i;
+                const double* qi = J->q + id * J->D;
+                const double* doi = J->dout + id * J->D;
+                double dot = 0.0, dpv = 0.0;
+                for (int64_t d = 0; d < J->D; ++d) dot += qi[d] * K[j * J->D + d];
+                for (int64_t d = 0; d < J->D; ++d) dpv += doi[d] * V[j * J->D + d];
+                const double pij = exp(J->scale * dot - J->lse[g * J->Lq + i]);
+                const double dsij = pij * (dpv - J->delta[g * J->Lq + i]);
+                for (int64_t d = 0; d < J->D; ++d) {
+                    dv[d] += pij * doi[d];
+                    dk[d] += J->scale * dsij * qi[d];
+                }
+            }
+        }
+    }
+    return NULL;
+}
+
+static int run_workers(void* (*fn)(void*), void* job, int64_t work, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (work < nthreads) nthreads = (int)(work > 0 ? work : 1);
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&tid[started], NULL, fn, job) == 0) ++started;
+    fn(job);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return 0;
+}
+
+/* dq[n,D] of the query rows ids[r] = (b*Hq + h)*Lq + i (causal or no mask). */
+int oracle_attn_bwd_dq_rows(const double* q, const double* k, const double* v,
+                            const double* dout, const int64_t* rows, int64_t n, double* dq,
+                            int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
+                            int64_t D, double scale, int causal, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    for (int64_t r = 0; r < n; ++r)
+        if (rows[r] < 0 || rows[r] >= B * Hq * Lq) return ORACLE_ERR_INDEX;
+    sel_job J = {q, k, v, dout, B, Hq, Hkv, Lq, Lk, D, scale, causal, rows, n, dq, NULL, NULL,
+                 0, NULL, NULL, 0, ORACLE_OK};
+    run_workers(dq_rows_worker, &J, n, nthreads);
+    return J.status;
+}
+
+/* dk[n,D], dv[n,D] of the keys ids[r] = (b*Hkv + h_kv)*Lk + j (causal or no mask). */
+int oracle_attn_bwd_dkv_keys(const double* q, const double* k, const double* v,
+                             const double* dout, const int64_t* keys, int64_t n, double* dk,
+                             double* dv, int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq,
+                             int64_t Lk, int64_t D, double scale, int causal, int nthreads) {
+    int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
+    if (rc) return rc;
+    for (int64_t r = 0; r < n; ++r)
+        if (keys[r] < 0 || keys[r] >= B * Hkv * Lk) return ORACLE_ERR_INDEX;
+    const int64_t group = Hq / Hkv;
+    double* lse = (double*)malloc(sizeof(double) * (size_t)(group * Lq + 1));
+    double* delta = (double*)malloc(sizeof(double) * (size_t)(group * Lq + 1));
+    if (!lse || !delta) {
+        free(lse); free(delta);
+        return ORACLE_ERR_NOMEM;
+    }
+    int status = ORACLE_OK;
+    /* One pass per distinct unit among the keys: its rows' statistics, then its keys. */
+    for (int64_t r0 = 0; r0 < n && status == ORACLE_OK; ++r0) {
+        const int64_t unit = keys[r0] / Lk;
+        int seen = 0;
+        for (int64_t r = 0; r < r0; ++r)
+            if (keys[r] / Lk == unit) seen = 1;
+        if (seen) continue;
+        sel_job J = {q, k, v, dout, B, Hq, Hkv, Lq, Lk, D, scale, causal, keys, n, NULL, dk, dv,
+                     unit, lse, delta, 0, ORACLE_OK};
+        run_workers(unit_stats_worker, &J, group * Lq, nthreads);
+        J.next = 0;
+        run_workers(dkv_keys_worker, &J, n, nthreads);
+        status = J.status;
+    }
+    free(lse); free(delta);
+    return status;
 }

@@ -9,6 +9,11 @@
   fully masked rows.
 * Restatements of the algebra the GPU kernels use (a tiled online softmax with lazy
   rescaling, and a split-KV log-sum-exp combine), checked against the oracle.
+* Backward pass: torch autograd in float64 through a plain statement of the forward,
+  central finite differences of the forward oracle, hand-derived examples
+  (tests/golden/backward_closed_form.json), and invariants of the definition (key
+  gradients sum to zero, value gradients sum to dO, identical keys and single-key
+  rows give dQ = 0, grouped heads equal summed repeated heads).
 
 Every ``pin_*`` function takes an optional oracle library handle so that
 test_pins_catch_planted_mistakes can run the same pins on deliberately broken builds
@@ -361,10 +366,155 @@ def pin_window(lib=None):
         close(l[0, :, i], 0.5 * np.einsum("hd,hd->h", q[0, :, i], k[0, :, i + 4]))
 
 
+# ------------------------------------------------------------------- backward pins
+BWD_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "backward_closed_form.json")
+
+
+def autograd_grads(q, k, v, dout, scale, causal, window=(-1, -1)):
+    """Independent derivation: torch autograd in float64 through a plain statement of
+    the forward (einsum scores, a boolean band mask, softmax, einsum with V)."""
+    q, k, v, do = (torch.tensor(np.asarray(t), dtype=torch.float64) for t in (q, k, v, dout))
+    q.requires_grad_(True)
+    k.requires_grad_(True)
+    v.requires_grad_(True)
+    G = q.shape[1] // k.shape[1]
+    K = k.repeat_interleave(G, dim=1)
+    V = v.repeat_interleave(G, dim=1)
+    Lq, Lk = q.shape[2], k.shape[2]
+    i = torch.arange(Lq)[:, None] + (Lk - Lq)
+    j = torch.arange(Lk)[None, :]
+    right = 0 if causal else window[1]
+    vis = torch.ones(Lq, Lk, dtype=torch.bool)
+    if right >= 0:
+        vis &= j <= i + right
+    if window[0] >= 0:
+        vis &= j >= i - window[0]
+    s = torch.einsum("bhid,bhjd->bhij", q, K) * scale
+    s = s.masked_fill(~vis, -math.inf)
+    p = torch.softmax(s, dim=-1).nan_to_num(0.0)  # rows with no visible key: P = 0
+    o = torch.einsum("bhij,bhjd->bhid", p, V)
+    (o * do).sum().backward()
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+BWD_CASES = [
+    # B, Hq, Hkv, Lq, Lk, D, causal, scale, window
+    (1, 1, 1, 1, 1, 1, False, 1.0, (-1, -1)),
+    (1, 2, 1, 5, 6, 4, True, 0.5, (-1, -1)),     # grouped heads, Lq < Lk causal
+    (2, 2, 2, 4, 4, 3, False, 0.7, (-1, -1)),
+    (1, 4, 2, 6, 3, 5, True, 0.35, (-1, -1)),    # Lq > Lk causal: fully masked rows
+    (1, 2, 2, 7, 7, 4, False, 0.6, (2, 1)),      # sliding window
+    (1, 2, 1, 6, 8, 3, True, 0.9, (3, -1)),      # causal window
+]
+
+
+def pin_bwd_autograd(lib=None):
+    for n, (B, Hq, Hkv, Lq, Lk, D, causal, scale, win) in enumerate(BWD_CASES):
+        q = rand((B, Hq, Lq, D), 500 + n)
+        k = rand((B, Hkv, Lk, D), 600 + n)
+        v = rand((B, Hkv, Lk, D), 700 + n)
+        do = rand((B, Hq, Lq, D), 800 + n)
+        ref = autograd_grads(q, k, v, do, scale, causal, win)
+        got = oracle.attn_bwd(q, k, v, do, scale, causal, win, lib=lib)
+        for a, b in zip(got, ref):
+            close(a, b)
+
+
+def pin_bwd_finite_differences(lib=None):
+    """Central differences of Loss = sum(dO * O) through the forward oracle, on every
+    coordinate of q, k and v (h = 1e-6; truncation and rounding stay below 1e-8)."""
+    B, Hq, Hkv, Lq, Lk, D, scale = 1, 2, 1, 4, 5, 3, 0.8
+    for causal, win in ((True, (-1, -1)), (False, (1, 2))):
+        q = rand((B, Hq, Lq, D), 901)
+        k = rand((B, Hkv, Lk, D), 902)
+        v = rand((B, Hkv, Lk, D), 903)
+        do = rand((B, Hq, Lq, D), 904)
+
+        def loss(qq, kk, vv):
+            o, _ = oracle.attn_fwd_window(qq, kk, vv, scale, causal, win, lib=lib)
+            return float((o.numpy() * do).sum())
+
+        got = oracle.attn_bwd(q, k, v, do, scale, causal, win, lib=lib)
+        for which, x in enumerate((q, k, v)):
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += 1e-6
+                xm[idx] -= 1e-6
+                args_p = [q, k, v]
+                args_m = [q, k, v]
+                args_p[which], args_m[which] = xp, xm
+                fd[idx] = (loss(*args_p) - loss(*args_m)) / 2e-6
+            close(got[which].numpy(), fd, 1e-7)
+
+
+def pin_bwd_golden(lib=None):
+    with open(BWD_GOLDEN) as f:
+        examples = json.load(f)["examples"]
+    for ex in examples:
+        got = oracle.attn_bwd(np.array(ex["q"]), np.array(ex["k"]), np.array(ex["v"]),
+                              np.array(ex["dout"]), ex["scale"], ex["causal"], lib=lib)
+        for a, key in zip(got, ("dq", "dk", "dv")):
+            close(a, np.array(ex[key]), 1e-14)
+
+
+def pin_bwd_invariants(lib=None):
+    """Facts fixed by the definition. (1) Scores move by the same amount for every
+    key when a constant vector is added to all keys, which changes nothing, so the
+    key gradients of a head sum to zero. (2) Probability rows sum to 1, so the value
+    gradients sum to the sum of dO over rows that see any key. (3) Identical keys give
+    dQ = 0. (4) A row that sees a single key (causal row 0) has dQ = 0."""
+    q = rand((2, 4, 6, 5), 910)
+    k = rand((2, 2, 6, 5), 911)
+    v = rand((2, 2, 6, 5), 912)
+    do = rand((2, 4, 6, 5), 913)
+    for causal in (False, True):
+        dq, dk, dv = (t.numpy() for t in oracle.attn_bwd(q, k, v, do, 0.7, causal, lib=lib))
+        close(dk.sum(axis=2), np.zeros((2, 2, 5)), 1e-12)
+        close(dv.sum(axis=2), do.reshape(2, 2, 2, 6, 5).sum(axis=(2, 3)), 1e-12)
+        if causal:
+            close(dq[:, :, 0], np.zeros((2, 4, 5)), 1e-12)
+    kk = np.repeat(rand((1, 1, 1, 5), 914), 6, axis=2)
+    dq, _, _ = oracle.attn_bwd(q[:1, :2], kk, v[:1, :1], do[:1, :2], 0.7, False, lib=lib)
+    close(dq.numpy(), np.zeros((1, 2, 6, 5)), 1e-12)
+
+
+def pin_bwd_gqa_equals_repeat(lib=None):
+    q = rand((1, 6, 5, 4), 920)
+    k = rand((1, 2, 7, 4), 921)
+    v = rand((1, 2, 7, 4), 922)
+    do = rand((1, 6, 5, 4), 923)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, 0.5, True, lib=lib)
+    dq2, dk2, dv2 = oracle.attn_bwd(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), do,
+                                    0.5, True, lib=lib)
+    close(dq, dq2)
+    close(dk, dk2.numpy().reshape(1, 2, 3, 7, 4).sum(axis=2))
+    close(dv, dv2.numpy().reshape(1, 2, 3, 7, 4).sum(axis=2))
+
+
+def pin_bwd_selected_outputs(lib=None):
+    """The selected-row and selected-key entry points give the full result's rows."""
+    q = rand((2, 4, 9, 4), 930)
+    k = rand((2, 2, 11, 4), 931)
+    v = rand((2, 2, 11, 4), 932)
+    do = rand((2, 4, 9, 4), 933)
+    for causal in (False, True):
+        dq, dk, dv = oracle.attn_bwd(q, k, v, do, 0.6, causal, lib=lib)
+        rows = np.array([0, 8, 17, 40, 71], np.int64)
+        close(oracle.attn_bwd_dq_rows(q, k, v, do, rows, 0.6, causal, lib=lib),
+              dq.reshape(-1, 4)[rows])
+        keys = np.array([3, 0, 30, 12, 43, 10], np.int64)
+        sk, sv = oracle.attn_bwd_dkv_keys(q, k, v, do, keys, 0.6, causal, lib=lib)
+        close(sk, dk.reshape(-1, 4)[keys])
+        close(sv, dv.reshape(-1, 4)[keys])
+
+
 PINS = [pin_brute_force, pin_golden, pin_probability_rows, pin_constant_values,
         pin_identical_keys, pin_argmax_limit, pin_causal_row0, pin_shift_invariance,
         pin_permutation_equivariance, pin_gqa_equals_repeat, pin_paged_equals_dense,
-        pin_fully_masked_rows, pin_online_softmax, pin_split_combine, pin_window]
+        pin_fully_masked_rows, pin_online_softmax, pin_split_combine, pin_window,
+        pin_bwd_autograd, pin_bwd_finite_differences, pin_bwd_golden, pin_bwd_invariants,
+        pin_bwd_gqa_equals_repeat, pin_bwd_selected_outputs]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -416,33 +566,75 @@ MUTANTS = {
                                "if (left >= 0 && last - left + 1 > a) a = last - left + 1;"),
     "window_right_off_by_one": ("if (right >= 0 && last + right + 1 < b) b = last + right + 1;",
                                 "if (right >= 0 && last + right < b) b = last + right;"),
+    "bwd_delta_dropped": ("for (j = lo; j < hi; ++j) ds[j] = p[j] * (ds[j] - delta);",
+                          "for (j = lo; j < hi; ++j) ds[j] = p[j] * ds[j];"),
+    "bwd_delta_sign": ("for (j = lo; j < hi; ++j) ds[j] = p[j] * (ds[j] - delta);",
+                       "for (j = lo; j < hi; ++j) ds[j] = p[j] * (ds[j] + delta);"),
+    "bwd_dq_scale_dropped": ("for (d = 0; d < D; ++d) dqi[d] *= scale;", ""),
+    "bwd_dk_scale_dropped": ("dK[j * D + d] += scale * ds[j] * qi[d];",
+                             "dK[j * D + d] += ds[j] * qi[d];"),
+    "bwd_dk_uses_keys": ("dK[j * D + d] += scale * ds[j] * qi[d];",
+                         "dK[j * D + d] += scale * ds[j] * K[j * D + d];"),
+    "bwd_dv_uses_ds": ("dV[j * D + d] += p[j] * doi[d];", "dV[j * D + d] += ds[j] * doi[d];"),
+    "bwd_dp_uses_keys": ("for (d = 0; d < D; ++d) dot += doi[d] * V[j * D + d];\n        ds[j] = dot;",
+                         "for (d = 0; d < D; ++d) dot += doi[d] * K[j * D + d];\n        ds[j] = dot;"),
+    "bwd_dq_uses_values": ("for (d = 0; d < D; ++d) dqi[d] += ds[j] * K[j * D + d];",
+                           "for (d = 0; d < D; ++d) dqi[d] += ds[j] * V[j * D + d];"),
+    "bwd_gqa_heads_not_summed": ("for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            for (int64_t i = 0; i < J->Lq; ++i) {",
+                                 "for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            if (g) for (int64_t x = 0; x < J->Lk * J->D; ++x) dK[x] = dV[x] = 0.0;\n            for (int64_t i = 0; i < J->Lq; ++i) {"),
+    "bwd_keys_lse_sign": ("exp(J->scale * dot - J->lse[g * J->Lq + i])",
+                          "exp(J->scale * dot + J->lse[g * J->Lq + i])"),
+    "bwd_keys_delta_dropped": ("pij * (dpv - J->delta[g * J->Lq + i])", "pij * dpv"),
+    "bwd_keys_mask_ignored": ("if (j < lo || j >= hi) continue;\n                const int64_t id",
+                              "const int64_t id"),
     "masked_row_nan": ("if (m == -INFINITY) { /* no visible key */",
                        "if (0) { /* no visible key */"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistakes(name):
-    old, new = MUTANTS[name]
+@pytest.fixture(scope="module")
+def mutant_results():
+    """Builds every mutant and runs the pins on each in a process of its own (a mutant
+    may overrun a buffer; a crash counts as caught). The processes run side by side."""
     src = open(os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")).read()
-    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
-    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    tmp = tempfile.mkdtemp(prefix="oracle_mutants_")
+    results = {}
     try:
-        c = os.path.join(tmp, "m.c")
-        so = os.path.join(tmp, "m.so")
-        with open(c, "w") as f:
-            f.write(src.replace(old, new))
-        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
-                               "-o", so, c, "-lm"])
-        # A mutant may also overrun a buffer, so it runs in a process of its own; a
-        # crash counts as caught.
-        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-        proc = subprocess.run([sys.executable, "-c", _CHILD, so], cwd=root, capture_output=True,
-                              text=True, timeout=300)
-        caught = proc.stdout.split() if proc.returncode == 0 else [f"crash:{proc.returncode}"]
-        assert caught, f"no pin caught the planted mistake {name}"
+        pending = []
+        for name, (old, new) in sorted(MUTANTS.items()):
+            if src.count(old) < 1:
+                results[name] = None
+                continue
+            c = os.path.join(tmp, name + ".c")
+            so = os.path.join(tmp, name + ".so")
+            with open(c, "w") as f:
+                f.write(src.replace(old, new))
+            subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared",
+                                   "-pthread", "-o", so, c, "-lm"])
+            pending.append((name, so))
+        width = max(1, min(8, (os.cpu_count() or 2) // 2))
+        running = []
+        while pending or running:
+            while pending and len(running) < width:
+                name, so = pending.pop(0)
+                proc = subprocess.Popen([sys.executable, "-c", _CHILD, so], cwd=root,
+                                        stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                        text=True)
+                running.append((name, proc))
+            name, proc = running.pop(0)
+            out, _ = proc.communicate(timeout=600)
+            results[name] = out.split() if proc.returncode == 0 else [f"crash:{proc.returncode}"]
     finally:
         shutil.rmtree(tmp, ignore_errors=True)
+    return results
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name, mutant_results):
+    caught = mutant_results[name]
+    assert caught is not None, f"mutation anchor for {name} not found"
+    assert caught, f"no pin caught the planted mistake {name}"
 
 
 _CHILD = """
