@@ -5,7 +5,8 @@
  * What the library computes
  *   O = softmax(Q K^T * scale [+ causal mask]) V, exactly (no approximation of
  *   the softmax), in tiles with an online softmax so the T x T score matrix is
- *   never written to device memory. Definitions:
+ *   never written to device memory; and the gradients of that attention from the
+ *   saved log-sum-exp by recomputing the tiles. Definitions:
  *   - Scores = Q K^T / sqrt(d_k), row-wise softmax, times V, computed per head:
  *     "Self-attention, CUDA kernels and FlashAttention" (russian.itimpress.au),
  *     section 1, the Scores and Attention(Q,K,V) formulas.
@@ -191,6 +192,59 @@ attn_status_t attn_fwd_paged_noalloc(const void* q, const void* k_cache, const v
                                      int H_q, int H_kv, int D, int max_blocks_per_seq,
                                      int num_blocks, float scale, attn_dtype_t dtype,
                                      void* stream);
+
+/*
+ * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs:
+ * 8 * B * H_q * ceil(Lq / 128) * 128 (two fp32 values per query row, rows padded
+ * to a multiple of 128).
+ */
+size_t attn_bwd_workspace_size(int B, int H_q, int Lq);
+
+/*
+ * attn_bwd -- dense attention backward pass: the gradients dQ, dK, dV of a scalar
+ * loss given dO = dLoss/dO, for the attention attn_fwd computed. The attention
+ * tiles are recomputed from q, k, v and the forward pass's lse; the score matrix is
+ * never written to device memory ("Self-attention, CUDA kernels and
+ * FlashAttention" (russian.itimpress.au), section 3: recomputation in the backward
+ * pass from the saved normalisation statistics). With P the attention probabilities
+ * and delta_i = dO_i . O_i:
+ *   dV_j = sum_i P_ij dO_i
+ *   dS_ij = P_ij (dO_i . v_j - delta_i)
+ *   dQ_i = scale sum_j dS_ij k_j
+ *   dK_j = scale sum_i dS_ij q_i
+ * Grouped K/V heads get the sum over the query heads that read them.
+ *
+ *   q, k, v  as attn_fwd (the forward pass's inputs)
+ *   out      [B, H_q, Lq, D] dtype: the forward pass's O
+ *   dout     [B, H_q, Lq, D] dtype: dLoss/dO
+ *   lse      [B, H_q, Lq] fp32: the forward pass's lse (-inf for rows that see no key)
+ *   dq       [B, H_q, Lq, D] dtype, written (every element)
+ *   dk, dv   [B, H_kv, Lk, D] dtype, written (every element)
+ *
+ *   causal and all sizes as attn_fwd. Tensor pointers 16-byte aligned (lse:
+ *   4-byte). workspace: device memory of at least attn_bwd_workspace_size(B, H_q,
+ *   Lq) bytes, 16-byte aligned, no initial contents required; it is overwritten on
+ *   `stream` by every call, so calls that overlap on the device need separate
+ *   workspaces. B == 0 is a no-op (pointers may be NULL); Lq == 0 writes dK = dV = 0;
+ *   Lk == 0 writes dQ = 0. No atomics: results do not depend on scheduling.
+ *   Returns ATTN_ERR_WORKSPACE for a missing or short workspace.
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                       int causal, attn_dtype_t dtype, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * attn_bwd_window -- attn_bwd for attn_fwd_window's sliding-window attention
+ * (window_left, window_right, causal as there); arguments otherwise as attn_bwd.
+ */
+attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                              int causal, int window_left, int window_right,
+                              attn_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                              void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* attn_error_string(attn_status_t status);

@@ -64,15 +64,15 @@ def load(path: str | None = None):
         lib.oracle_attn_paged.argtypes = [_dp, _dp, _dp, _i32p, _i32p, _i64, _dp, _dp, _i64,
                                           _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                           ctypes.c_int]
-        lib.oracle_attn_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64,
-                                        _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _i64,
-                                        _i64, ctypes.c_int]
-        lib.oracle_attn_bwd_dq_rows.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _i64, _i64,
-                                                _i64, _i64, _i64, _i64, ctypes.c_double,
+        lib.oracle_attn_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64,
+                                        _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                        ctypes.c_int, _i64, _i64, ctypes.c_int]
+        lib.oracle_attn_bwd_dq_rows.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _dp, _i64,
+                                                _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                                 ctypes.c_int, ctypes.c_int]
-        lib.oracle_attn_bwd_dkv_keys.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _dp, _i64,
-                                                 _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
-                                                 ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_bwd_dkv_keys.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _dp, _dp,
+                                                 _dp, _i64, _i64, _i64, _i64, _i64, _i64,
+                                                 ctypes.c_double, ctypes.c_int, ctypes.c_int]
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_probs,
                   lib.oracle_attn_paged, lib.oracle_attn_fwd_window, lib.oracle_attn_bwd,
                   lib.oracle_attn_bwd_dq_rows, lib.oracle_attn_bwd_dkv_keys):
@@ -182,52 +182,65 @@ def attn_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float,
 
 
 def attn_bwd(q, k, v, dout, scale: float, causal: bool = False, window=(-1, -1),
-             threads: int | None = None, lib=None):
+             threads: int | None = None, lib=None, sensitivity: bool = False):
     """Gradients of attention given dout = dLoss/dO: (dq[B,Hq,Lq,D], dk[B,Hkv,Lk,D],
-    dv[B,Hkv,Lk,D]) in fp64. window = (left, right) as in attn_fwd_window."""
+    dv[B,Hkv,Lk,D]) in fp64. window = (left, right) as in attn_fwd_window. With
+    sensitivity=True, also (mq, mk, mv): each element's first-order rounding
+    sensitivity (see attn_oracle.c), which the tests' tolerances scale with."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     assert k.shape == (B, Hkv, Lk, D) and v.shape == k.shape and do.shape == q.shape
-    dq = np.zeros_like(q)
-    dk = np.zeros_like(k)
-    dv = np.zeros_like(v)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    m = (np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)) if sensitivity else None
+    mp = (_ptr(m[0]), _ptr(m[1]), _ptr(m[2])) if m else (None, None, None)
     rc = (lib or load()).oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
-                                         _ptr(dv), B, Hq, Hkv, Lq, Lk, D, float(scale),
+                                         _ptr(dv), *mp, B, Hq, Hkv, Lq, Lk, D, float(scale),
                                          int(bool(causal)), int(window[0]), int(window[1]),
                                          threads or default_threads())
     _check(rc, "attn_bwd")
-    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+    g = (torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv))
+    return g + tuple(torch.from_numpy(a) for a in m) if m else g
 
 
 def attn_bwd_dq_rows(q, k, v, dout, rows, scale: float, causal: bool = False,
-                     threads: int | None = None, lib=None):
-    """dq of selected query rows, ids (b*Hq + h)*Lq + i -> dq[n, D] fp64."""
+                     threads: int | None = None, lib=None, sensitivity: bool = False):
+    """dq of selected query rows, ids (b*Hq + h)*Lq + i -> dq[n, D] fp64 (and mq[n, D]
+    with sensitivity=True)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
     dq = np.zeros((rows.shape[0], D), np.float64)
+    mq = np.zeros_like(dq) if sensitivity else None
     rc = (lib or load()).oracle_attn_bwd_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do),
-                                                 _ptr(rows, _i64p), rows.shape[0], _ptr(dq), B,
-                                                 Hq, Hkv, Lq, Lk, D, float(scale),
-                                                 int(bool(causal)), threads or default_threads())
+                                                 _ptr(rows, _i64p), rows.shape[0], _ptr(dq),
+                                                 _ptr(mq) if mq is not None else None, B, Hq,
+                                                 Hkv, Lq, Lk, D, float(scale), int(bool(causal)),
+                                                 threads or default_threads())
     _check(rc, "attn_bwd_dq_rows")
+    if sensitivity:
+        return torch.from_numpy(dq), torch.from_numpy(mq)
     return torch.from_numpy(dq)
 
 
 def attn_bwd_dkv_keys(q, k, v, dout, keys, scale: float, causal: bool = False,
-                      threads: int | None = None, lib=None):
-    """dk, dv of selected keys, ids (b*Hkv + h_kv)*Lk + j -> (dk[n, D], dv[n, D]) fp64."""
+                      threads: int | None = None, lib=None, sensitivity: bool = False):
+    """dk, dv of selected keys, ids (b*Hkv + h_kv)*Lk + j -> (dk[n, D], dv[n, D]) fp64
+    (and mk, mv with sensitivity=True)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64).reshape(-1))
     dk = np.zeros((keys.shape[0], D), np.float64)
     dv = np.zeros((keys.shape[0], D), np.float64)
+    m = (np.zeros_like(dk), np.zeros_like(dv)) if sensitivity else None
     rc = (lib or load()).oracle_attn_bwd_dkv_keys(_ptr(q), _ptr(k), _ptr(v), _ptr(do),
                                                   _ptr(keys, _i64p), keys.shape[0], _ptr(dk),
-                                                  _ptr(dv), B, Hq, Hkv, Lq, Lk, D, float(scale),
-                                                  int(bool(causal)), threads or default_threads())
+                                                  _ptr(dv), _ptr(m[0]) if m else None,
+                                                  _ptr(m[1]) if m else None, B, Hq, Hkv, Lq, Lk,
+                                                  D, float(scale), int(bool(causal)),
+                                                  threads or default_threads())
     _check(rc, "attn_bwd_dkv_keys")
-    return torch.from_numpy(dk), torch.from_numpy(dv)
+    g = (torch.from_numpy(dk), torch.from_numpy(dv))
+    return g + tuple(torch.from_numpy(a) for a in m) if m else g

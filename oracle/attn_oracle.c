@@ -349,19 +349,33 @@ int oracle_attn_paged(const double* q, const double* k_cache, const double* v_ca
 /* ------------------------------------------------------------------------ */
 
 /*
+ * Rounding sensitivity of the gradients, for the tests' tolerances (not part of the
+ * gradient arithmetic). A kernel that rounds P and dS to a 16-bit type (relative
+ * error u each) and computes delta_i from the rounded O (an error of at most
+ * u A_i, A_i = sum_d |do_id o_id|) perturbs dS_ij by at most u (|dS_ij| + P_ij A_i)
+ * and P_ij by u P_ij. To first order the gradient errors are then bounded by u times
+ *   mQ_i = scale sum_j (|dS_ij| + P_ij A_i) |k_j|
+ *   mK_j = scale sum_i (|dS_ij| + P_ij A_i) |q_i|
+ *   mV_j = sum_i P_ij |do_i|        (elementwise over d)
+ */
+
+/*
  * One query row of the backward pass. Recomputes the row's probabilities p (with
  * attention_row), then the row of dP_ij = do_i . v_j over the visible keys, the
  * row's delta = sum_j P_ij dP_ij, and dS_ij = P_ij (dP_ij - delta).
  *   dqi      : receives dQ_i = scale sum_j dS_ij k_j (may be NULL)
  *   dK, dV   : Lk rows each, accumulated into (may be NULL):
  *              dV_j += P_ij do_i and dK_j += scale dS_ij q_i
+ *   mq, mK, mV : the sensitivities mQ_i (D values) and mK_j, mV_j (Lk rows each,
+ *              accumulated into); each may be NULL
  *   s, p, ds : scratch of Lk values; o : scratch of D values
  * Returns the row's delta (0 for a row with no visible key).
  */
 static double backward_row(const double* qi, const double* doi, const double* K,
                            const double* V, int64_t Lk, int64_t lo, int64_t hi, int64_t D,
                            double scale, double* s, double* p, double* ds, double* o,
-                           double* dqi, double* dK, double* dV) {
+                           double* dqi, double* dK, double* dV, double* mq, double* mK,
+                           double* mV) {
     int64_t j, d;
     attention_row(qi, K, V, Lk, lo, hi, D, scale, s, o, NULL, p);
     /* dP_ij = do_i . v_j (kept in ds for now) and delta = sum_j P_ij dP_ij. */
@@ -386,12 +400,27 @@ static double backward_row(const double* qi, const double* doi, const double* K,
         if (dK)
             for (d = 0; d < D; ++d) dK[j * D + d] += scale * ds[j] * qi[d];
     }
+    if (mq || mK || mV) {
+        double A = 0.0;
+        for (d = 0; d < D; ++d) A += fabs(doi[d] * o[d]);
+        if (mq)
+            for (d = 0; d < D; ++d) mq[d] = 0.0;
+        for (j = lo; j < hi; ++j) {
+            const double w = fabs(ds[j]) + p[j] * A;
+            for (d = 0; d < D; ++d) {
+                if (mq) mq[d] += scale * w * fabs(K[j * D + d]);
+                if (mK) mK[j * D + d] += scale * w * fabs(qi[d]);
+                if (mV) mV[j * D + d] += p[j] * fabs(doi[d]);
+            }
+        }
+    }
     return delta;
 }
 
 typedef struct {
     const double *q, *k, *v, *dout;
     double *dq, *dk, *dv;
+    double *mq, *mk, *mv; /* sensitivities, all NULL or all set */
     int64_t B, Hq, Hkv, Lq, Lk, D;
     double scale;
     int causal;
@@ -423,7 +452,11 @@ static void* bwd_worker(void* arg) {
         const double* V = J->v + u * J->Lk * J->D;
         double* dK = J->dk + u * J->Lk * J->D;
         double* dV = J->dv + u * J->Lk * J->D;
+        double* mK = J->mk ? J->mk + u * J->Lk * J->D : NULL;
+        double* mV = J->mv ? J->mv + u * J->Lk * J->D : NULL;
         for (int64_t x = 0; x < J->Lk * J->D; ++x) dK[x] = dV[x] = 0.0;
+        if (mK)
+            for (int64_t x = 0; x < J->Lk * J->D; ++x) mK[x] = mV[x] = 0.0;
         for (int64_t g = 0; g < group; ++g) {
             const int64_t h = hkv * group + g;
             for (int64_t i = 0; i < J->Lq; ++i) {
@@ -431,7 +464,8 @@ static void* bwd_worker(void* arg) {
                 int64_t lo, hi;
                 visible_range(i, J->Lq, J->Lk, J->causal, J->win_left, J->win_right, &lo, &hi);
                 backward_row(J->q + id * J->D, J->dout + id * J->D, K, V, J->Lk, lo, hi, J->D,
-                             J->scale, s, p, ds, o, J->dq + id * J->D, dK, dV);
+                             J->scale, s, p, ds, o, J->dq + id * J->D, dK, dV,
+                             J->mq ? J->mq + id * J->D : NULL, mK, mV);
             }
         }
     }
@@ -442,17 +476,20 @@ static void* bwd_worker(void* arg) {
 /*
  * Gradients of attention: dq[B,Hq,Lq,D], dk[B,Hkv,Lk,D], dv[B,Hkv,Lk,D] from
  * q[B,Hq,Lq,D], k/v[B,Hkv,Lk,D] and dout[B,Hq,Lq,D] = dLoss/dO, with the mask of
- * oracle_attn_fwd_window (left = right = -1 and causal = 0: no mask).
+ * oracle_attn_fwd_window (left = right = -1 and causal = 0: no mask). mq, mk, mv
+ * (shaped like dq, dk, dv) receive the rounding sensitivities when all three are
+ * given; pass NULL for none.
  */
 int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
-                    double* dq, double* dk, double* dv, int64_t B, int64_t Hq, int64_t Hkv,
-                    int64_t Lq, int64_t Lk, int64_t D, double scale, int causal, int64_t left,
-                    int64_t right, int nthreads) {
+                    double* dq, double* dk, double* dv, double* mq, double* mk, double* mv,
+                    int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t D,
+                    double scale, int causal, int64_t left, int64_t right, int nthreads) {
     int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
     if (rc) return rc;
     if (left < -1 || right < -1) return ORACLE_ERR_ARG;
-    bwd_job J = {q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Lq, Lk, D, scale, causal, left, right,
-                 0, ORACLE_OK};
+    if (!mq || !mk || !mv) mq = mk = mv = NULL;
+    bwd_job J = {q, k, v, dout, dq, dk, dv, mq, mk, mv, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+                 left, right, 0, ORACLE_OK};
     int64_t units = B * Hkv;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
@@ -475,8 +512,10 @@ typedef struct {
     const int64_t* ids; /* query rows (dq) or keys (dk, dv), flattened */
     int64_t n;
     double *dq, *dk, *dv;  /* n rows of D each */
+    double *mq, *mk, *mv;  /* their sensitivities (may be NULL) */
     int64_t unit;          /* keys: the (b * Hkv + h_kv) unit the row statistics are for */
-    double *lse, *delta;   /* keys: per query row of the unit's group, [group * Lq] */
+    double *lse, *delta, *absdo; /* keys: per query row of the unit's group, [group * Lq];
+                                    absdo = sum_d |do_id o_id| */
     int64_t next;
     int status;
 } sel_job;
@@ -506,7 +545,7 @@ static void* dq_rows_worker(void* arg) {
         visible_range(i, J->Lq, J->Lk, J->causal, -1, -1, &lo, &hi);
         backward_row(J->q + id * J->D, J->dout + id * J->D, J->k + u * J->Lk * J->D,
                      J->v + u * J->Lk * J->D, J->Lk, lo, hi, J->D, J->scale, s, p, ds, o,
-                     J->dq + r * J->D, NULL, NULL);
+                     J->dq + r * J->D, NULL, NULL, J->mq ? J->mq + r * J->D : NULL, NULL, NULL);
     }
     free(s); free(p); free(ds); free(o);
     return NULL;
@@ -544,6 +583,9 @@ static void* unit_stats_worker(void* arg) {
             delta += p[j] * dot;
         }
         J->delta[r] = delta;
+        double A = 0.0;
+        for (int64_t d = 0; d < J->D; ++d) A += fabs(doi[d] * o[d]);
+        J->absdo[r] = A;
     }
     free(s); free(p); free(o);
     return NULL;
@@ -564,7 +606,11 @@ static void* dkv_keys_worker(void* arg) {
         const int64_t j = J->ids[r] % J->Lk;
         double* dk = J->dk + r * J->D;
         double* dv = J->dv + r * J->D;
+        double* mk = J->mk ? J->mk + r * J->D : NULL;
+        double* mv = J->mv ? J->mv + r * J->D : NULL;
         for (int64_t d = 0; d < J->D; ++d) dk[d] = dv[d] = 0.0;
+        if (mk)
+            for (int64_t d = 0; d < J->D; ++d) mk[d] = mv[d] = 0.0;
         for (int64_t g = 0; g < group; ++g) {
             for (int64_t i = 0; i < J->Lq; ++i) {
                 int64_t lo, hi;
@@ -581,6 +627,13 @@ static void* dkv_keys_worker(void* arg) {
                 for (int64_t d = 0; d < J->D; ++d) {
                     dv[d] += pij * doi[d];
                     dk[d] += J->scale * dsij * qi[d];
+                }
+                if (mk) {
+                    const double w = fabs(dsij) + pij * J->absdo[g * J->Lq + i];
+                    for (int64_t d = 0; d < J->D; ++d) {
+                        mk[d] += J->scale * w * fabs(qi[d]);
+                        mv[d] += pij * fabs(doi[d]);
+                    }
                 }
             }
         }
@@ -601,35 +654,40 @@ static int run_workers(void* (*fn)(void*), void* job, int64_t work, int nthreads
     return 0;
 }
 
-/* dq[n,D] of the query rows ids[r] = (b*Hq + h)*Lq + i (causal or no mask). */
+/* dq[n,D] of the query rows ids[r] = (b*Hq + h)*Lq + i (causal or no mask); mq[n,D]
+ * receives their sensitivities if not NULL. */
 int oracle_attn_bwd_dq_rows(const double* q, const double* k, const double* v,
                             const double* dout, const int64_t* rows, int64_t n, double* dq,
-                            int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
-                            int64_t D, double scale, int causal, int nthreads) {
+                            double* mq, int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq,
+                            int64_t Lk, int64_t D, double scale, int causal, int nthreads) {
     int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
     if (rc) return rc;
     for (int64_t r = 0; r < n; ++r)
         if (rows[r] < 0 || rows[r] >= B * Hq * Lq) return ORACLE_ERR_INDEX;
     sel_job J = {q, k, v, dout, B, Hq, Hkv, Lq, Lk, D, scale, causal, rows, n, dq, NULL, NULL,
-                 0, NULL, NULL, 0, ORACLE_OK};
+                 mq, NULL, NULL, 0, NULL, NULL, NULL, 0, ORACLE_OK};
     run_workers(dq_rows_worker, &J, n, nthreads);
     return J.status;
 }
 
-/* dk[n,D], dv[n,D] of the keys ids[r] = (b*Hkv + h_kv)*Lk + j (causal or no mask). */
+/* dk[n,D], dv[n,D] of the keys ids[r] = (b*Hkv + h_kv)*Lk + j (causal or no mask);
+ * mk, mv [n,D] receive their sensitivities when both are given. */
 int oracle_attn_bwd_dkv_keys(const double* q, const double* k, const double* v,
                              const double* dout, const int64_t* keys, int64_t n, double* dk,
-                             double* dv, int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq,
-                             int64_t Lk, int64_t D, double scale, int causal, int nthreads) {
+                             double* dv, double* mk, double* mv, int64_t B, int64_t Hq,
+                             int64_t Hkv, int64_t Lq, int64_t Lk, int64_t D, double scale,
+                             int causal, int nthreads) {
     int rc = check_dims(B, Hq, Hkv, Lq, Lk, D);
     if (rc) return rc;
     for (int64_t r = 0; r < n; ++r)
         if (keys[r] < 0 || keys[r] >= B * Hkv * Lk) return ORACLE_ERR_INDEX;
     const int64_t group = Hq / Hkv;
+    if (!mk || !mv) mk = mv = NULL;
     double* lse = (double*)malloc(sizeof(double) * (size_t)(group * Lq + 1));
     double* delta = (double*)malloc(sizeof(double) * (size_t)(group * Lq + 1));
-    if (!lse || !delta) {
-        free(lse); free(delta);
+    double* absdo = (double*)malloc(sizeof(double) * (size_t)(group * Lq + 1));
+    if (!lse || !delta || !absdo) {
+        free(lse); free(delta); free(absdo);
         return ORACLE_ERR_NOMEM;
     }
     int status = ORACLE_OK;
@@ -641,12 +699,12 @@ int oracle_attn_bwd_dkv_keys(const double* q, const double* k, const double* v,
             if (keys[r] / Lk == unit) seen = 1;
         if (seen) continue;
         sel_job J = {q, k, v, dout, B, Hq, Hkv, Lq, Lk, D, scale, causal, keys, n, NULL, dk, dv,
-                     unit, lse, delta, 0, ORACLE_OK};
+                     NULL, mk, mv, unit, lse, delta, absdo, 0, ORACLE_OK};
         run_workers(unit_stats_worker, &J, group * Lq, nthreads);
         J.next = 0;
         run_workers(dkv_keys_worker, &J, n, nthreads);
         status = J.status;
     }
-    free(lse); free(delta);
+    free(lse); free(delta); free(absdo);
     return status;
 }

@@ -1,0 +1,151 @@
+"""Parity of the attention backward pass (attn_bwd, attn_bwd_window) with the fp64 oracle.
+
+The forward pass runs on the GPU (attn_fwd / attn_fwd_window) and its O and lse feed
+the backward pass, as in training; the oracle computes dQ, dK, dV from q, k, v and dO
+alone, by the chain rule through the definition.
+
+Tolerance. The pages give none for gradients; this one follows from the rounding the
+kernels do. They round P and dS to the input dtype (relative error u = 2^-9 for bf16,
+2^-11 for f16) before the tensor-core products that form dV, dK and dQ. They compute
+delta_i = dO_i . O_i from the rounded output. They accumulate in fp32 and round each
+gradient to the dtype (another u). To first order every gradient element g is then
+off by at most u (m + |g|). Here m is the element's rounding sensitivity, which the
+oracle returns beside the gradient (for dQ_i: scale sum_j (|dS_ij| + P_ij sum_d
+|dO_id O_id|) |k_j|). fp32 accumulation over up to 8192 terms adds at most about
+2^-11 m. So each element is checked against
+    |g_gpu - g_ref| <= 3 u (m + |g_ref|).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_attention_19_b200 as ta
+from tiled_attention_19_b200 import inputs
+from tests.parity import guarded_empty, guards_intact
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+U = {torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -9}
+
+
+def check_grad(got, ref, sens, dtype, what):
+    g = got.detach().to("cpu", torch.float64)
+    ref = ref.to(torch.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    assert torch.isfinite(g).all(), f"{what}: non-finite gradient"
+    err = (g - ref).abs()
+    bound = 3 * U[dtype] * (sens.to(torch.float64) + ref.abs())
+    ok = err <= bound
+    if not bool(ok.all()):
+        at = tuple(int(i) for i in torch.nonzero(~ok)[0])
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements over the bound; first at {at}: "
+                             f"|err| {float(err[at]):.3e} > {float(bound[at]):.3e}")
+    ratio = float((err / bound.clamp_min(1e-300)).max()) if err.numel() else 0.0
+    print(f"{what}: max |err| / bound = {ratio:.3f}")
+    return ratio
+
+
+def run_case(B, Hq, Hkv, Lq, Lk, D, dtype, causal, window, seed):
+    s = inputs.DenseSpec("bwd", B, Hq, Hkv, Lq, Lk, D, dtype, causal, 1 / math.sqrt(D), seed)
+    x = inputs.make(s)
+    do = inputs.dense_grad_output(s)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    dout = do.to(DEV)
+    out, lse = ta.fwd(q, k, v, causal=causal, scale=s.scale, window=window)
+    qb, dq, qg = guarded_empty((B, Hq, Lq, D), dtype, DEV)
+    kb, dk, kg = guarded_empty((B, Hkv, Lk, D), dtype, DEV)
+    vb, dv, vg = guarded_empty((B, Hkv, Lk, D), dtype, DEV)
+    ta.bwd(q, k, v, out, dout, lse, causal=causal, scale=s.scale, window=window, dq=dq, dk=dk,
+           dv=dv)
+    torch.cuda.synchronize()
+    assert guards_intact(qb, qg) and guards_intact(kb, kg) and guards_intact(vb, vg)
+    assert ta.device_status() == 0
+    return s, x, do, (dq, dk, dv)
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, D, dtype, causal, window
+    (1, 2, 2, 300, 300, 64, torch.float16, False, None),
+    (1, 2, 2, 300, 300, 128, torch.bfloat16, True, None),
+    (2, 4, 2, 200, 333, 64, torch.bfloat16, True, None),     # grouped heads, Lq < Lk
+    (1, 2, 1, 260, 130, 128, torch.float16, True, None),      # Lq > Lk: rows that see no key
+    (1, 1, 1, 1, 1, 64, torch.float16, False, None),
+    (1, 2, 2, 65, 129, 128, torch.bfloat16, False, None),     # ragged sub-tiles and tiles
+    (1, 3, 3, 512, 512, 128, torch.float16, False, None),
+    (1, 4, 1, 256, 256, 64, torch.float16, True, None),       # group of 4
+    (1, 2, 2, 400, 400, 64, torch.bfloat16, False, (64, 32)),
+    (1, 2, 1, 333, 333, 128, torch.float16, True, (100, -1)),
+    (1, 2, 2, 300, 300, 128, torch.bfloat16, False, (0, 0)),  # each row sees one key
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}_H{}-{}_Lq{}_Lk{}_D{}_{}_{}_w{}".format(
+    *c[:6], str(c[6]).split(".")[-1], "causal" if c[7] else "full", c[8]))
+def test_backward_parity(case):
+    B, Hq, Hkv, Lq, Lk, D, dtype, causal, window = case
+    s, x, do, got = run_case(*case, seed=11 * Lq + Lk + D)
+    ref = oracle.attn_bwd(x["q"], x["k"], x["v"], do, s.scale, causal,
+                          window if window is not None else (-1, -1), sensitivity=True)
+    for i, name in enumerate(("dq", "dk", "dv")):
+        check_grad(got[i], ref[i], ref[3 + i], dtype, f"{case} {name}")
+
+
+def test_backward_is_deterministic():
+    case = (1, 4, 2, 333, 333, 128, torch.bfloat16, True, None)
+    _, _, _, a = run_case(*case, seed=3)
+    _, _, _, b = run_case(*case, seed=3)
+    for t, u in zip(a, b):
+        assert torch.equal(t, u)
+
+
+def test_backward_empty_sides():
+    q = torch.randn(1, 2, 5, 64, device=DEV).to(torch.float16)
+    k = torch.empty(1, 1, 0, 64, device=DEV, dtype=torch.float16)
+    out, lse = ta.fwd(q, k, k, causal=False)
+    dq = torch.full_like(q, 3.0)
+    ta.bwd(q, k, k, out, torch.ones_like(q), lse, dq=dq, dk=k.clone(), dv=k.clone())
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dq) == 0          # no keys: dQ = 0
+    q0 = torch.empty(1, 2, 0, 64, device=DEV, dtype=torch.float16)
+    kk = torch.randn(1, 1, 7, 64, device=DEV).to(torch.float16)
+    dk = torch.full_like(kk, 3.0)
+    dv = torch.full_like(kk, 3.0)
+    lse0 = torch.empty(1, 2, 0, device=DEV)
+    ta.bwd(q0, kk, kk, q0, q0, lse0, dq=q0.clone(), dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dk) == 0 and torch.count_nonzero(dv) == 0  # no queries
+    assert ta.device_status() == 0
+
+
+def test_backward_long_causal_prefill_sampled():
+    """The long causal prefill workload (B1 H16 L8192 D128 bf16) end to end on the GPU;
+    the oracle checks dQ on sampled rows of every head and dK, dV on sampled keys of one
+    head (it recomputes that head's row statistics)."""
+    s = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
+    x = inputs.make(s)
+    do = inputs.dense_grad_output(s)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    out, lse = ta.fwd(q, k, v, causal=True, scale=s.scale)
+    dq, dk, dv = ta.bwd(q, k, v, out, do.to(DEV), lse, causal=True, scale=s.scale)
+    torch.cuda.synchronize()
+    assert ta.device_status() == 0
+    L, H, D = s.Lq, s.Hq, s.D
+    rng = np.random.default_rng(7)
+    rows = np.concatenate([[0, 63, 64, 127, 128, L - 1], rng.integers(0, L, 42)])
+    heads = rng.integers(0, H, rows.shape[0])
+    ids = heads * L + rows
+    ref_dq, m_dq = oracle.attn_bwd_dq_rows(x["q"], x["k"], x["v"], do, ids, s.scale, True,
+                                           sensitivity=True)
+    check_grad(dq.reshape(-1, D)[torch.as_tensor(ids)].cpu(), ref_dq, m_dq, s.dtype, "dq rows")
+    h = 5
+    keys = np.concatenate([[0, 1, 127, 128, 4095, L - 1], rng.integers(0, L, 26)])
+    kid = h * L + keys
+    ref_dk, ref_dv, m_dk, m_dv = oracle.attn_bwd_dkv_keys(x["q"], x["k"], x["v"], do, kid,
+                                                          s.scale, True, sensitivity=True)
+    check_grad(dk.reshape(-1, D)[torch.as_tensor(kid)].cpu(), ref_dk, m_dk, s.dtype, "dk keys")
+    check_grad(dv.reshape(-1, D)[torch.as_tensor(kid)].cpu(), ref_dv, m_dv, s.dtype, "dv keys")

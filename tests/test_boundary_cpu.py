@@ -170,3 +170,64 @@ def test_workspace_size():
     assert ws(0, 12, 2, 128, 256) == 0
     assert ws(1, 4, 4, 64, 9) > 0
     assert ws(1024, 8, 2, 128, 256) == 0       # > 1024 units: one CTA per unit, no split
+
+
+def bwd_args(**kw):
+    a = dict(q=P, k=P, v=P, out=P, dout=P, lse=P, dq=P, dk=P, dv=P, B=1, Hq=2, Hkv=1, Lq=8, Lk=8,
+             D=64, scale=0.125, causal=0, dtype=0, ws=P, ws_n=1 << 20, stream=None)
+    a.update(kw)
+    return a
+
+
+BWD_BAD = [
+    ("null_dout", dict(dout=None), -1),
+    ("null_lse", dict(lse=None), -1),
+    ("null_dq", dict(dq=None), -1),
+    ("null_dk", dict(dk=None), -1),
+    ("neg_Lk", dict(Lk=-1), -1),
+    ("group_not_divisible", dict(Hq=3, Hkv=2), -1),
+    ("scale_nan", dict(scale=float("nan")), -1),
+    ("D_32", dict(D=32), -2),
+    ("dtype_fp32", dict(dtype=7), -2),
+    ("misaligned_dout", dict(dout=P + 2), -3),
+    ("misaligned_dv", dict(dv=P + 8), -3),
+    ("misaligned_lse", dict(lse=P + 1), -3),
+    ("workspace_missing", dict(ws=None, ws_n=0), -7),
+    ("workspace_small", dict(ws_n=8 * 2 * 128 - 1), -7),
+]
+
+
+def call_bwd(a, window=None):
+    lib = ta.load()
+    args = (a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"], a["dq"], a["dk"], a["dv"],
+            a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"], a["D"], a["scale"], a["causal"])
+    if window is None:
+        return lib.attn_bwd(*args, a["dtype"], a["ws"], a["ws_n"], a["stream"])
+    return lib.attn_bwd_window(*args, window[0], window[1], a["dtype"], a["ws"], a["ws_n"],
+                               a["stream"])
+
+
+@pytest.mark.parametrize("name,kw,code", BWD_BAD, ids=[c[0] for c in BWD_BAD])
+def test_attn_bwd_validation(name, kw, code):
+    rc = call_bwd(bwd_args(**kw))
+    assert rc == code, (rc, ta.STATUS.get(rc))
+
+
+def test_attn_bwd_window_validation():
+    assert call_bwd(bwd_args(), window=(-2, 3)) == -1
+    assert call_bwd(bwd_args(), window=(3, -5)) == -1
+    assert call_bwd(bwd_args(D=80), window=(3, 3)) == -2
+
+
+def test_bwd_empty_problems_and_workspace_size():
+    lib = ta.load()
+    # B == 0, or no queries and no keys: nothing to write, pointers may be NULL
+    assert lib.attn_bwd(None, None, None, None, None, None, None, None, None, 0, 2, 1, 8, 8, 64,
+                        0.1, 1, 0, None, 0, None) == 0
+    assert lib.attn_bwd(None, None, None, None, None, None, None, None, None, 1, 2, 1, 0, 0, 64,
+                        0.1, 1, 0, None, 0, None) == 0
+    ws = ta.bwd_workspace_size
+    assert ws(1, 16, 8192) == 8 * 16 * 8192
+    assert ws(2, 3, 1) == 8 * 6 * 128          # rows padded to a multiple of 128
+    assert ws(32, 12, 196) == 8 * 384 * 256
+    assert ws(0, 4, 100) == 0 and ws(1, 4, 0) == 0

@@ -509,12 +509,45 @@ def pin_bwd_selected_outputs(lib=None):
         close(sv, dv.reshape(-1, 4)[keys])
 
 
+def pin_bwd_sensitivity(lib=None):
+    """The rounding sensitivities the GPU tests scale their tolerances with: a numpy
+    statement from the oracle's probability matrix, the triangle inequality |g| <= m,
+    and the selected-output entry points agreeing with the whole."""
+    q = rand((1, 4, 7, 5), 940)
+    k = rand((1, 2, 9, 5), 941)
+    v = rand((1, 2, 9, 5), 942)
+    do = rand((1, 4, 7, 5), 943)
+    sc = 0.45
+    for causal in (False, True):
+        dq, dk, dv, mq, mk, mv = (t.numpy() for t in oracle.attn_bwd(
+            q, k, v, do, sc, causal, lib=lib, sensitivity=True))
+        P = oracle.attn_probs(q, k, v, sc, causal, lib=lib).numpy()
+        K, V = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+        dP = np.einsum("bhid,bhjd->bhij", do, V)
+        dS = P * (dP - (P * dP).sum(-1, keepdims=True))
+        A = np.abs(do * np.einsum("bhij,bhjd->bhid", P, V)).sum(-1)
+        W = np.abs(dS) + P * A[..., None]
+        close(mq, sc * np.einsum("bhij,bhjd->bhid", W, np.abs(K)))
+        close(mk, sc * np.einsum("bhij,bhid->bhjd", W, np.abs(q)).reshape(1, 2, 2, 9, 5).sum(2))
+        close(mv, np.einsum("bhij,bhid->bhjd", P, np.abs(do)).reshape(1, 2, 2, 9, 5).sum(2))
+        for g, m in ((dq, mq), (dk, mk), (dv, mv)):
+            assert (np.abs(g) <= m * (1 + 1e-12) + 1e-300).all()
+        rows = np.array([0, 6, 13, 27], np.int64)
+        _, mr = oracle.attn_bwd_dq_rows(q, k, v, do, rows, sc, causal, lib=lib, sensitivity=True)
+        close(mr, mq.reshape(-1, 5)[rows])
+        keys = np.array([0, 8, 9, 17], np.int64)
+        _, _, mkr, mvr = oracle.attn_bwd_dkv_keys(q, k, v, do, keys, sc, causal, lib=lib,
+                                                  sensitivity=True)
+        close(mkr, mk.reshape(-1, 5)[keys])
+        close(mvr, mv.reshape(-1, 5)[keys])
+
+
 PINS = [pin_brute_force, pin_golden, pin_probability_rows, pin_constant_values,
         pin_identical_keys, pin_argmax_limit, pin_causal_row0, pin_shift_invariance,
         pin_permutation_equivariance, pin_gqa_equals_repeat, pin_paged_equals_dense,
         pin_fully_masked_rows, pin_online_softmax, pin_split_combine, pin_window,
         pin_bwd_autograd, pin_bwd_finite_differences, pin_bwd_golden, pin_bwd_invariants,
-        pin_bwd_gqa_equals_repeat, pin_bwd_selected_outputs]
+        pin_bwd_gqa_equals_repeat, pin_bwd_selected_outputs, pin_bwd_sensitivity]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)

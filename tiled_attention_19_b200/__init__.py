@@ -1,5 +1,5 @@
-"""Python binding of libattn_b200: exact tiled attention forward and paged-KV decode on
-B200 (sm_100a).
+"""Python binding of libattn_b200: exact tiled attention forward and backward, and
+paged-KV decode on B200 (sm_100a).
 
 The binding only marshals arguments: tensors become raw device pointers and sizes, the
 stream is torch's current stream, and every step of the computation runs in the CUDA
@@ -7,6 +7,7 @@ kernels behind the C ABI in ``include/attn.h``. There is no CPU fallback: if the
 library is missing or the device is not sm_100, calls raise.
 
     out, lse = fwd(q, k, v, causal=True)                  # q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D]
+    dq, dk, dv = bwd(q, k, v, out, dout, lse, causal=True)
     out, lse = fwd_paged(q, k_cache, v_cache, block_table, seq_lens)
 """
 from __future__ import annotations
@@ -38,6 +39,11 @@ SIGNATURES = {
                             _i, _vp, _sz, _vp]),
     "attn_fwd_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i,
                                     _i, _f, _i, _vp]),
+    "attn_bwd_workspace_size": (_sz, [_i, _i, _i]),
+    "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
+                      _i, _vp, _sz, _vp]),
+    "attn_bwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                             _f, _i, _i, _i, _i, _vp, _sz, _vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_get_device_status": (_i, [_vp]),
     "attn_selftest_bounded_wait": (_i, [_vp]),
@@ -132,6 +138,51 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                                     _stream(stream))
         _check(rc, "attn_fwd_window")
     return out, lse
+
+
+def bwd_workspace_size(B: int, Hq: int, Lq: int) -> int:
+    return int(load().attn_bwd_workspace_size(B, Hq, Lq))
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+        dout: torch.Tensor, lse: torch.Tensor, causal: bool = False, scale: float | None = None,
+        window: tuple | None = None, dq: torch.Tensor | None = None,
+        dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+        workspace: torch.Tensor | None = None, stream=None):
+    """Gradients (dq, dk, dv) of attention given dout = dLoss/dO, from the forward pass's
+    inputs, output and lse (fwd with the same causal / window / scale). dk, dv have the
+    K/V heads' shape. The workspace (attn_bwd_workspace_size bytes) is allocated when not
+    given."""
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape or out.shape != q.shape or \
+            dout.shape != q.shape or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("shape mismatch")
+    if len({q.dtype, k.dtype, v.dtype, out.dtype, dout.dtype}) != 1:
+        raise TypeError("q, k, v, out, dout must share a dtype")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    n = bwd_workspace_size(B, Hq, Lq)
+    if workspace is None:
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_n = workspace.numel() * workspace.element_size()
+    args = (_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(dout, "dout"),
+            _dev(lse, "lse"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, Hq, Hkv, Lq, Lk,
+            D, float(scale), int(bool(causal)))
+    if window is None:
+        rc = load().attn_bwd(*args, _dtype_code(q.dtype), _dev(workspace, "workspace"), ws_n,
+                             _stream(stream))
+        _check(rc, "attn_bwd")
+    else:
+        rc = load().attn_bwd_window(*args, int(window[0]), int(window[1]), _dtype_code(q.dtype),
+                                    _dev(workspace, "workspace"), ws_n, _stream(stream))
+        _check(rc, "attn_bwd_window")
+    return dq, dk, dv
 
 
 def paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, D: int, max_blocks_per_seq: int,

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "backward_sm100.cuh"
 #include "paged_decode.cuh"
 #include "prefill_sm100.cuh"
 
@@ -67,16 +68,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view (D, L, planes) of a contiguous [planes, L, D] tensor; box 64 x 128 x 1 with
-// 128-byte swizzle. Rows past L read as zero and are never written.
-bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, long long planes) {
+// 3-D view (D, L, planes) of a contiguous [planes, L, D] tensor; box 64 x box_rows x 1
+// with 128-byte swizzle. Rows past L read as zero and are never written.
+bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, long long planes,
+                     int box_rows = attn::kBM) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                                 static_cast<cuuint64_t>(planes)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                    static_cast<cuuint64_t>(L) * D * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(attn::kBM), 1};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -224,9 +226,187 @@ attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, f
                 : dispatch_mask<128, false>(m, tq, tk, tv, args, planes, stream);
 }
 
+// ------------------------------------------------------------------ backward
+template <int D, bool BF16, int MASK, int KIND>
+attn_status_t launch_bwd(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                         const CUtensorMap& tz, const attn::BwdArgs& args, long long planes,
+                         int tiles, cudaStream_t stream) {
+    auto kern = attn::bwd_kernel<D, BF16, MASK, KIND>;
+    constexpr int smem = attn::BwdCfg<D>::kSmemBytes;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(tiles));
+    kern<<<grid, attn::kBwdThreads, smem, stream>>>(tx, tw, ty, tz, args);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool BF16, int MASK>
+attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* out,
+                      const void* dout, const float* lse, const attn::BwdArgs& args,
+                      long long planes_q, long long planes_kv, cudaStream_t stream) {
+    // dK, dV: fixed K and V (128-row boxes), streamed Q and dO (64-row boxes);
+    // dQ: fixed Q and dO, streamed K and V.
+    alignas(64) CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64;
+    if (!encode_tile_map(&k128, k, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
+        !encode_tile_map(&v128, v, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
+        !encode_tile_map(&q64, q, BF16, D, args.Lq, planes_q, attn::kBwdSub) ||
+        !encode_tile_map(&do64, dout, BF16, D, args.Lq, planes_q, attn::kBwdSub) ||
+        !encode_tile_map(&q128, q, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
+        !encode_tile_map(&do128, dout, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
+        !encode_tile_map(&k64, k, BF16, D, args.Lk, planes_kv, attn::kBwdSub) ||
+        !encode_tile_map(&v64, v, BF16, D, args.Lk, planes_kv, attn::kBwdSub))
+        return ATTN_ERR_CUDA;
+    const long long rows_pad = planes_q * args.Lq_pad;  // a multiple of 128: whole warps
+    const long long blocks = rows_pad * 8 / 256;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    attn::bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(out), static_cast<const uint16_t*>(dout), lse,
+        const_cast<float*>(args.lse2), const_cast<float*>(args.delta), args.Lq, args.Lq_pad,
+        rows_pad);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    attn_status_t st = launch_bwd<D, BF16, MASK, attn::kDKDV>(
+        k128, v128, q64, do64, args, planes_kv, (args.Lk + attn::kBwdFix - 1) / attn::kBwdFix,
+        stream);
+    if (st != ATTN_OK) return st;
+    return launch_bwd<D, BF16, MASK, attn::kDQ>(q128, do128, k64, v64, args, planes_q,
+                                                (args.Lq + attn::kBwdFix - 1) / attn::kBwdFix,
+                                                stream);
+}
+
+template <int D, bool BF16>
+attn_status_t dispatch_bwd(int mask, const void* q, const void* k, const void* v,
+                           const void* out, const void* dout, const float* lse,
+                           const attn::BwdArgs& args, long long planes_q, long long planes_kv,
+                           cudaStream_t stream) {
+    if (mask == attn::kMaskCausal)
+        return run_bwd<D, BF16, attn::kMaskCausal>(q, k, v, out, dout, lse, args, planes_q,
+                                                   planes_kv, stream);
+    if (mask == attn::kMaskWindow)
+        return run_bwd<D, BF16, attn::kMaskWindow>(q, k, v, out, dout, lse, args, planes_q,
+                                                   planes_kv, stream);
+    return run_bwd<D, BF16, attn::kMaskNone>(q, k, v, out, dout, lse, args, planes_q, planes_kv,
+                                             stream);
+}
+
+size_t bwd_workspace_bytes(long long planes_q, int Lq) {
+    const long long pad = (static_cast<long long>(Lq) + attn::kBwdFix - 1) / attn::kBwdFix *
+                          attn::kBwdFix;
+    return static_cast<size_t>(planes_q) * static_cast<size_t>(pad) * 2 * sizeof(float);
+}
+
+template <bool BF16>
+void fill_zero(void* p, size_t n, cudaStream_t stream) {
+    attn::fill_empty_kernel<BF16><<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(p), nullptr, n, 0);
+}
+
+attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int left, int right,
+                       attn_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream_) {
+    if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (Lq > kMaxSeq || Lk > kMaxSeq) return ATTN_ERR_UNSUPPORTED;
+    const long long planes_q = static_cast<long long>(B) * H_q;
+    const long long planes_kv = static_cast<long long>(B) * H_kv;
+    if (planes_q > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || (Lq == 0 && Lk == 0)) return ATTN_OK;  // nothing to write
+    const bool have_q = Lq > 0, have_k = Lk > 0;
+    if ((have_q && (q == nullptr || dq == nullptr)) ||
+        (have_k && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)) ||
+        (have_q && have_k && (out == nullptr || dout == nullptr || lse == nullptr)))
+        return ATTN_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4))
+        return ATTN_ERR_MISALIGNED;
+    if (have_q && have_k) {
+        if (workspace == nullptr || workspace_bytes < bwd_workspace_bytes(planes_q, Lq))
+            return ATTN_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return ATTN_ERR_MISALIGNED;
+    }
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool bf16 = dtype == ATTN_BF16;
+    if (!have_q || !have_k) {  // no queries: dK = dV = 0; no keys: dQ = 0
+        if (!have_q) {
+            const size_t n = static_cast<size_t>(planes_kv) * Lk * D;
+            if (bf16) { fill_zero<true>(dk, n, stream); fill_zero<true>(dv, n, stream); }
+            else { fill_zero<false>(dk, n, stream); fill_zero<false>(dv, n, stream); }
+        } else {
+            const size_t n = static_cast<size_t>(planes_q) * Lq * D;
+            if (bf16) fill_zero<true>(dq, n, stream);
+            else fill_zero<false>(dq, n, stream);
+        }
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
+
+    attn::BwdArgs args{};
+    args.Lq_pad = static_cast<int>((static_cast<long long>(Lq) + attn::kBwdFix - 1) /
+                                   attn::kBwdFix * attn::kBwdFix);
+    float* ws = static_cast<float*>(workspace);
+    args.lse2 = ws;
+    args.delta = ws + static_cast<size_t>(planes_q) * args.Lq_pad;
+    args.dq = dq;
+    args.dk = dk;
+    args.dv = dv;
+    args.Hq = H_q;
+    args.Hkv = H_kv;
+    args.group = H_q / H_kv;
+    args.Lq = Lq;
+    args.Lk = Lk;
+    args.win_left = left;
+    args.win_right = right;
+    args.scale = scale;
+    args.scale_log2 = scale * attn::kLog2e;
+    const int m = (left < 0 && right < 0) ? attn::kMaskNone
+                  : (left < 0 && right == 0) ? attn::kMaskCausal
+                                             : attn::kMaskWindow;
+    if (D == 64)
+        return bf16 ? dispatch_bwd<64, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream)
+                    : dispatch_bwd<64, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
+    return bf16 ? dispatch_bwd<128, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream)
+                : dispatch_bwd<128, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t attn_bwd_workspace_size(int B, int H_q, int Lq) {
+    if (B < 0 || H_q < 1 || Lq < 0) return 0;
+    return bwd_workspace_bytes(static_cast<long long>(B) * H_q, Lq);
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,
+                       attn_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_band(q, k, v, out, dout, lse, dq, dk, dv, B, H_q, H_kv, Lq, Lk, D, scale, -1,
+                    causal ? 0 : -1, dtype, workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int H_q, int H_kv, int Lq, int Lk, int D, float scale,
+                              int causal, int window_left, int window_right, attn_dtype_t dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID;
+    return bwd_band(q, k, v, out, dout, lse, dq, dk, dv, B, H_q, H_kv, Lq, Lk, D, scale,
+                    window_left, causal ? 0 : window_right, dtype, workspace, workspace_bytes,
+                    stream);
+}
+
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                        int H_q, int H_kv, int Lq, int Lk, int D, float scale, int causal,

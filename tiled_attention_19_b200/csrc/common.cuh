@@ -71,6 +71,9 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
     }
 }
 
+// Mask modes, fixed at compile time so the common cases carry no window arithmetic.
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
+
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 

@@ -91,9 +91,6 @@ struct PrefillArgs {
     float scale_log2;  // scale * log2(e)
 };
 
-// Mask modes, fixed at compile time so the common cases carry no window arithmetic.
-enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
-
 // First and one-past-last visible key of query row i (empty if hi <= lo).
 template <int MASK>
 __device__ __forceinline__ void row_keys(int i, const PrefillArgs& a, int& lo, int& hi) {

@@ -130,6 +130,19 @@ def dense_inputs(spec: DenseSpec) -> dict:
     return {"q": q.to(spec.dtype), "k": k.to(spec.dtype), "v": v.to(spec.dtype)}
 
 
+def dense_grad_output(spec: DenseSpec) -> torch.Tensor:
+    """dO = dLoss/dO for the backward pass: N(0,1) of q's shape in spec.dtype, from its
+    own generator (seed + 1000003) so the forward inputs are unchanged."""
+    g = torch.Generator().manual_seed(spec.seed + 1000003)
+    return _randn(g, (spec.B, spec.Hq, spec.Lq, spec.D)).to(spec.dtype)
+
+
+def backward_flops(spec: DenseSpec) -> float:
+    """Algorithmic FLOPs of the backward pass: five D-deep products (S, dP, dV, dK, dQ)
+    over the visible (query, key) pairs, 2.5 times the forward's."""
+    return 2.5 * spec.flops()
+
+
 def paged_inputs(spec: PagedSpec) -> dict:
     """Paged-decode inputs on the CPU. Draw order: seq_lens, block_table, k_cache,
     v_cache, q."""
