@@ -8,6 +8,10 @@ prefill kernel's device time; the decode's HBM GB/s is reported beside it. Both 
 are timed with CUDA events on the stream they run on. Inputs rotate over enough copies
 that every step reads data that is not in L2.
 
+After the step's timed region, the backward pass of the same prefill workload (attn_bwd)
+is timed on its own and reported in the line's ``backward`` object (--no-backward skips
+it); it is not part of ``value``.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 For N > 1 (launched by torch.distributed.run) every rank runs the same step on its own
@@ -249,6 +253,11 @@ def run_ours(args, ws, rank, local):
     pre_avg = reduce_max(sum(pre_ms) / len(pre_ms), ws, device)
     dec_avg = reduce_max(sum(dec_ms) / len(dec_ms), ws, device)
 
+    bwd_ms = None
+    if args.backward and do_pre:
+        bwd_ms = measure_backward(w, ta, stream, device, steps=max(3, min(100, args.steps)),
+                                  warmup=args.warmup, ws=ws, window=args.window)
+
     if args.e2e:
         e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)), window=args.window)
     else:
@@ -337,9 +346,71 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": (int(do_pre) + int(do_dec)) * args.steps,
         "clocks": clocks.summary(),
     }
+    if bwd_ms is not None:
+        bwd_flops = 2.5 * w.prefill_flops
+        bwd_tf = job_rate(bwd_flops, bwd_ms, ws, 1e12) / ws
+        line["backward"] = {
+            "what": "attn_bwd of the prefill workload: dQ, dK, dV from O, lse and a seeded dO",
+            "kernels": "bwd_prep_kernel + bwd_kernel<dK,dV> + bwd_kernel<dQ>",
+            "value": r2(bwd_tf * ws, 2),
+            "unit": "TFLOP/s",
+            "flops": bwd_flops,
+            "flops_note": "algorithmic: 2.5 x the forward's (five D-deep products per visible "
+                          "pair); the kernels execute seven (S and dP are recomputed by both "
+                          "the dK/dV and the dQ kernel), so 5/7 of the peak is their ceiling",
+            "bound": "tensor",
+            "achieved": r2(bwd_tf, 2),
+            "peak": pk_t,
+            "frac": r2(bwd_tf / pk_t, 4),
+            "avg_call_ms": round(bwd_ms, 5),
+            "steps": max(3, min(100, args.steps)),
+            "gpu_launches": 3 * max(3, min(100, args.steps)),
+        }
     if args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
+
+
+def measure_backward(w, ta, stream, device, steps: int, warmup: int, ws: int, window=None):
+    """The backward pass (attn_bwd) of the prefill workload, timed on its own after the
+    step: dO is seeded like the inputs, O and lse come from one forward call per input
+    copy, and the calls rotate over the copies as the step does."""
+    do_host = inputs.dense_grad_output(PREFILL)
+    sets = []
+    for p in w.pf:
+        out, lse = ta.fwd(p["q"], p["k"], p["v"], causal=PREFILL.causal, scale=PREFILL.scale,
+                          window=window, stream=stream)
+        sets.append((p, out, lse, do_host.to(device)))
+    dq = torch.empty_like(w.pf[0]["q"])
+    dk = torch.empty_like(w.pf[0]["k"])
+    dv = torch.empty_like(w.pf[0]["v"])
+    wsb = torch.empty(max(16, ta.bwd_workspace_size(PREFILL.B, PREFILL.Hq, PREFILL.Lq)),
+                      dtype=torch.uint8, device=device)
+
+    def call(i):
+        p, out, lse, do = sets[i % len(sets)]
+        ta.bwd(p["q"], p["k"], p["v"], out, do, lse, causal=PREFILL.causal, scale=PREFILL.scale,
+               window=window, dq=dq, dk=dk, dv=dv, workspace=wsb, stream=stream)
+
+    for i in range(warmup):
+        call(i)
+    torch.cuda.synchronize()
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set by the backward warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        call(warmup + i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set during the backward timing")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    return reduce_max(ms, ws, device)
 
 
 def measure_e2e(w, ta, stream, device, steps: int, window=None):
@@ -478,6 +549,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false",
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--no-backward", dest="backward", action="store_false",
+                    help="skip the separately timed backward pass of the prefill workload")
     ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",
                     help="run one kernel of the step only (profiling runs)")
     ap.add_argument("--copies", type=int, default=4,

@@ -4,6 +4,9 @@ Tolerances (fp32 accumulation, f16/bf16 outputs), compared element by element ag
 the fp64 oracle on the same inputs:
   O:   max |O_gpu - O_ref| <= 2e-3 (f16 outputs), <= 1.6e-2 (bf16 outputs)
   lse: |lse_gpu - lse_ref| <= 1e-4 * max(1, |lse_ref|); -inf exactly where the oracle has it
+Gradients (backward pass): |g_gpu - g_ref| <= 3 u (m + |g_ref|) element by element, with
+u the dtype's unit roundoff and m the element's first-order rounding sensitivity from the
+oracle (the derivation is in tests/test_backward_gpu.py).
 """
 from __future__ import annotations
 
@@ -49,3 +52,23 @@ def guards_intact(buf, g):
     el = buf.element_size()
     raw = buf.view(torch.int16 if el == 2 else torch.int32)
     return bool((raw[:g] == SENTINEL).all() and (raw[-g:] == SENTINEL).all())
+
+
+GRAD_U = {torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -9}
+
+
+def check_grad(got, ref, sens, dtype, what):
+    g = got.detach().to("cpu", torch.float64)
+    ref = ref.to(torch.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    assert torch.isfinite(g).all(), f"{what}: non-finite gradient"
+    err = (g - ref).abs()
+    bound = 3 * GRAD_U[dtype] * (sens.to(torch.float64) + ref.abs())
+    ok = err <= bound
+    if not bool(ok.all()):
+        at = tuple(int(i) for i in torch.nonzero(~ok)[0])
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements over the bound; first at {at}: "
+                             f"|err| {float(err[at]):.3e} > {float(bound[at]):.3e}")
+    ratio = float((err / bound.clamp_min(1e-300)).max()) if err.numel() else 0.0
+    print(f"{what}: max |err| / bound = {ratio:.3f}")
+    return ratio

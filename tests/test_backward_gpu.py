@@ -26,30 +26,10 @@ import torch
 import oracle
 import tiled_attention_19_b200 as ta
 from tiled_attention_19_b200 import inputs
-from tests.parity import guarded_empty, guards_intact
+from tests.parity import check_grad, guarded_empty, guards_intact
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
-U = {torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -9}
-
-
-def check_grad(got, ref, sens, dtype, what):
-    g = got.detach().to("cpu", torch.float64)
-    ref = ref.to(torch.float64)
-    assert g.shape == ref.shape, (what, g.shape, ref.shape)
-    assert torch.isfinite(g).all(), f"{what}: non-finite gradient"
-    err = (g - ref).abs()
-    bound = 3 * U[dtype] * (sens.to(torch.float64) + ref.abs())
-    ok = err <= bound
-    if not bool(ok.all()):
-        at = tuple(int(i) for i in torch.nonzero(~ok)[0])
-        raise AssertionError(f"{what}: {int((~ok).sum())} elements over the bound; first at {at}: "
-                             f"|err| {float(err[at]):.3e} > {float(bound[at]):.3e}")
-    ratio = float((err / bound.clamp_min(1e-300)).max()) if err.numel() else 0.0
-    print(f"{what}: max |err| / bound = {ratio:.3f}")
-    return ratio
-
-
 def run_case(B, Hq, Hkv, Lq, Lk, D, dtype, causal, window, seed):
     s = inputs.DenseSpec("bwd", B, Hq, Hkv, Lq, Lk, D, dtype, causal, 1 / math.sqrt(D), seed)
     x = inputs.make(s)
