@@ -44,8 +44,11 @@ DECODE = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
 METRIC = "fwd attention TFLOP/s & % of FP16 tensor peak; paged decode HBM GB/s"
 L2_BYTES = 126 * 1000 * 1000
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["tiled_attention_19_b200/csrc/" + f for f in
-                  ("api.cu", "common.cuh", "ptx.cuh", "prefill_sm100.cuh", "paged_decode.cuh")]
+# Device code of each kernel the committed ncu traffic figures were taken on.
+KERNEL_SOURCES = {
+    name: ["tiled_attention_19_b200/csrc/" + f for f in ("common.cuh", "ptx.cuh", header)]
+    for name, header in (("prefill", "prefill_sm100.cuh"), ("decode", "paged_decode.cuh"))
+}
 
 
 # ------------------------------------------------------------------------ helpers
@@ -58,25 +61,26 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, keyed by workload name, if
-    it was taken on the kernel sources as they are now (else empty)."""
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary,
+    if it was taken on that kernel's device code as it is now (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return {}
+        return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
-        return {}
-    return d.get("kernels", {})
+    e = d.get("kernels", {}).get(kernel, {})
+    if e.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return e.get("per_launch", {}).get(workload)
 
 
 class ClockSampler:
@@ -96,6 +100,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # nvidia-smi takes a moment to start: begin the timed region once it samples
+            t0 = time.perf_counter()
+            while not self.rows and time.perf_counter() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.rows.clear()
         except (OSError, ValueError):
             self.proc = None
         return self
@@ -277,7 +286,6 @@ def run_ours(args, ws, rank, local):
     r2 = lambda x, n: None if x is None else round(x, n)  # noqa: E731
     e2e_tf = job_rate(w.prefill_flops, e2e_pre, ws, 1e12) if do_pre else None
     e2e_gb = job_rate(w.decode_bytes, e2e_dec, ws, 1e9) if do_dec else None
-    traffic = profiled_traffic()
     pk_t = peaks["bf16_tflops_sustained"]
     pk_h = peaks["hbm_gbs"]
     line = {
@@ -319,7 +327,7 @@ def run_ours(args, ws, rank, local):
             "unit": "TFLOP/s",
             "frac": r2(per_gpu_tflops and per_gpu_tflops / pk_t, 4),
             "frac_of_burst_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops"], 4),
-            "traffic": None if args.window else traffic.get(PREFILL.name),
+            "traffic": None if args.window else profiled_traffic("prefill", PREFILL.name),
             "avg_launch_ms": round(pre_avg, 5),
         },
         "paged_decode": {
@@ -331,7 +339,7 @@ def run_ours(args, ws, rank, local):
             "peak": pk_h,
             "peak_source": f"{peaks_src} hbm_gbs",
             "frac": r2(per_gpu_gbs and per_gpu_gbs / pk_h, 4),
-            "traffic": traffic.get(DECODE.name),
+            "traffic": profiled_traffic("decode", DECODE.name),
             "avg_launch_ms": round(dec_avg, 5),
         },
         "e2e": {
@@ -541,7 +549,7 @@ def run_reference(args, ws, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,

@@ -114,6 +114,44 @@ attn_status_t attn_fwd_window(const void* q, const void* k, const void* v, void*
                               void* stream);
 
 /*
+ * attn_strides_t -- element strides of a tensor of shape [B, H, L, D] whose D elements
+ * are contiguous: element (b, h, l, d) sits at base + b*batch + h*head + l*seq + d.
+ * The contiguous layout [B, H, L, D] is {H*L*D, L*D, D}; flash_attn's [B, L, H, D] is
+ * {L*H*D, D, H*D}.
+ */
+typedef struct {
+    int64_t batch;
+    int64_t head;
+    int64_t seq;
+} attn_strides_t;
+
+/*
+ * attn_fwd_strided -- attn_fwd_window on tensors with arbitrary strides: the layouts
+ * of [B, L, H, D] tensors (flash_attn_func's q, k, v and output, "Flash Attention"
+ * skill page (hermes-agent-app.ru), Scenario 2), of q, k and v sliced from a packed
+ * QKV projection, or of any view whose D elements are contiguous.
+ *
+ *   q, k, v, out  base pointers, 16-byte aligned, with the strides in q_strides,
+ *                 k_strides, v_strides, out_strides (a NULL strides pointer means the
+ *                 contiguous [B, H, L, D] layout). Each stride of a dimension longer than
+ *                 1 must be positive, a multiple of 8 elements (16 bytes) and below 2^38;
+ *                 a stride of a dimension of length 1 is ignored.
+ *   lse           [B, H_q, Lq] fp32, contiguous, written if non-NULL.
+ *
+ *   out must not overlap q, k or v. All other arguments, results and errors as
+ *   attn_fwd_window (window_left = window_right = -1 for no window). Returns
+ *   ATTN_ERR_INVALID for a non-positive or oversized stride and ATTN_ERR_MISALIGNED
+ *   for a stride that is not a multiple of 8.
+ */
+attn_status_t attn_fwd_strided(const void* q, const attn_strides_t* q_strides, const void* k,
+                               const attn_strides_t* k_strides, const void* v,
+                               const attn_strides_t* v_strides, void* out,
+                               const attn_strides_t* out_strides, float* lse, int B, int H_q,
+                               int H_kv, int Lq, int Lk, int D, float scale, int causal,
+                               int window_left, int window_right, attn_dtype_t dtype,
+                               void* stream);
+
+/*
  * attn_paged_workspace_size -- bytes of device workspace attn_fwd_paged needs
  * for these sizes (0 when no sequence is ever split). The workspace holds the
  * partial results of the split-KV chunks (one per CTA of the balanced

@@ -231,3 +231,18 @@ def test_bwd_empty_problems_and_workspace_size():
     assert ws(2, 3, 1) == 8 * 6 * 128          # rows padded to a multiple of 128
     assert ws(32, 12, 196) == 8 * 384 * 256
     assert ws(0, 4, 100) == 0 and ws(1, 4, 0) == 0
+
+
+def test_attn_fwd_strided_validation():
+    lib = ta.load()
+    S = ta.Strides
+
+    def call(qs=None, ks=None, vs=None, os_=None, **kw):
+        a = fwd_args(**kw)
+        return lib.attn_fwd_strided(a["q"], qs, a["k"], ks, a["v"], vs, a["out"], os_, a["lse"],
+                                    a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"], a["D"],
+                                    a["scale"], a["causal"], -1, -1, a["dtype"], None)
+    assert call(qs=S(8 * 64 * 2, 64, 64 * 2 + 4)) == -3          # seq stride not a multiple of 8
+    assert call(ks=S(-8, 512, 64), B=2) == -1                    # negative stride of a used dim
+    assert call(os_=S(1 << 38, 512, 64), B=2) == -1              # oversized
+    assert call(qs=S(0, 0, 0), B=1, Hq=1, Hkv=1, Lq=1, D=96) == -2  # unused strides; D refused

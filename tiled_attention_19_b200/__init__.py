@@ -28,12 +28,22 @@ STATUS = {
     -4: "ATTN_ERR_DEVICE", -5: "ATTN_ERR_CUDA", -6: "ATTN_ERR_TIMEOUT", -7: "ATTN_ERR_WORKSPACE",
     -8: "ATTN_ERR_BAD_INDEX", -9: "ATTN_ERR_SCRATCH_LIMIT",
 }
+
+
+class Strides(ctypes.Structure):
+    """attn_strides_t: element strides over (batch, head, seq); D is contiguous."""
+    _fields_ = [("batch", ctypes.c_int64), ("head", ctypes.c_int64), ("seq", ctypes.c_int64)]
+
+
 # Every function include/attn.h declares, with its ctypes signature.
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_sp = ctypes.POINTER(Strides)
 SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _i,
                              _vp]),
+    "attn_fwd_strided": (_i, [_vp, _sp, _vp, _sp, _vp, _sp, _vp, _sp, _vp, _i, _i, _i, _i, _i, _i,
+                              _f, _i, _i, _i, _i, _vp]),
     "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                             _i, _vp, _sz, _vp]),
@@ -107,6 +117,14 @@ def _check(rc: int, what: str) -> None:
         raise AttnError(rc, what)
 
 
+def _strides(t: torch.Tensor, name: str) -> Strides:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError(f"{name} must be a 4-D view [B, H, L, D] with contiguous D")
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: float | None = None, out: torch.Tensor | None = None,
         lse: torch.Tensor | None = None, return_lse: bool = True, stream=None,
@@ -114,7 +132,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     """softmax(q k^T * scale [+ causal / window mask]) v.  q [B,Hq,Lq,D]; k, v [B,Hkv,Lk,D].
     window = (left, right) restricts query i to keys i'-left..i'+right (i' = i + Lk - Lq,
     -1 = unbounded). Returns (out [B,Hq,Lq,D], lse [B,Hq,Lq] fp32 or None). scale defaults
-    to 1/sqrt(D)."""
+    to 1/sqrt(D). q, k, v and out may be any views with a contiguous last dimension (for
+    example x.transpose(1, 2) of flash_attn's [B, L, H, D] tensors); those go through
+    attn_fwd_strided, and a default out takes q's strides."""
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
@@ -127,6 +147,16 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if not all(t.is_contiguous() for t in (q, k, v, out)):
+        st = [_strides(t, n) for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"))]
+        w = window if window is not None else (-1, -1)
+        rc = load().attn_fwd_strided(q.data_ptr(), st[0], k.data_ptr(), st[1], v.data_ptr(), st[2],
+                                     out.data_ptr(), st[3],
+                                     _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv,
+                                     Lq, Lk, D, float(scale), int(bool(causal)), int(w[0]),
+                                     int(w[1]), _dtype_code(q.dtype), _stream(stream))
+        _check(rc, "attn_fwd_strided")
+        return out, lse
     args = (_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
             _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv, Lq, Lk, D, float(scale),
             int(bool(causal)))

@@ -86,6 +86,63 @@ bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Element strides of a (batch, head, row) tensor with contiguous rows of D elements.
+struct Strides {
+    long long b, h, l;
+};
+
+Strides contiguous_strides(int H, int L, int D) {
+    return {static_cast<long long>(H) * L * D, static_cast<long long>(L) * D, D};
+}
+
+// Caller strides (NULL: contiguous [B, H, L, D]). Each stride of a dimension longer than
+// 1 must be a positive multiple of 8 elements (16 bytes, the TMA and vector-store unit)
+// below 2^38; the stride of a dimension of length 1 is never used and is replaced.
+attn_status_t take_strides(const attn_strides_t* in, int B, int H, int L, int D, Strides* out) {
+    *out = contiguous_strides(H, L, D);
+    if (in == nullptr) return ATTN_OK;
+    const long long v[3] = {in->batch, in->head, in->seq};
+    const long long ext[3] = {B, H, L};
+    long long* dst[3] = {&out->b, &out->h, &out->l};
+    for (int i = 0; i < 3; ++i) {
+        if (ext[i] <= 1) continue;  // keep the contiguous value
+        if (v[i] <= 0 || v[i] >= (1LL << 38)) return ATTN_ERR_INVALID;
+        if (v[i] % 8 != 0) return ATTN_ERR_MISALIGNED;
+        *dst[i] = v[i];
+    }
+    return ATTN_OK;
+}
+
+// 4-D view (D, L, H, B) of a tensor with element strides (l, h, b) and contiguous D;
+// box 64 x box_rows x 1 x 1 with 128-byte swizzle. Rows past L read as zero.
+bool encode_strided_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, int H, int B,
+                        const Strides& st, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.l) * 2, static_cast<cuuint64_t>(st.h) * 2,
+                                   static_cast<cuuint64_t>(st.b) * 2};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Zeros the D elements of every (batch, head, row) of a strided output.
+__global__ void zero_rows_kernel(uint16_t* out, long long sb, long long sh, long long sl, int H,
+                                 int L, int D, long long rows) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; r < rows;
+         r += stride) {
+        const long long i = r % L, bh = r / L;
+        uint4* p = reinterpret_cast<uint4*>(out + (bh / H) * sb + (bh % H) * sh + i * sl);
+        for (int c = 0; c < D / 8; ++c) p[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 // ------------------------------------------------------------------ launchers
 template <int D, bool BF16, int MASK>
 attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -164,7 +221,10 @@ attn_status_t launch_paged(const CUtensorMap& tk, const CUtensorMap& tv, const P
 // i' - left <= j <= i' + right with i' = i + (Lk - Lq); -1 leaves a side unbounded.
 attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                        int H_q, int H_kv, int Lq, int Lk, int D, float scale, int left,
-                       int right, attn_dtype_t dtype, void* stream_) {
+                       int right, attn_dtype_t dtype, void* stream_,
+                       const attn_strides_t* q_st = nullptr, const attn_strides_t* k_st = nullptr,
+                       const attn_strides_t* v_st = nullptr,
+                       const attn_strides_t* o_st = nullptr) {
     if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
     if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -180,11 +240,29 @@ attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, f
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         (lse != nullptr && !aligned(lse, 4)))
         return ATTN_ERR_MISALIGNED;
+    Strides sq, sk, sv, so;
+    attn_status_t st = take_strides(q_st, B, H_q, Lq, D, &sq);
+    if (st == ATTN_OK) st = take_strides(k_st, B, H_kv, Lk, D, &sk);
+    if (st == ATTN_OK) st = take_strides(v_st, B, H_kv, Lk, D, &sv);
+    if (st == ATTN_OK) st = take_strides(o_st, B, H_q, Lq, D, &so);
+    if (st != ATTN_OK) return st;
+    const bool out_contiguous = o_st == nullptr ||
+                                (so.b == static_cast<long long>(H_q) * Lq * D &&
+                                 so.h == static_cast<long long>(Lq) * D && so.l == D);
     const attn_status_t dev = check_device();
     if (dev != ATTN_OK) return dev;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const bool bf16 = dtype == ATTN_BF16;
 
+    if (Lk == 0 && !out_contiguous) {  // no keys: O = 0 through the strides, lse = -inf
+        const long long rows = planes_q * Lq;
+        zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(out), so.b, so.h, so.l,
+                                                   H_q, Lq, D, rows);
+        if (lse != nullptr)
+            attn::fill_empty_kernel<true><<<1184, 256, 0, stream>>>(nullptr, lse, 0,
+                                                                    static_cast<size_t>(rows));
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
     if (Lk == 0) {  // no keys at all: O = 0, lse = -inf
         const size_t rows = static_cast<size_t>(planes_q) * Lq;
         if (bf16)
@@ -197,14 +275,16 @@ attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, f
     }
 
     alignas(64) CUtensorMap tq, tk, tv;
-    const long long planes_kv = static_cast<long long>(B) * H_kv;
-    if (!encode_tile_map(&tq, q, bf16, D, Lq, planes_q) ||
-        !encode_tile_map(&tk, k, bf16, D, Lk, planes_kv) ||
-        !encode_tile_map(&tv, v, bf16, D, Lk, planes_kv))
+    if (!encode_strided_map(&tq, q, bf16, D, Lq, H_q, B, sq, attn::kBM) ||
+        !encode_strided_map(&tk, k, bf16, D, Lk, H_kv, B, sk, attn::kBN) ||
+        !encode_strided_map(&tv, v, bf16, D, Lk, H_kv, B, sv, attn::kBN))
         return ATTN_ERR_CUDA;
 
     PrefillArgs args{};
     args.out = out;
+    args.out_sb = so.b;
+    args.out_sh = so.h;
+    args.out_sl = so.l;
     args.lse = lse;
     args.Hq = H_q;
     args.Hkv = H_kv;
@@ -422,6 +502,19 @@ attn_status_t attn_fwd_window(const void* q, const void* k, const void* v, void*
     if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID;
     return fwd_band(q, k, v, out, lse, B, H_q, H_kv, Lq, Lk, D, scale, window_left,
                     causal ? 0 : window_right, dtype, stream);
+}
+
+attn_status_t attn_fwd_strided(const void* q, const attn_strides_t* q_strides, const void* k,
+                               const attn_strides_t* k_strides, const void* v,
+                               const attn_strides_t* v_strides, void* out,
+                               const attn_strides_t* out_strides, float* lse, int B, int H_q,
+                               int H_kv, int Lq, int Lk, int D, float scale, int causal,
+                               int window_left, int window_right, attn_dtype_t dtype,
+                               void* stream) {
+    if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID;
+    return fwd_band(q, k, v, out, lse, B, H_q, H_kv, Lq, Lk, D, scale, window_left,
+                    causal ? 0 : window_right, dtype, stream, q_strides, k_strides, v_strides,
+                    out_strides);
 }
 
 size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D, int max_blocks_per_seq,

@@ -83,6 +83,7 @@ struct PrefillCfg {
 
 struct PrefillArgs {
     void* out;
+    long long out_sb, out_sh, out_sl;  // element strides of out over (batch, head, row)
     float* lse;
     int Hq, Hkv, group, Lq, Lk;
     int n_q_blocks;    // ceil(Lq / 256): CTAs along the query axis
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int qb = args.n_q_blocks - 1 - blockIdx.y;     // longest causal blocks first
     const int h = bh % args.Hq;
     const int b = bh / args.Hq;
-    const int kv_plane = b * args.Hkv + h / args.group;  // grouped-query head mapping
+    const int hkv = h / args.group;  // grouped-query head mapping
     const int q0 = qb * 2 * kBM;
     // key-tile ranges of the two query tiles and of the CTA (their union, no gaps:
     // the band edges are monotone in the row)
@@ -236,8 +237,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
-                tma_load_3d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, bh);
-                tma_load_3d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, bh);
+                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, h, b);
+                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, h, b);
             }
             for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile jlo + n
                 const int j = jlo + n;
@@ -246,15 +247,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
-                                bar(K_FULL + sk), c * 64, j * kBN, kv_plane);
+                    tma_load_4d(sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
+                                bar(K_FULL + sk), c * 64, j * kBN, hkv, b);
                 k_issued = n + 1;
                 if (n >= NV && !wait_phase(bar(V_EMPTY + sv), ((n / NV) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(V_FULL + sv), Cfg::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
-                                bar(V_FULL + sv), c * 64, j * kBN, kv_plane);
+                    tma_load_4d(sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
+                                bar(V_FULL + sv), c * 64, j * kBN, hkv, b);
                 v_issued = n + 1;
             }
         }
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // ------------------------------------------------------------ epilogue
             const bool has = l > 0.f;
             const float inv_l = has ? 1.f / l : 0.f;
-            uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) +
-                                (static_cast<size_t>(bh) * args.Lq + row) * D;
+            uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) + b * args.out_sb +
+                                h * args.out_sh + static_cast<long long>(row) * args.out_sl;
 #pragma unroll
             for (int d0 = 0; d0 < D; d0 += 32) {
                 uint32_t o[32];
