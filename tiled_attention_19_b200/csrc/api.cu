@@ -312,15 +312,28 @@ attn_status_t launch_bwd(const CUtensorMap& tx, const CUtensorMap& tw, const CUt
                          const CUtensorMap& tz, const attn::BwdArgs& args, long long planes,
                          int tiles, cudaStream_t stream) {
     auto kern = attn::bwd_kernel<D, BF16, MASK, KIND>;
-    constexpr int smem = attn::BwdCfg<D>::kSmemBytes;
+    constexpr int smem = attn::BwdCfg<D, KIND>::kSmemBytes;
     static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
+    static attn_status_t setup = ATTN_OK;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+            setup = ATTN_ERR_CUDA;
+            return;
+        }
+        // The kernel moves registers between warpgroups with setmaxnreg; refuse to
+        // launch unless the registers it is launched with cover the split.
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+            setup = ATTN_ERR_CUDA;
+            return;
+        }
+        if (static_cast<long long>(fa.numRegs) * attn::kBwdThreads < attn::kBwdRegBudget)
+            setup = ATTN_ERR_UNSUPPORTED;
     });
-    if (attr_err != cudaSuccess) {
+    if (setup != ATTN_OK) {
         cudaGetLastError();
-        return ATTN_ERR_CUDA;
+        return setup;
     }
     const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(tiles));
     kern<<<grid, attn::kBwdThreads, smem, stream>>>(tx, tw, ty, tz, args);
@@ -331,31 +344,27 @@ template <int D, bool BF16, int MASK>
 attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* out,
                       const void* dout, const float* lse, const attn::BwdArgs& args,
                       long long planes_q, long long planes_kv, cudaStream_t stream) {
-    // dK, dV: fixed K and V (128-row boxes), streamed Q and dO (64-row boxes);
-    // dQ: fixed Q and dO, streamed K and V.
-    alignas(64) CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64;
-    if (!encode_tile_map(&k128, k, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
-        !encode_tile_map(&v128, v, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
-        !encode_tile_map(&q64, q, BF16, D, args.Lq, planes_q, attn::kBwdSub) ||
-        !encode_tile_map(&do64, dout, BF16, D, args.Lq, planes_q, attn::kBwdSub) ||
-        !encode_tile_map(&q128, q, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
-        !encode_tile_map(&do128, dout, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
-        !encode_tile_map(&k64, k, BF16, D, args.Lk, planes_kv, attn::kBwdSub) ||
-        !encode_tile_map(&v64, v, BF16, D, args.Lk, planes_kv, attn::kBwdSub))
+    // dK, dV: fixed K and V, streamed Q and dO; dQ: fixed Q and dO, streamed K and V
+    // (128-row boxes throughout).
+    static_assert(attn::kBwdFix == attn::kBwdSub, "one box height for fixed and streamed tiles");
+    alignas(64) CUtensorMap tk, tv, tq, tdo;
+    if (!encode_tile_map(&tk, k, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
+        !encode_tile_map(&tv, v, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
+        !encode_tile_map(&tq, q, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
+        !encode_tile_map(&tdo, dout, BF16, D, args.Lq, planes_q, attn::kBwdFix))
         return ATTN_ERR_CUDA;
     const long long rows_pad = planes_q * args.Lq_pad;  // a multiple of 128: whole warps
     const long long blocks = rows_pad * 8 / 256;
     if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     attn::bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const uint16_t*>(out), static_cast<const uint16_t*>(dout), lse,
-        const_cast<float*>(args.lse2), const_cast<float*>(args.delta), args.Lq, args.Lq_pad,
+        const_cast<float*>(args.nlse2), const_cast<float*>(args.delta), args.Lq, args.Lq_pad,
         rows_pad);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     attn_status_t st = launch_bwd<D, BF16, MASK, attn::kDKDV>(
-        k128, v128, q64, do64, args, planes_kv, (args.Lk + attn::kBwdFix - 1) / attn::kBwdFix,
-        stream);
+        tk, tv, tq, tdo, args, planes_kv, (args.Lk + attn::kBwdFix - 1) / attn::kBwdFix, stream);
     if (st != ATTN_OK) return st;
-    return launch_bwd<D, BF16, MASK, attn::kDQ>(q128, do128, k64, v64, args, planes_q,
+    return launch_bwd<D, BF16, MASK, attn::kDQ>(tq, tdo, tk, tv, args, planes_q,
                                                 (args.Lq + attn::kBwdFix - 1) / attn::kBwdFix,
                                                 stream);
 }
@@ -435,7 +444,7 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
     args.Lq_pad = static_cast<int>((static_cast<long long>(Lq) + attn::kBwdFix - 1) /
                                    attn::kBwdFix * attn::kBwdFix);
     float* ws = static_cast<float*>(workspace);
-    args.lse2 = ws;
+    args.nlse2 = ws;
     args.delta = ws + static_cast<size_t>(planes_q) * args.Lq_pad;
     args.dq = dq;
     args.dk = dk;

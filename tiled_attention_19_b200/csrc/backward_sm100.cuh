@@ -16,26 +16,29 @@
 //                    are padded to a multiple of 128 (padding: lse2 = +inf, delta = 0,
 //                    so padded and fully masked rows give P = 0).
 //   bwd_kernel<kDKDV> one CTA per 128-key tile of one (batch, K/V head): K and V stay in
-//                    shared memory while 64-row sub-tiles of Q and dO (of every query head
-//                    of the group) stream through a ring; dV and dK accumulate in TMEM.
+//                    shared memory while 128-row sub-tiles of Q and dO (of every query
+//                    head of the group) stream through a ring; dV and dK accumulate in TMEM.
 //   bwd_kernel<kDQ>  one CTA per 128-row query tile of one (batch, head): Q and dO stay,
-//                    64-key sub-tiles of K and V stream; dQ accumulates in TMEM.
+//                    128-key sub-tiles of K and V stream; dQ accumulates in TMEM.
 // Both kinds run the same pipeline. Call the fixed pair (X, W) and a streamed pair
 // (Y, Z): (K, V) and (Q, dO) for kDKDV, (Q, dO) and (K, V) for kDQ. Per sub-tile n:
-//   S  = X Y^T, dP = W Z^T            (M = 128 fixed rows, N = 64, K = D; both operands
-//                                      K-major from shared memory), into TMEM buffer n & 1
-//   softmax warps: P and dS from S, dP and the row statistics, written back over the
-//                 first half of their own S / dP columns in f16/bf16
+//   S  = X Y^T, dP = W Z^T     (M = N = 128, K = D; both operands K-major from shared
+//                               memory; fp32 in TMEM)
+//   softmax warps: copy their half of S and dP to registers and release the dP columns
+//                 at once (DP_FREE), so dP of sub-tile n+1 is computed while they work;
+//                 then write P (kDKDV only) and dS in f16/bf16 over their own S columns
 //   kDKDV: dV += P Z, dK += dS Y;  kDQ: dQ += dS Y   (A from TMEM, B MN-major from
-//                                      shared memory; M = 128, N = D, K = 64)
-// For kDKDV the TMEM rows are keys and S is the transpose of the forward's scores; for
-// kDQ the rows are queries. The S and dP buffers are double-buffered, so the MMAs of
-// sub-tile n+1 run while the softmax warps work on sub-tile n.
+//                               shared memory; M = 128, N = D, K = 128)
+// For kDKDV the TMEM rows are keys and S is the transpose of the forward's scores; its
+// single S buffer takes S of sub-tile n+1 once the gradient MMAs of n are issued. kDQ
+// has two S buffers, so S and dP of n+1 are both computed while the softmax works on n.
+// Every product is 128 wide: a 64-wide product of the same work runs at a fraction of the
+// tensor core's rate.
 //
-// Roles (320 threads): warps 0-7 softmax (warp w reads TMEM lanes 32 (w % 4) .. +32 and
-// the sub-tile's columns 32 (w / 4) .. +32), warp 8 TMA producer, warp 9 MMA issuer and
-// TMEM owner. TMEM (512 columns): S0 at 0, S1 at 64, dP0 at 128, dP1 at 192, then the
-// accumulators (kDKDV: dV at 256, dK at 256 + D; kDQ: dQ at 256).
+// Roles (384 threads): warps 0-7 softmax (warp w reads TMEM lanes 32 (w % 4) .. +32 and
+// the sub-tile's columns 64 (w / 4) .. +64), warp 8 TMA producer, warp 9 MMA issuer and
+// TMEM owner, warps 10-11 idle (they complete the third warpgroup for setmaxnreg). TMEM (512 columns): kDQ: S0 at 0, S1 at 128, dP at 256, dQ at 384; kDKDV: S
+// at 0, dP at 128, dV at 256, dK at 256 + D.
 #pragma once
 #include <cuda.h>
 
@@ -43,31 +46,45 @@
 
 namespace attn {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 384;
+// Register split between warpgroups (setmaxnreg), as in the forward kernel: the two
+// softmax warpgroups take 192 registers, the third (producer, MMA issuer, two idle warps)
+// keeps 104. The launcher checks that the CTA's launch registers (384 x registers per
+// thread) cover 2 x 128 x 192 + 128 x 104 before the first launch: an unsatisfiable
+// setmaxnreg.inc would wait forever.
+constexpr int kBwdSoftmaxRegs = 192;
+constexpr int kBwdOtherRegs = 104;
+constexpr int kBwdRegBudget = 2 * 128 * kBwdSoftmaxRegs + 128 * kBwdOtherRegs;  // 62,464
 constexpr int kBwdFix = 128;  // rows of the fixed tiles (TMEM lanes)
-constexpr int kBwdSub = 64;   // rows of a streamed sub-tile
+constexpr int kBwdSub = 128;  // rows of a streamed sub-tile
 enum : int { kDKDV = 0, kDQ = 1 };
 
-template <int D>
+template <int D, int KIND>
 struct BwdCfg {
     static constexpr int kChunks = D / 64;                 // 128-byte column chunks
     static constexpr int kFixChunk = kBwdFix * 128;        // one chunk of a fixed tile
     static constexpr int kSubChunk = kBwdSub * 128;        // one chunk of a sub-tile
     static constexpr int kFixBytes = kBwdFix * D * 2;
     static constexpr int kSubBytes = kBwdSub * D * 2;
-    static constexpr int kStages = (D == 64) ? 8 : 4;
-    static constexpr int kTileRegion = 2 * kFixBytes + kStages * 2 * kSubBytes;
-    static constexpr int kStatBytes = kStages * 2 * kBwdSub * 4;  // lse2 + delta per stage
-    // barriers: FIX_FULL, FULL/EMPTY per stage, ST_FULL[2], P_FULL[2], DONE, DRAIN
-    static constexpr int kNumBars = 1 + 2 * kStages + 6;
+    // Separate rings for the two streamed tiles. kDQ frees V (Z) after dP and K (Y) only
+    // after dQ += dS K, so K gets the extra stage.
+    static constexpr int kYStages = (D == 64) ? 4 : (KIND == kDQ ? 3 : 2);
+    static constexpr int kZStages = (D == 64) ? 4 : 2;
+    static constexpr int kTileRegion = 2 * kFixBytes + (kYStages + kZStages) * kSubBytes;
+    // kDKDV: -lse*log2(e) and delta of the 128 query rows of each Y stage
+    static constexpr int kStatBytes = (KIND == kDKDV) ? kYStages * 2 * kBwdSub * 4 : 0;
+    // barriers: FIX_FULL, FULL/EMPTY per Y and per Z stage, ST_FULL, DP_FREE, P_FULL, DONE, DRAIN
+    static constexpr int kNumBars = 1 + 2 * (kYStages + kZStages) + 5;
     static constexpr int kSmemBytes = 1024 + kTileRegion + kStatBytes + kNumBars * 8 + 16;
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
-    static constexpr int kSCol0 = 0, kSCol1 = 64, kDPCol0 = 128, kDPCol1 = 192, kGCol = 256;
+    // TMEM: kDQ: S0 at 0, S1 at 128, dP at 256, dQ at 384;
+    //       kDKDV: S at 0, dP at 128, dV at 256, dK at 256 + D.
+    static constexpr int kSCol0 = 0, kSCol1 = 128;
     static constexpr int kTmemCols = 512;
 };
 
 struct BwdArgs {
-    const float* lse2;   // [B*Hq][Lq_pad] log2-domain lse (+inf: row sees no key / padding)
+    const float* nlse2;  // [B*Hq][Lq_pad] -lse * log2(e) (-inf: row sees no key / padding)
     const float* delta;  // [B*Hq][Lq_pad] dO . O
     void* dq;            // [B, Hq, Lq, D]
     void* dk;            // [B, Hkv, Lk, D]
@@ -85,6 +102,18 @@ __device__ __forceinline__ bool bwd_visible(int i, int j, const BwdArgs& a) {
     if (MASK == kMaskCausal) return j <= ii;
     if (MASK == kMaskWindow)
         return (a.win_left < 0 || j >= ii - a.win_left) && (a.win_right < 0 || j <= ii + a.win_right);
+    return true;
+}
+
+// True if every query of [i0, i0 + ni) sees every key of [j0, j0 + nj) (no element mask
+// needed; rows past Lq are zeroed through their -inf statistics instead).
+template <int MASK>
+__device__ __forceinline__ bool bwd_all_visible(int i0, int ni, int j0, int nj, const BwdArgs& a) {
+    const int off = a.Lk - a.Lq;
+    if (MASK == kMaskCausal) return j0 + nj - 1 <= i0 + off;
+    if (MASK == kMaskWindow)
+        return (a.win_left < 0 || j0 >= i0 + ni - 1 + off - a.win_left) &&
+               (a.win_right < 0 || j0 + nj - 1 <= i0 + off + a.win_right);
     return true;
 }
 
@@ -115,13 +144,13 @@ __device__ __forceinline__ void bwd_range(int base, const BwdArgs& a, int& lo, i
     }
 }
 
-// lse2 = lse * log2(e) (+inf where lse = -inf) and delta = dO . O per query row, into
-// rows padded to Lq_pad (padding: +inf and 0). Eight threads per row.
+// nlse2 = -lse * log2(e) (-inf where lse = -inf) and delta = dO . O per query row, into
+// rows padded to Lq_pad (padding: -inf and 0). Eight threads per row.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ out,
                                                        const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse,
-                                                       float* __restrict__ lse2,
+                                                       float* __restrict__ nlse2,
                                                        float* __restrict__ delta, int Lq,
                                                        int Lq_pad, long long rows_pad) {
     constexpr int kPer = D / 8;  // elements per thread: 16 (D = 128) or 8 (D = 64)
@@ -150,12 +179,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 #pragma unroll
     for (int o = 4; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (sub == 0) {
-        float l2 = INFINITY;
+        float nl2 = -INFINITY;
         if (i < Lq) {
             const float l = lse[static_cast<size_t>(plane) * Lq + i];
-            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
+            nl2 = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
         }
-        lse2[r] = l2;
+        nlse2[r] = nl2;
         delta[r] = (i < Lq) ? acc : 0.f;
     }
 }
@@ -165,16 +194,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_z,
                const BwdArgs args) {
-    using Cfg = BwdCfg<D>;
-    constexpr int NS = Cfg::kStages;
+    using Cfg = BwdCfg<D, KIND>;
+    constexpr int NY = Cfg::kYStages;
+    constexpr int NZ = Cfg::kZStages;
     constexpr int FIX_FULL = 0;
-    constexpr int FULL = 1;
-    constexpr int EMPTY = FULL + NS;
-    constexpr int ST_FULL = EMPTY + NS;  // [2]
-    constexpr int P_FULL = ST_FULL + 2;  // [2]
-    constexpr int DONE = P_FULL + 2;
+    constexpr int Y_FULL = 1;
+    constexpr int Y_EMPTY = Y_FULL + NY;
+    constexpr int Z_FULL = Y_EMPTY + NY;
+    constexpr int Z_EMPTY = Z_FULL + NZ;
+    constexpr int ST_FULL = Z_EMPTY + NZ;  // S and dP of the next sub-tile are in TMEM
+    constexpr int DP_FREE = ST_FULL + 1;   // the softmax warps hold S and dP in registers
+    constexpr int P_FULL = DP_FREE + 1;    // P / dS of the sub-tile are in TMEM
+    constexpr int DONE = P_FULL + 1;
     constexpr int DRAIN = DONE + 1;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
+    constexpr uint32_t DP_COL = (KIND == kDKDV) ? 128 : 256;
+    constexpr uint32_t G_COL = (KIND == kDKDV) ? 256 : 384;
+    static_assert(G_COL + (KIND == kDKDV ? 2 * D : D) <= Cfg::kTmemCols, "TMEM budget");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -182,15 +218,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t s_base = smem_u32(smem);
     const uint32_t sX = s_base;
     const uint32_t sW = s_base + Cfg::kFixBytes;
-    const uint32_t sStage0 = s_base + 2 * Cfg::kFixBytes;  // stage s: Y at +2s*Sub, Z after it
-    float* stats = reinterpret_cast<float*>(smem + Cfg::kTileRegion);  // [NS][2][64]
+    const uint32_t sY0 = s_base + 2 * Cfg::kFixBytes;
+    const uint32_t sZ0 = sY0 + NY * Cfg::kSubBytes;
+    float* stats = reinterpret_cast<float*>(smem + Cfg::kTileRegion);  // kDKDV: [NY][2][128]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kTileRegion + Cfg::kStatBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t bar0 = smem_u32(bars);
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
-    auto sY = [&](int st) -> uint32_t { return sStage0 + 2u * st * Cfg::kSubBytes; };
-    auto sZ = [&](int st) -> uint32_t { return sStage0 + (2u * st + 1) * Cfg::kSubBytes; };
+    auto sY = [&](int n) -> uint32_t { return sY0 + (n % NY) * Cfg::kSubBytes; };
+    auto sZ = [&](int n) -> uint32_t { return sZ0 + (n % NZ) * Cfg::kSubBytes; };
+    // TMEM column of the S buffer sub-tile n uses (kDQ alternates two; kDKDV has one)
+    auto s_col_of = [&](int n) -> uint32_t {
+        return (KIND == kDQ && (n & 1)) ? Cfg::kSCol1 : Cfg::kSCol0;
+    };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -209,14 +250,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar(FIX_FULL), 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(bar(FULL + s), 1);
-            mbar_init(bar(EMPTY + s), 1);
+        for (int s = 0; s < NY; ++s) {
+            mbar_init(bar(Y_FULL + s), 1);
+            mbar_init(bar(Y_EMPTY + s), 1);
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(ST_FULL + t), 1);
-            mbar_init(bar(P_FULL + t), 256);
+        for (int s = 0; s < NZ; ++s) {
+            mbar_init(bar(Z_FULL + s), 1);
+            mbar_init(bar(Z_EMPTY + s), 1);
         }
+        mbar_init(bar(ST_FULL), 1);
+        mbar_init(bar(DP_FREE), 256);
+        mbar_init(bar(P_FULL), 256);
         mbar_init(bar(DONE), 1);
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
@@ -237,11 +281,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int issued = 0;  // producer: sub-tiles issued (for the abort drain)
+    int y_issued = 0, z_issued = 0;  // producer: sub-tiles issued per ring (abort drain)
     bool mma_started = false;
 
-    if (warp == 8) {
+    if (warp >= 10) {
+        regs_decrease<kBwdOtherRegs>();  // idle warps of the third warpgroup
+    } else if (warp == 8) {
         // ------------------------------------------------------------ producer
+        regs_decrease<kBwdOtherRegs>();
         if (lane == 0 && n_all > 0) {
             const int fix_plane = (KIND == kDKDV) ? kv_plane : plane;
             mbar_arrive_expect_tx(bar(FIX_FULL), 2 * Cfg::kFixBytes);
@@ -251,8 +298,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_3d(sW + c * Cfg::kFixChunk, &tm_w, bar(FIX_FULL), c * 64, base, fix_plane);
             }
             for (int n = 0; n < n_all; ++n) {
-                const int st = n % NS;
-                if (n >= NS && !wait_phase(bar(EMPTY + st), ((n / NS) - 1) & 1, abort_flag)) break;
                 int sub, y_plane;
                 if (KIND == kDKDV) {
                     const int g = n / n_sub;
@@ -263,160 +308,199 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     y_plane = kv_plane;
                 }
                 const int row = sub * kBwdSub;
-                mbar_arrive_expect_tx(bar(FULL + st), 2 * Cfg::kSubBytes +
-                                                          (KIND == kDKDV ? 2 * kBwdSub * 4 : 0));
+                // Z first: its slot frees earlier (kDQ: after dP; kDKDV: after dV, before dK)
+                const int zs = n % NZ, ys = n % NY;
+                if (n >= NZ && !wait_phase(bar(Z_EMPTY + zs), ((n / NZ) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(Z_FULL + zs), Cfg::kSubBytes);
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c) {
-                    tma_load_3d(sY(st) + c * Cfg::kSubChunk, &tm_y, bar(FULL + st), c * 64, row, y_plane);
-                    tma_load_3d(sZ(st) + c * Cfg::kSubChunk, &tm_z, bar(FULL + st), c * 64, row, y_plane);
-                }
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                    tma_load_3d(sZ(n) + c * Cfg::kSubChunk, &tm_z, bar(Z_FULL + zs), c * 64, row, y_plane);
+                z_issued = n + 1;
+                if (n >= NY && !wait_phase(bar(Y_EMPTY + ys), ((n / NY) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(Y_FULL + ys),
+                                      Cfg::kSubBytes + (KIND == kDKDV ? 2 * kBwdSub * 4 : 0));
+#pragma unroll
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                    tma_load_3d(sY(n) + c * Cfg::kSubChunk, &tm_y, bar(Y_FULL + ys), c * 64, row, y_plane);
                 if (KIND == kDKDV) {
                     const size_t so = static_cast<size_t>(y_plane) * args.Lq_pad + row;
-                    bulk_load(smem_u32(stats + st * 2 * kBwdSub), args.lse2 + so, kBwdSub * 4,
-                              bar(FULL + st));
-                    bulk_load(smem_u32(stats + st * 2 * kBwdSub + kBwdSub), args.delta + so,
-                              kBwdSub * 4, bar(FULL + st));
+                    bulk_load(smem_u32(stats + ys * 2 * kBwdSub), args.nlse2 + so, kBwdSub * 4,
+                              bar(Y_FULL + ys));
+                    bulk_load(smem_u32(stats + ys * 2 * kBwdSub + kBwdSub), args.delta + so,
+                              kBwdSub * 4, bar(Y_FULL + ys));
                 }
-                issued = n + 1;
+                y_issued = n + 1;
             }
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
+        regs_decrease<kBwdOtherRegs>();
         if (lane == 0 && n_all > 0) {
             constexpr uint32_t kIdescSD = idesc_f16(BF16, kBwdFix, kBwdSub, false, false);
             constexpr uint32_t kIdescG = idesc_f16(BF16, kBwdFix, D, false, true);
             mma_started = true;
-            // S = X Y^T and dP = W Z^T into buffer n & 1 (K-major: 16 elements = 32 bytes
-            // per step inside a 128-byte swizzle row, then the next chunk).
-            auto issue_sd = [&](int n) {
-                const int st = n % NS;
-                const uint32_t s_col = (n & 1) ? Cfg::kSCol1 : Cfg::kSCol0;
-                const uint32_t dp_col = (n & 1) ? Cfg::kDPCol1 : Cfg::kDPCol0;
+            // S = X Y^T into column s_col, or dP = W Z^T into DP_COL (K-major operands: 16
+            // elements = 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
+            auto issue_prod = [&](uint32_t a_tile, uint32_t b_tile, uint32_t d_col) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t fa = (kk >> 2) * Cfg::kFixChunk + (kk & 3) * 32;
                     const uint32_t fb = (kk >> 2) * Cfg::kSubChunk + (kk & 3) * 32;
-                    mma_ss(tmem + s_col, sdesc_sw128(sX + fa, 16, 1024),
-                           sdesc_sw128(sY(st) + fb, 16, 1024), kIdescSD, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + d_col, sdesc_sw128(a_tile + fa, 16, 1024),
+                           sdesc_sw128(b_tile + fb, 16, 1024), kIdescSD, kk > 0 ? 1u : 0u);
                 }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t fa = (kk >> 2) * Cfg::kFixChunk + (kk & 3) * 32;
-                    const uint32_t fb = (kk >> 2) * Cfg::kSubChunk + (kk & 3) * 32;
-                    mma_ss(tmem + dp_col, sdesc_sw128(sW + fa, 16, 1024),
-                           sdesc_sw128(sZ(st) + fb, 16, 1024), kIdescSD, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(ST_FULL + (n & 1)));
             };
-            // Gradient MMAs: A from TMEM (the f16/bf16 P or dS; rows 16ks..16ks+15 of the
-            // sub-tile sit in the columns of the softmax warpgroup ks / 2 that wrote them),
-            // B MN-major from the sub-tile (16 rows = two 8-row swizzle atoms, 2048 bytes;
+            // acc += A B with A the f16/bf16 tile the softmax warps packed into TMEM at
+            // a_col (sub-tile rows 64w .. 64w+63 sit at columns 64w .. 64w+31 of it), B
+            // MN-major from a sub-tile (16 rows = two 8-row swizzle atoms, 2048 bytes;
             // D chunks kSubChunk apart).
-            auto issue_grad = [&](int n) {
-                const int st = n % NS;
-                const uint32_t s_col = (n & 1) ? Cfg::kSCol1 : Cfg::kSCol0;
-                const uint32_t dp_col = (n & 1) ? Cfg::kDPCol1 : Cfg::kDPCol0;
+            auto issue_grad = [&](uint32_t acc_col, uint32_t a_col, uint32_t b_tile, bool first) {
 #pragma unroll
-                for (int ks = 0; ks < kBwdSub / 16; ++ks) {
-                    const uint32_t a_off = (ks >> 1) * 32 + (ks & 1) * 8;
-                    const uint32_t acc = (n > 0 || ks > 0) ? 1u : 0u;
-                    if (KIND == kDKDV)  // dV += P dO
-                        mma_ts(tmem + Cfg::kGCol, tmem + s_col + a_off,
-                               sdesc_sw128(sZ(st) + ks * 2048, Cfg::kSubChunk, 1024), kIdescG, acc);
-                    // kDKDV: dK += dS Q;  kDQ: dQ += dS K
-                    mma_ts(tmem + Cfg::kGCol + (KIND == kDKDV ? D : 0), tmem + dp_col + a_off,
-                           sdesc_sw128(sY(st) + ks * 2048, Cfg::kSubChunk, 1024), kIdescG, acc);
-                }
-                mma_commit(bar(EMPTY + st));
+                for (int ks = 0; ks < kBwdSub / 16; ++ks)
+                    mma_ts(tmem + acc_col, tmem + a_col + (ks >> 2) * 64 + (ks & 3) * 8,
+                           sdesc_sw128(b_tile + ks * 2048, Cfg::kSubChunk, 1024), kIdescG,
+                           (!first || ks > 0) ? 1u : 0u);
             };
             bool ok = wait_phase(bar(FIX_FULL), 0, abort_flag) &&
-                      wait_phase(bar(FULL + 0), 0, abort_flag);
+                      wait_phase(bar(Y_FULL + 0), 0, abort_flag) &&
+                      wait_phase(bar(Z_FULL + 0), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_sd(0);
+                issue_prod(sX, sY(0), s_col_of(0));
+                issue_prod(sW, sZ(0), DP_COL);
+                mma_commit(bar(ST_FULL));
+                if (KIND == kDQ) mma_commit(bar(Z_EMPTY + 0));  // V(0) was needed by dP only
             }
             for (int n = 0; ok && n < n_all; ++n) {
-                if (n + 1 < n_all) {
-                    // Buffer (n+1) & 1 was last read by the softmax of n-1 (done: its
-                    // P_FULL was awaited) and by the gradient MMAs of n-1 (issued earlier,
-                    // so they execute first).
-                    ok = wait_phase(bar(FULL + (n + 1) % NS), ((n + 1) / NS) & 1, abort_flag);
+                const int m = n + 1;
+                const bool more = m < n_all;
+                if (more) {
+                    // The softmax warps copied S(n) and dP(n) to registers: dP(n+1) may take
+                    // the dP columns. kDQ: S(n+1) goes to the other S buffer, last read by
+                    // the gradient MMA of n-1, issued before this one.
+                    ok = wait_phase(bar(Z_FULL + m % NZ), (m / NZ) & 1, abort_flag) &&
+                         (KIND == kDKDV || wait_phase(bar(Y_FULL + m % NY), (m / NY) & 1, abort_flag)) &&
+                         wait_phase(bar(DP_FREE), n & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_sd(n + 1);
+                    if (KIND == kDQ) issue_prod(sX, sY(m), s_col_of(m));
+                    issue_prod(sW, sZ(m), DP_COL);
+                    if (KIND == kDQ) {
+                        mma_commit(bar(ST_FULL));
+                        mma_commit(bar(Z_EMPTY + m % NZ));
+                    }
                 }
-                ok = wait_phase(bar(P_FULL + (n & 1)), (n >> 1) & 1, abort_flag);
+                ok = wait_phase(bar(P_FULL), n & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                issue_grad(n);
+                if (KIND == kDKDV) {
+                    // dV += P dO, then dK += dS Q; P and dS sit in the S columns
+                    issue_grad(G_COL, Cfg::kSCol0, sZ(n), n == 0);
+                    mma_commit(bar(Z_EMPTY + n % NZ));
+                    issue_grad(G_COL + D, Cfg::kSCol0 + 32, sY(n), n == 0);
+                    mma_commit(bar(Y_EMPTY + n % NY));
+                    if (more) {
+                        // S(n+1) overwrites the P and dS just read (those MMAs run first)
+                        ok = wait_phase(bar(Y_FULL + m % NY), (m / NY) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_prod(sX, sY(m), Cfg::kSCol0);
+                        mma_commit(bar(ST_FULL));
+                    }
+                } else {
+                    issue_grad(G_COL, s_col_of(n), sY(n), n == 0);  // dQ += dS K
+                    mma_commit(bar(Y_EMPTY + n % NY));
+                }
             }
             if (ok) mma_commit(bar(DONE));
         }
     } else {
         // ------------------------------------------------------------- softmax
-        const int wg = warp >> 2;  // which 32 columns of the 64-wide sub-tile
+        regs_increase<kBwdSoftmaxRegs>();
+        const int wg = warp >> 2;  // which 64 columns of the 128-wide sub-tile
         const int quad = warp & 3;
         const int r = base + quad * 32 + lane;  // this thread's fixed row (key or query)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const float c = args.scale_log2;
-        float row_lse2 = 0.f, row_delta = 0.f;
+        const uint64_t c2 = f2pack(args.scale_log2, args.scale_log2);
+        uint64_t nl2_row = 0, dl2_row = 0;
         if (KIND == kDQ) {  // padded rows exist up to Lq_pad > r
-            row_lse2 = args.lse2[static_cast<size_t>(plane) * args.Lq_pad + r];
-            row_delta = args.delta[static_cast<size_t>(plane) * args.Lq_pad + r];
+            const float nl = args.nlse2[static_cast<size_t>(plane) * args.Lq_pad + r];
+            const float dl = args.delta[static_cast<size_t>(plane) * args.Lq_pad + r];
+            nl2_row = f2pack(nl, nl);
+            dl2_row = f2pack(dl, dl);
         }
         bool ok = true;
         for (int n = 0; n < n_all; ++n) {
-            const int buf = n & 1;
-            const int st = n % NS;
             const int sub = (KIND == kDKDV) ? s_lo + n % n_sub : s_lo + n;
-            bool w = wait_phase(bar(ST_FULL + buf), (n >> 1) & 1, abort_flag);
-            if (KIND == kDKDV) w = w && wait_phase(bar(FULL + st), (n / NS) & 1, abort_flag);
+            bool w = wait_phase(bar(ST_FULL), n & 1, abort_flag);
+            if (KIND == kDKDV) w = w && wait_phase(bar(Y_FULL + n % NY), (n / NY) & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t s_col = (buf ? Cfg::kSCol1 : Cfg::kSCol0) + wg * 32;
-            const uint32_t dp_col = (buf ? Cfg::kDPCol1 : Cfg::kDPCol0) + wg * 32;
-            uint32_t sr[32], dr[32];
-            tmem_ld32(lane_base + s_col, sr);
-            tmem_ld32(lane_base + dp_col, dr);
+            const uint32_t s_col = s_col_of(n) + wg * 64;
+            const uint32_t dp_col = DP_COL + wg * 64;
+            uint32_t sr[64], dr[64];
+            tmem_ld32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld32(lane_base + dp_col, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+            tmem_ld32(lane_base + dp_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
             tmem_wait_ld();
-            const int cbase = sub * kBwdSub + wg * 32;  // first column index (query or key)
-            uint32_t pk[16], dk[16];
-            if (KIND == kDKDV) {
-                const float* L = stats + st * 2 * kBwdSub + wg * 32;
-                const float* Dl = L + kBwdSub;
+            tc_fence_before();
+            mbar_arrive(bar(DP_FREE));
+            const int cbase = sub * kBwdSub + wg * 64;  // first column index (query or key)
+            const float* st = stats + (n % NY) * 2 * kBwdSub + wg * 64;
 #pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[x]), c, -L[x]));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[x + 1]), c, -L[x + 1]));
-                    if (MASK != kMaskNone) {
-                        if (!bwd_visible<MASK>(cbase + x, r, args)) p0 = 0.f;
-                        if (!bwd_visible<MASK>(cbase + x + 1, r, args)) p1 = 0.f;
+            for (int h = 0; h < 2; ++h) {
+                const int c0 = cbase + h * 32;  // first column of this half
+                bool full;
+                if (KIND == kDKDV) full = bwd_all_visible<MASK>(c0, 32, r, 1, args);
+                else full = c0 + 32 <= args.Lk && bwd_all_visible<MASK>(r, 1, c0, 32, args);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int x = h * 32 + 2 * q;
+                    uint64_t nl2, dl2;
+                    if (KIND == kDKDV) {
+                        const float2 nl = reinterpret_cast<const float2*>(st + h * 32)[q];
+                        const float2 dl = reinterpret_cast<const float2*>(st + kBwdSub + h * 32)[q];
+                        nl2 = f2pack(nl.x, nl.y);
+                        dl2 = f2pack(dl.x, dl.y);
+                    } else {
+                        nl2 = nl2_row;
+                        dl2 = dl2_row;
                     }
-                    const float d0 = p0 * (__uint_as_float(dr[x]) - Dl[x]);
-                    const float d1 = p1 * (__uint_as_float(dr[x + 1]) - Dl[x + 1]);
-                    pk[x / 2] = pack2<BF16>(p0, p1);
-                    dk[x / 2] = pack2<BF16>(d0, d1);
+                    float t0, t1;
+                    f2unpack(fma2(f2pack(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), c2, nl2),
+                             t0, t1);
+                    float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    if (!full) {
+                        if (KIND == kDKDV) {
+                            if (!bwd_visible<MASK>(c0 + 2 * q, r, args)) p0 = 0.f;
+                            if (!bwd_visible<MASK>(c0 + 2 * q + 1, r, args)) p1 = 0.f;
+                        } else {
+                            if (c0 + 2 * q >= args.Lk || !bwd_visible<MASK>(r, c0 + 2 * q, args)) p0 = 0.f;
+                            if (c0 + 2 * q + 1 >= args.Lk || !bwd_visible<MASK>(r, c0 + 2 * q + 1, args))
+                                p1 = 0.f;
+                        }
+                    }
+                    if (KIND == kDKDV) pk[q] = pack2<BF16>(p0, p1);
+                    float d0, d1;
+                    f2unpack(mul2(f2pack(p0, p1),
+                                  sub2(f2pack(__uint_as_float(dr[x]), __uint_as_float(dr[x + 1])), dl2)),
+                             d0, d1);
+                    dk[q] = pack2<BF16>(d0, d1);
                 }
-                tmem_st16(lane_base + s_col, pk);
-            } else {
-                const bool edge = (MASK != kMaskNone) || (cbase + 32 > args.Lk);
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[x]), c, -row_lse2));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[x + 1]), c, -row_lse2));
-                    if (edge) {
-                        if (cbase + x >= args.Lk || !bwd_visible<MASK>(r, cbase + x, args)) p0 = 0.f;
-                        if (cbase + x + 1 >= args.Lk || !bwd_visible<MASK>(r, cbase + x + 1, args))
-                            p1 = 0.f;
-                    }
-                    dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - row_delta),
-                                            p1 * (__uint_as_float(dr[x + 1]) - row_delta));
+                if (KIND == kDKDV) {
+                    // P at columns 64w + [0, 32), dS at 64w + [32, 64) of the S buffer: this
+                    // warpgroup's own S columns, already copied to registers
+                    tmem_st16(lane_base + s_col + h * 16, pk);
+                    tmem_st16(lane_base + s_col + 32 + h * 16, dk);
+                } else {
+                    tmem_st16(lane_base + s_col + h * 16, dk);  // dS at 64w + [0, 32)
                 }
             }
-            tmem_st16(lane_base + dp_col, dk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_FULL + buf));
+            mbar_arrive(bar(P_FULL));
         }
         if (ok && n_all > 0) {
             const bool w = wait_phase(bar(DONE), 0, abort_flag);
@@ -436,14 +520,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       (static_cast<size_t>(plane) * args.Lk + r) * D;
                 col0 = 0;
                 ncols = D;
-                g_col = Cfg::kGCol + wg * D;
+                g_col = G_COL + wg * D;
                 mul = wg == 0 ? 1.f : args.scale;
                 valid = r < args.Lk;
             } else {
                 dst = static_cast<uint16_t*>(args.dq) + (static_cast<size_t>(plane) * args.Lq + r) * D;
                 col0 = wg * (D / 2);
                 ncols = D / 2;
-                g_col = Cfg::kGCol + col0;
+                g_col = G_COL + col0;
                 mul = args.scale;
                 valid = r < args.Lq;
             }
@@ -479,8 +563,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // exits: wait for the loads already issued and for every MMA issued.
         if (warp == 8 && lane == 0 && n_all > 0) {
             drain_phase(bar(FIX_FULL), 0);
-            for (int n = max(0, issued - NS); n < issued; ++n)
-                drain_phase(bar(FULL + n % NS), (n / NS) & 1);
+            for (int n = max(0, y_issued - NY); n < y_issued; ++n)
+                drain_phase(bar(Y_FULL + n % NY), (n / NY) & 1);
+            for (int n = max(0, z_issued - NZ); n < z_issued; ++n)
+                drain_phase(bar(Z_FULL + n % NZ), (n / NZ) & 1);
         }
         if (warp == 9 && lane == 0 && mma_started) {
             mma_commit(bar(DRAIN));
