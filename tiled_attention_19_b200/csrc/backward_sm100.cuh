@@ -24,21 +24,23 @@
 // (Y, Z): (K, V) and (Q, dO) for kDKDV, (Q, dO) and (K, V) for kDQ. Per sub-tile n:
 //   S  = X Y^T, dP = W Z^T     (M = N = 128, K = D; both operands K-major from shared
 //                               memory; fp32 in TMEM)
-//   softmax warps: copy their half of S and dP to registers and release the dP columns
-//                 at once (DP_FREE), so dP of sub-tile n+1 is computed while they work;
-//                 then write P (kDKDV only) and dS in f16/bf16 over their own S columns
-//   kDKDV: dV += P Z, dK += dS Y;  kDQ: dQ += dS Y   (A from TMEM, B MN-major from
+//   softmax warps: copy S and dP to registers, release the dP columns (DP_FREE) and
+//                 form P and dS; kDKDV does it in two phases (P from S as soon as S is
+//                 there, dS once dP is); write P (kDKDV only) and dS in f16/bf16 over
+//                 their own S columns
+//   kDKDV: dK += dS Y, dV += P Z;  kDQ: dQ += dS Y   (A from TMEM, B MN-major from
 //                               shared memory; M = 128, N = D, K = 128)
-// For kDKDV the TMEM rows are keys and S is the transpose of the forward's scores; its
-// single S buffer takes S of sub-tile n+1 once the gradient MMAs of n are issued. kDQ
-// has two S buffers, so S and dP of n+1 are both computed while the softmax works on n.
+// For kDKDV the TMEM rows are keys and S is the transpose of the forward's scores. Its
+// two 128-column regions swap roles every sub-tile: S(n+1) goes where dP(n) was as soon
+// as the softmax warps hold dP(n), so their exponentials for n+1 overlap the gradient
+// MMAs of n; dP(n+1) then takes the region of S(n) behind those MMAs. kDQ keeps two S
+// buffers and one dP buffer and computes S and dP of n+1 while the softmax works on n.
 // Every product is 128 wide: a 64-wide product of the same work runs at a fraction of the
 // tensor core's rate.
 //
 // Roles (384 threads): warps 0-7 softmax (warp w reads TMEM lanes 32 (w % 4) .. +32 and
 // the sub-tile's columns 64 (w / 4) .. +64), warp 8 TMA producer, warp 9 MMA issuer and
-// TMEM owner, warps 10-11 idle (they complete the third warpgroup for setmaxnreg). TMEM (512 columns): kDQ: S0 at 0, S1 at 128, dP at 256, dQ at 384; kDKDV: S
-// at 0, dP at 128, dV at 256, dK at 256 + D.
+// TMEM owner, warps 10-11 idle (they complete the third warpgroup for setmaxnreg).
 #pragma once
 #include <cuda.h>
 
@@ -73,13 +75,14 @@ struct BwdCfg {
     static constexpr int kTileRegion = 2 * kFixBytes + (kYStages + kZStages) * kSubBytes;
     // kDKDV: -lse*log2(e) and delta of the 128 query rows of each Y stage
     static constexpr int kStatBytes = (KIND == kDKDV) ? kYStages * 2 * kBwdSub * 4 : 0;
-    // barriers: FIX_FULL, FULL/EMPTY per Y and per Z stage, ST_FULL, DP_FREE, P_FULL, DONE, DRAIN
-    static constexpr int kNumBars = 1 + 2 * (kYStages + kZStages) + 5;
+    // barriers: FIX_FULL, FULL/EMPTY per Y and per Z stage, S_FULL, DP_FULL, DP_FREE, P_FULL,
+    // DONE, DRAIN
+    static constexpr int kNumBars = 1 + 2 * (kYStages + kZStages) + 6;
     static constexpr int kSmemBytes = 1024 + kTileRegion + kStatBytes + kNumBars * 8 + 16;
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
-    // TMEM: kDQ: S0 at 0, S1 at 128, dP at 256, dQ at 384;
-    //       kDKDV: S at 0, dP at 128, dV at 256, dK at 256 + D.
-    static constexpr int kSCol0 = 0, kSCol1 = 128;
+    // TMEM: kDQ: S of even / odd sub-tiles at 0 / 128, dP at 256, dQ at 384;
+    //       kDKDV: two regions at 0 and 128 that swap roles every sub-tile (S of sub-tile n
+    //       in region n & 1, its dP in the other), dV at 256, dK at 256 + D.
     static constexpr int kTmemCols = 512;
 };
 
@@ -202,13 +205,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr int Y_EMPTY = Y_FULL + NY;
     constexpr int Z_FULL = Y_EMPTY + NY;
     constexpr int Z_EMPTY = Z_FULL + NZ;
-    constexpr int ST_FULL = Z_EMPTY + NZ;  // S and dP of the next sub-tile are in TMEM
-    constexpr int DP_FREE = ST_FULL + 1;   // the softmax warps hold S and dP in registers
+    constexpr int S_FULL = Z_EMPTY + NZ;   // S of the next sub-tile is in TMEM
+    constexpr int DP_FULL = S_FULL + 1;    // dP of the next sub-tile is in TMEM
+    constexpr int DP_FREE = DP_FULL + 1;   // the softmax warps hold S and dP in registers
     constexpr int P_FULL = DP_FREE + 1;    // P / dS of the sub-tile are in TMEM
     constexpr int DONE = P_FULL + 1;
     constexpr int DRAIN = DONE + 1;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
-    constexpr uint32_t DP_COL = (KIND == kDKDV) ? 128 : 256;
     constexpr uint32_t G_COL = (KIND == kDKDV) ? 256 : 384;
     static_assert(G_COL + (KIND == kDKDV ? 2 * D : D) <= Cfg::kTmemCols, "TMEM budget");
 
@@ -228,9 +231,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
     auto sY = [&](int n) -> uint32_t { return sY0 + (n % NY) * Cfg::kSubBytes; };
     auto sZ = [&](int n) -> uint32_t { return sZ0 + (n % NZ) * Cfg::kSubBytes; };
-    // TMEM column of the S buffer sub-tile n uses (kDQ alternates two; kDKDV has one)
-    auto s_col_of = [&](int n) -> uint32_t {
-        return (KIND == kDQ && (n & 1)) ? Cfg::kSCol1 : Cfg::kSCol0;
+    // TMEM columns of S and dP of sub-tile n (P and dS are written over S)
+    auto s_col_of = [&](int n) -> uint32_t { return (n & 1) ? 128u : 0u; };
+    auto dp_col_of = [&](int n) -> uint32_t {
+        return (KIND == kDQ) ? 256u : ((n & 1) ? 0u : 128u);
     };
 
     const int warp = threadIdx.x >> 5;
@@ -258,7 +262,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(bar(Z_FULL + s), 1);
             mbar_init(bar(Z_EMPTY + s), 1);
         }
-        mbar_init(bar(ST_FULL), 1);
+        mbar_init(bar(S_FULL), 1);
+        mbar_init(bar(DP_FULL), 1);
         mbar_init(bar(DP_FREE), 256);
         mbar_init(bar(P_FULL), 256);
         mbar_init(bar(DONE), 1);
@@ -308,28 +313,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     y_plane = kv_plane;
                 }
                 const int row = sub * kBwdSub;
-                // Z first: its slot frees earlier (kDQ: after dP; kDKDV: after dV, before dK)
+                // Load first the tile whose slot frees first and is needed first: kDQ
+                // frees V (Z) after dP; kDKDV needs Q (Y) early, for S of the next sub-tile.
                 const int zs = n % NZ, ys = n % NY;
-                if (n >= NZ && !wait_phase(bar(Z_EMPTY + zs), ((n / NZ) - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(Z_FULL + zs), Cfg::kSubBytes);
+                auto load_z = [&]() -> bool {
+                    if (n >= NZ && !wait_phase(bar(Z_EMPTY + zs), ((n / NZ) - 1) & 1, abort_flag))
+                        return false;
+                    mbar_arrive_expect_tx(bar(Z_FULL + zs), Cfg::kSubBytes);
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sZ(n) + c * Cfg::kSubChunk, &tm_z, bar(Z_FULL + zs), c * 64, row, y_plane);
-                z_issued = n + 1;
-                if (n >= NY && !wait_phase(bar(Y_EMPTY + ys), ((n / NY) - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(Y_FULL + ys),
-                                      Cfg::kSubBytes + (KIND == kDKDV ? 2 * kBwdSub * 4 : 0));
+                    for (int c = 0; c < Cfg::kChunks; ++c)
+                        tma_load_3d(sZ(n) + c * Cfg::kSubChunk, &tm_z, bar(Z_FULL + zs), c * 64, row,
+                                    y_plane);
+                    z_issued = n + 1;
+                    return true;
+                };
+                auto load_y = [&]() -> bool {
+                    if (n >= NY && !wait_phase(bar(Y_EMPTY + ys), ((n / NY) - 1) & 1, abort_flag))
+                        return false;
+                    mbar_arrive_expect_tx(bar(Y_FULL + ys),
+                                          Cfg::kSubBytes + (KIND == kDKDV ? 2 * kBwdSub * 4 : 0));
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_3d(sY(n) + c * Cfg::kSubChunk, &tm_y, bar(Y_FULL + ys), c * 64, row, y_plane);
-                if (KIND == kDKDV) {
-                    const size_t so = static_cast<size_t>(y_plane) * args.Lq_pad + row;
-                    bulk_load(smem_u32(stats + ys * 2 * kBwdSub), args.nlse2 + so, kBwdSub * 4,
-                              bar(Y_FULL + ys));
-                    bulk_load(smem_u32(stats + ys * 2 * kBwdSub + kBwdSub), args.delta + so,
-                              kBwdSub * 4, bar(Y_FULL + ys));
+                    for (int c = 0; c < Cfg::kChunks; ++c)
+                        tma_load_3d(sY(n) + c * Cfg::kSubChunk, &tm_y, bar(Y_FULL + ys), c * 64, row,
+                                    y_plane);
+                    if (KIND == kDKDV) {
+                        const size_t so = static_cast<size_t>(y_plane) * args.Lq_pad + row;
+                        bulk_load(smem_u32(stats + ys * 2 * kBwdSub), args.nlse2 + so, kBwdSub * 4,
+                                  bar(Y_FULL + ys));
+                        bulk_load(smem_u32(stats + ys * 2 * kBwdSub + kBwdSub), args.delta + so,
+                                  kBwdSub * 4, bar(Y_FULL + ys));
+                    }
+                    y_issued = n + 1;
+                    return true;
+                };
+                if (KIND == kDQ) {
+                    if (!load_z() || !load_y()) break;
+                } else {
+                    if (!load_y() || !load_z()) break;
                 }
-                y_issued = n + 1;
             }
         }
     } else if (warp == 9) {
@@ -367,26 +388,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (ok) {
                 tc_fence_after();
                 issue_prod(sX, sY(0), s_col_of(0));
-                issue_prod(sW, sZ(0), DP_COL);
-                mma_commit(bar(ST_FULL));
+                mma_commit(bar(S_FULL));
+                issue_prod(sW, sZ(0), dp_col_of(0));
+                mma_commit(bar(DP_FULL));
                 if (KIND == kDQ) mma_commit(bar(Z_EMPTY + 0));  // V(0) was needed by dP only
             }
             for (int n = 0; ok && n < n_all; ++n) {
                 const int m = n + 1;
                 const bool more = m < n_all;
                 if (more) {
-                    // The softmax warps copied S(n) and dP(n) to registers: dP(n+1) may take
-                    // the dP columns. kDQ: S(n+1) goes to the other S buffer, last read by
-                    // the gradient MMA of n-1, issued before this one.
-                    ok = wait_phase(bar(Z_FULL + m % NZ), (m / NZ) & 1, abort_flag) &&
-                         (KIND == kDKDV || wait_phase(bar(Y_FULL + m % NY), (m / NY) & 1, abort_flag)) &&
+                    // The softmax warps copied S(n) and dP(n) to registers. S(n+1) takes
+                    // the region dP(n) used (kDKDV) or the S buffer of n-1, whose dS the
+                    // gradient MMA of n-1 (issued earlier) reads first (kDQ); kDQ's dP(n+1)
+                    // takes the dP columns.
+                    ok = wait_phase(bar(Y_FULL + m % NY), (m / NY) & 1, abort_flag) &&
+                         (KIND == kDKDV || wait_phase(bar(Z_FULL + m % NZ), (m / NZ) & 1, abort_flag)) &&
                          wait_phase(bar(DP_FREE), n & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    if (KIND == kDQ) issue_prod(sX, sY(m), s_col_of(m));
-                    issue_prod(sW, sZ(m), DP_COL);
+                    issue_prod(sX, sY(m), s_col_of(m));
+                    mma_commit(bar(S_FULL));
                     if (KIND == kDQ) {
-                        mma_commit(bar(ST_FULL));
+                        issue_prod(sW, sZ(m), dp_col_of(m));
+                        mma_commit(bar(DP_FULL));
                         mma_commit(bar(Z_EMPTY + m % NZ));
                     }
                 }
@@ -394,18 +418,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if (KIND == kDKDV) {
-                    // dV += P dO, then dK += dS Q; P and dS sit in the S columns
-                    issue_grad(G_COL, Cfg::kSCol0, sZ(n), n == 0);
-                    mma_commit(bar(Z_EMPTY + n % NZ));
-                    issue_grad(G_COL + D, Cfg::kSCol0 + 32, sY(n), n == 0);
+                    // dK += dS Q, then dV += P dO; P and dS sit in the S region of n
+                    issue_grad(G_COL + D, s_col_of(n) + 32, sY(n), n == 0);
                     mma_commit(bar(Y_EMPTY + n % NY));
+                    issue_grad(G_COL, s_col_of(n), sZ(n), n == 0);
+                    mma_commit(bar(Z_EMPTY + n % NZ));
                     if (more) {
-                        // S(n+1) overwrites the P and dS just read (those MMAs run first)
-                        ok = wait_phase(bar(Y_FULL + m % NY), (m / NY) & 1, abort_flag);
+                        // dP(n+1) takes the S region of n, read by the MMAs just issued
+                        ok = wait_phase(bar(Z_FULL + m % NZ), (m / NZ) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_prod(sX, sY(m), Cfg::kSCol0);
-                        mma_commit(bar(ST_FULL));
+                        issue_prod(sW, sZ(m), dp_col_of(m));
+                        mma_commit(bar(DP_FULL));
                     }
                 } else {
                     issue_grad(G_COL, s_col_of(n), sY(n), n == 0);  // dQ += dS K
@@ -432,41 +456,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int n = 0; n < n_all; ++n) {
             const int sub = (KIND == kDKDV) ? s_lo + n % n_sub : s_lo + n;
-            bool w = wait_phase(bar(ST_FULL), n & 1, abort_flag);
+            // kDKDV, phase 1: P from S (and the statistics) alone; dP comes later.
+            // kDQ: S and dP arrive together; both are copied and released at once.
+            bool w = wait_phase(bar(S_FULL), n & 1, abort_flag);
             if (KIND == kDKDV) w = w && wait_phase(bar(Y_FULL + n % NY), (n / NY) & 1, abort_flag);
+            else w = w && wait_phase(bar(DP_FULL), n & 1, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
             const uint32_t s_col = s_col_of(n) + wg * 64;
-            const uint32_t dp_col = DP_COL + wg * 64;
+            const uint32_t dp_col = dp_col_of(n) + wg * 64;
             uint32_t sr[64], dr[64];
             tmem_ld32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
             tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld32(lane_base + dp_col, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-            tmem_ld32(lane_base + dp_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+            if (KIND == kDQ) {
+                tmem_ld32(lane_base + dp_col, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+                tmem_ld32(lane_base + dp_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+            }
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(DP_FREE));
+            if (KIND == kDQ) {
+                tc_fence_before();
+                mbar_arrive(bar(DP_FREE));  // S and dP of n are in registers
+            }
             const int cbase = sub * kBwdSub + wg * 64;  // first column index (query or key)
             const float* st = stats + (n % NY) * 2 * kBwdSub + wg * 64;
+            uint64_t p2[32];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int c0 = cbase + h * 32;  // first column of this half
                 bool full;
                 if (KIND == kDKDV) full = bwd_all_visible<MASK>(c0, 32, r, 1, args);
                 else full = c0 + 32 <= args.Lk && bwd_all_visible<MASK>(r, 1, c0, 32, args);
-                uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int x = h * 32 + 2 * q;
-                    uint64_t nl2, dl2;
+                    uint64_t nl2;
                     if (KIND == kDKDV) {
                         const float2 nl = reinterpret_cast<const float2*>(st + h * 32)[q];
-                        const float2 dl = reinterpret_cast<const float2*>(st + kBwdSub + h * 32)[q];
                         nl2 = f2pack(nl.x, nl.y);
-                        dl2 = f2pack(dl.x, dl.y);
                     } else {
                         nl2 = nl2_row;
-                        dl2 = dl2_row;
                     }
                     float t0, t1;
                     f2unpack(fma2(f2pack(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), c2, nl2),
@@ -482,15 +510,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 p1 = 0.f;
                         }
                     }
+                    p2[h * 16 + q] = f2pack(p0, p1);
+                }
+            }
+            if (KIND == kDKDV) {
+                // Phase 2: dS = P (dP - delta) once dP is there.
+                w = wait_phase(bar(DP_FULL), n & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+                tc_fence_after();
+                tmem_ld32(lane_base + dp_col, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+                tmem_ld32(lane_base + dp_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(DP_FREE));  // S and dP of n are in registers
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int x = h * 32 + 2 * q;
+                    uint64_t dl2;
+                    if (KIND == kDKDV) {
+                        const float2 dl = reinterpret_cast<const float2*>(st + kBwdSub + h * 32)[q];
+                        dl2 = f2pack(dl.x, dl.y);
+                    } else {
+                        dl2 = dl2_row;
+                    }
+                    float p0, p1, d0, d1;
+                    f2unpack(p2[h * 16 + q], p0, p1);
                     if (KIND == kDKDV) pk[q] = pack2<BF16>(p0, p1);
-                    float d0, d1;
-                    f2unpack(mul2(f2pack(p0, p1),
+                    f2unpack(mul2(p2[h * 16 + q],
                                   sub2(f2pack(__uint_as_float(dr[x]), __uint_as_float(dr[x + 1])), dl2)),
                              d0, d1);
                     dk[q] = pack2<BF16>(d0, d1);
                 }
                 if (KIND == kDKDV) {
-                    // P at columns 64w + [0, 32), dS at 64w + [32, 64) of the S buffer: this
+                    // P at columns 64w + [0, 32), dS at 64w + [32, 64) of the S region: this
                     // warpgroup's own S columns, already copied to registers
                     tmem_st16(lane_base + s_col + h * 16, pk);
                     tmem_st16(lane_base + s_col + 32 + h * 16, dk);
