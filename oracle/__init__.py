@@ -73,6 +73,10 @@ def load(path: str | None = None):
         lib.oracle_attn_bwd_dkv_keys.argtypes = [_dp, _dp, _dp, _dp, _i64p, _i64, _dp, _dp, _dp,
                                                  _dp, _i64, _i64, _i64, _i64, _i64, _i64,
                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_paged_prefill.argtypes = [_dp, _dp, _dp, _i32p, _i32p, _i32p, _i64, _dp,
+                                                  _dp, _i64, _i64, _i64, _i64, _i64, _i64, _i64,
+                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_paged_prefill.restype = ctypes.c_int
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_probs,
                   lib.oracle_attn_paged, lib.oracle_attn_fwd_window, lib.oracle_attn_bwd,
                   lib.oracle_attn_bwd_dq_rows, lib.oracle_attn_bwd_dkv_keys):
@@ -244,3 +248,27 @@ def attn_bwd_dkv_keys(q, k, v, dout, keys, scale: float, causal: bool = False,
     _check(rc, "attn_bwd_dkv_keys")
     g = (torch.from_numpy(dk), torch.from_numpy(dv))
     return g + tuple(torch.from_numpy(a) for a in m) if m else g
+
+
+def attn_paged_prefill(q, k_cache, v_cache, block_table, seq_lens, scale: float,
+                       causal: bool = True, q_lens=None, threads: int | None = None, lib=None):
+    """Prefill over a paged cache. q[S,Hq,Lq,D]: each sequence's chunk of queries, its
+    last q_lens[s] positions (all Lq if q_lens is None); caches [NB,Hkv,bs,D];
+    block_table[S,MB]; seq_lens[S] -> (out[S,Hq,Lq,D], lse[S,Hq,Lq]) fp64. Rows past a
+    sequence's chunk come out as rows with no key (0, -inf)."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    bt = np.ascontiguousarray(torch.as_tensor(block_table).to(torch.int32).numpy())
+    sl = np.ascontiguousarray(torch.as_tensor(seq_lens).to(torch.int32).numpy())
+    ql = None if q_lens is None else np.ascontiguousarray(
+        torch.as_tensor(q_lens).to(torch.int32).numpy())
+    S, Hq, Lq, D = q.shape
+    NB, Hkv, bs, _ = kc.shape
+    MB = bt.shape[1] if bt.ndim == 2 else 0
+    out = np.zeros((S, Hq, Lq, D), np.float64)
+    lse = np.zeros((S, Hq, Lq), np.float64)
+    rc = (lib or load()).oracle_attn_paged_prefill(
+        _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt, _i32p), _ptr(sl, _i32p),
+        _ptr(ql, _i32p) if ql is not None else None, bs, _ptr(out), _ptr(lse), S, Hq, Hkv, Lq, D,
+        MB, NB, float(scale), int(bool(causal)), threads or default_threads())
+    _check(rc, "attn_paged_prefill")
+    return torch.from_numpy(out), torch.from_numpy(lse)

@@ -51,6 +51,11 @@
  *    section "FlashAttention-style attention and paged attention". Layout
  *    taken: cache[num_blocks][H_kv][block_size][D]; token t of sequence s is
  *    row t % block_size of physical block block_table[s][t / block_size].
+ *  - Prefill over a paged cache: the same page says the kernel translates every
+ *    position through the block table, and that long prefill is where the T x T
+ *    score matrix hurts. Reading taken: a chunk of q_len queries per sequence
+ *    occupies its last q_len positions (causal alignment bottom-right, as for
+ *    dense attention with Lq = q_len, Lk = seq_len).
  *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math, so
  * every operation is the IEEE double operation written here).
@@ -707,4 +712,99 @@ int oracle_attn_bwd_dkv_keys(const double* q, const double* k, const double* v,
     }
     free(lse); free(delta); free(absdo);
     return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Paged prefill: a chunk of queries per sequence over its paged cache.     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Each sequence s has seq_lens[s] tokens in the paged cache (resolved through
+ * block_table exactly as in oracle_attn_paged) and a chunk of q_lens[s] queries,
+ * which are its last q_lens[s] positions: query i sits at position
+ * seq_lens[s] - q_lens[s] + i, the bottom-right alignment of the dense causal mask
+ * (Lq = q_lens[s], Lk = seq_lens[s]). Without causal every query sees all
+ * seq_lens[s] keys. Rows i >= q_lens[s] of the [num_seqs, Hq, Lq, D] output are
+ * written as rows with no key (O = 0, lse = -inf).
+ */
+typedef struct {
+    const double *q, *kc, *vc;
+    const int32_t *block_table, *seq_lens, *q_lens;
+    double *out, *lse;
+    int64_t block_size, num_seqs, Hq, Hkv, Lq, D, max_blocks, num_blocks;
+    double scale;
+    int causal;
+    int64_t next;
+    int status;
+} paged_prefill_job;
+
+static void* paged_prefill_worker(void* arg) {
+    paged_prefill_job* J = (paged_prefill_job*)arg;
+    const int64_t cap = J->max_blocks * J->block_size;
+    double* Kd = (double*)malloc(sizeof(double) * (size_t)(cap * J->D + 1));
+    double* Vd = (double*)malloc(sizeof(double) * (size_t)(cap * J->D + 1));
+    double* s = (double*)malloc(sizeof(double) * (size_t)(cap + 1));
+    if (!Kd || !Vd || !s) {
+        __atomic_store_n(&J->status, ORACLE_ERR_NOMEM, __ATOMIC_RELAXED);
+        free(Kd); free(Vd); free(s);
+        return NULL;
+    }
+    const int64_t group = J->Hq / J->Hkv;
+    for (;;) {
+        int64_t u = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (u >= J->num_seqs * J->Hkv) break;
+        int64_t sq = u / J->Hkv, hkv = u % J->Hkv;
+        int64_t len = J->seq_lens[sq];
+        int64_t ql = J->q_lens ? J->q_lens[sq] : J->Lq;
+        /* Gather this sequence's keys and values in logical order. */
+        for (int64_t t = 0; t < len; ++t) {
+            int64_t phys = J->block_table[sq * J->max_blocks + t / J->block_size];
+            if (phys < 0 || phys >= J->num_blocks) {
+                __atomic_store_n(&J->status, ORACLE_ERR_INDEX, __ATOMIC_RELAXED);
+                len = 0;
+                break;
+            }
+            const int64_t row = ((phys * J->Hkv + hkv) * J->block_size + t % J->block_size) * J->D;
+            memcpy(Kd + t * J->D, J->kc + row, sizeof(double) * (size_t)J->D);
+            memcpy(Vd + t * J->D, J->vc + row, sizeof(double) * (size_t)J->D);
+        }
+        for (int64_t g = 0; g < group; ++g) {
+            const int64_t h = hkv * group + g;
+            for (int64_t i = 0; i < J->Lq; ++i) {
+                const int64_t id = (sq * J->Hq + h) * J->Lq + i;
+                double* o = J->out + id * J->D;
+                double* l = J->lse ? J->lse + id : NULL;
+                int64_t lo = 0, hi = 0; /* rows past the chunk see no key */
+                if (i < ql) visible_range(i, ql, len, J->causal, -1, -1, &lo, &hi);
+                attention_row(J->q + id * J->D, Kd, Vd, len, lo, hi, J->D, J->scale, s, o, l, NULL);
+            }
+        }
+    }
+    free(Kd); free(Vd); free(s);
+    return NULL;
+}
+
+/*
+ * q[num_seqs,Hq,Lq,D]; k_cache, v_cache [num_blocks,Hkv,block_size,D];
+ * block_table[num_seqs,max_blocks]; seq_lens[num_seqs]; q_lens[num_seqs] (NULL: all
+ * Lq); out[num_seqs,Hq,Lq,D]; lse[num_seqs,Hq,Lq] (may be NULL).
+ */
+int oracle_attn_paged_prefill(const double* q, const double* k_cache, const double* v_cache,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              const int32_t* q_lens, int64_t block_size, double* out,
+                              double* lse, int64_t num_seqs, int64_t Hq, int64_t Hkv, int64_t Lq,
+                              int64_t D, int64_t max_blocks, int64_t num_blocks, double scale,
+                              int causal, int nthreads) {
+    if (num_seqs < 0 || Hq < 1 || Hkv < 1 || Lq < 0 || D < 1 || block_size < 1 ||
+        max_blocks < 0 || num_blocks < 0 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        if (seq_lens[s] < 0 || seq_lens[s] > max_blocks * block_size) return ORACLE_ERR_INDEX;
+        if (q_lens && (q_lens[s] < 0 || q_lens[s] > Lq)) return ORACLE_ERR_INDEX;
+    }
+    paged_prefill_job J = {q, k_cache, v_cache, block_table, seq_lens, q_lens, out, lse,
+                           block_size, num_seqs, Hq, Hkv, Lq, D, max_blocks, num_blocks, scale,
+                           causal, 0, ORACLE_OK};
+    run_workers(paged_prefill_worker, &J, num_seqs * Hkv, nthreads);
+    return J.status;
 }

@@ -146,6 +146,12 @@ def pin_golden(lib=None):
         if ex["kind"] == "dense":
             o, l = oracle.attn_fwd(np.array(ex["q"]), np.array(ex["k"]), np.array(ex["v"]),
                                    ex["scale"], ex["causal"], lib=lib)
+        elif ex["kind"] == "paged_prefill":
+            o, l = oracle.attn_paged_prefill(np.array(ex["q"]), np.array(ex["k_cache"]),
+                                             np.array(ex["v_cache"]),
+                                             torch.tensor(ex["block_table"], dtype=torch.int32),
+                                             torch.tensor(ex["seq_lens"], dtype=torch.int32),
+                                             ex["scale"], ex["causal"], lib=lib)
         else:
             o, l = oracle.attn_paged(np.array(ex["q"]), np.array(ex["k_cache"]),
                                      np.array(ex["v_cache"]),
@@ -542,12 +548,45 @@ def pin_bwd_sensitivity(lib=None):
         close(mvr, mv.reshape(-1, 5)[keys])
 
 
+def pin_paged_prefill(lib=None):
+    """Paged prefill equals the dense oracle on the gathered cache (Lq = q_len, Lk =
+    seq_len, bottom-right causal), for every sequence and head; rows past a sequence's
+    chunk are empty rows; one query per sequence is the paged decode."""
+    g = torch.Generator().manual_seed(950)
+    S, Hq, Hkv, Lq, D, bs, MB = 3, 4, 2, 6, 5, 4, 5
+    NB = S * MB + 2
+    kc = rand((NB, Hkv, bs, D), 951)
+    vc = rand((NB, Hkv, bs, D), 952)
+    q = rand((S, Hq, Lq, D), 953)
+    bt = torch.randperm(NB, generator=g)[:S * MB].reshape(S, MB).to(torch.int32)
+    sl = torch.tensor([17, 6, 1], dtype=torch.int32)
+    ql = torch.tensor([6, 4, 1], dtype=torch.int32)
+    for causal in (True, False):
+        o, l = oracle.attn_paged_prefill(q, kc, vc, bt, sl, 0.6, causal, q_lens=ql, lib=lib)
+        for s_ in range(S):
+            n, m = int(sl[s_]), int(ql[s_])
+            t = torch.arange(n)
+            rows = bt[s_][t // bs].long()
+            K = torch.from_numpy(kc)[rows, :, t % bs].permute(1, 0, 2).unsqueeze(0).numpy()
+            V = torch.from_numpy(vc)[rows, :, t % bs].permute(1, 0, 2).unsqueeze(0).numpy()
+            od, ld = oracle.attn_fwd(q[s_:s_ + 1, :, :m], K, V, 0.6, causal, lib=lib)
+            close(o[s_:s_ + 1, :, :m], od)
+            close(l[s_:s_ + 1, :, :m], ld)
+            close(o[s_, :, m:], np.zeros((Hq, Lq - m, D)))
+            assert bool((l[s_, :, m:] == -math.inf).all())
+    o1, l1 = oracle.attn_paged_prefill(q[:, :, :1], kc, vc, bt, sl, 0.6, True, lib=lib)
+    od, ld = oracle.attn_paged(q[:, :, 0], kc, vc, bt, sl, 0.6, lib=lib)
+    close(o1[:, :, 0], od)
+    close(l1[:, :, 0], ld)
+
+
 PINS = [pin_brute_force, pin_golden, pin_probability_rows, pin_constant_values,
         pin_identical_keys, pin_argmax_limit, pin_causal_row0, pin_shift_invariance,
         pin_permutation_equivariance, pin_gqa_equals_repeat, pin_paged_equals_dense,
         pin_fully_masked_rows, pin_online_softmax, pin_split_combine, pin_window,
         pin_bwd_autograd, pin_bwd_finite_differences, pin_bwd_golden, pin_bwd_invariants,
-        pin_bwd_gqa_equals_repeat, pin_bwd_selected_outputs, pin_bwd_sensitivity]
+        pin_bwd_gqa_equals_repeat, pin_bwd_selected_outputs, pin_bwd_sensitivity,
+        pin_paged_prefill]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -613,13 +652,17 @@ MUTANTS = {
                          "for (d = 0; d < D; ++d) dot += doi[d] * K[j * D + d];\n        ds[j] = dot;"),
     "bwd_dq_uses_values": ("for (d = 0; d < D; ++d) dqi[d] += ds[j] * K[j * D + d];",
                            "for (d = 0; d < D; ++d) dqi[d] += ds[j] * V[j * D + d];"),
-    "bwd_gqa_heads_not_summed": ("for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            for (int64_t i = 0; i < J->Lq; ++i) {",
-                                 "for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            if (g) for (int64_t x = 0; x < J->Lk * J->D; ++x) dK[x] = dV[x] = 0.0;\n            for (int64_t i = 0; i < J->Lq; ++i) {"),
+    "bwd_gqa_heads_not_summed": ("for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            for (int64_t i = 0; i < J->Lq; ++i) {\n                const int64_t id = (b * J->Hq + h) * J->Lq + i;",
+                                 "for (int64_t g = 0; g < group; ++g) {\n            const int64_t h = hkv * group + g;\n            if (g) for (int64_t x = 0; x < J->Lk * J->D; ++x) dK[x] = dV[x] = 0.0;\n            for (int64_t i = 0; i < J->Lq; ++i) {\n                const int64_t id = (b * J->Hq + h) * J->Lq + i;"),
     "bwd_keys_lse_sign": ("exp(J->scale * dot - J->lse[g * J->Lq + i])",
                           "exp(J->scale * dot + J->lse[g * J->Lq + i])"),
     "bwd_keys_delta_dropped": ("pij * (dpv - J->delta[g * J->Lq + i])", "pij * dpv"),
     "bwd_keys_mask_ignored": ("if (j < lo || j >= hi) continue;\n                const int64_t id",
                               "const int64_t id"),
+    "paged_prefill_top_left": ("if (i < ql) visible_range(i, ql, len, J->causal, -1, -1, &lo, &hi);",
+                               "if (i < ql) visible_range(i, len, len, J->causal, -1, -1, &lo, &hi);"),
+    "paged_prefill_rows_past_chunk": ("int64_t lo = 0, hi = 0; /* rows past the chunk see no key */\n                if (i < ql)",
+                                      "int64_t lo = 0, hi = 0; /* rows past the chunk see no key */\n                if (1)"),
     "masked_row_nan": ("if (m == -INFINITY) { /* no visible key */",
                        "if (0) { /* no visible key */"),
 }
@@ -636,7 +679,7 @@ def mutant_results():
     try:
         pending = []
         for name, (old, new) in sorted(MUTANTS.items()):
-            if src.count(old) < 1:
+            if src.count(old) < 1:  # a shared pattern is planted everywhere it occurs
                 results[name] = None
                 continue
             c = os.path.join(tmp, name + ".c")
