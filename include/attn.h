@@ -174,7 +174,9 @@ size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D,
  *   lse          [num_seqs, H_q] fp32, written if non-NULL
  *
  *   block_size must be 16; H_q / H_kv <= 16; D in {64, 128}. Entries of
- *   block_table past ceil(seq_lens[s] / 16) are never read. An entry outside
+ *   block_table past ceil(seq_lens[s] / 16) are never read. The cache rows of a
+ *   sequence's last block past seq_lens[s] are read but weigh nothing; they must hold
+ *   finite values (a NaN there would reach the output through 0 * NaN). An entry outside
  *   [0, num_blocks), or a seq_len past the table, is skipped on the device and
  *   reported as ATTN_ERR_BAD_INDEX by attn_get_device_status(). A sequence of
  *   length 0 gets O = 0 and lse = -inf. num_seqs == 0 is a no-op (every
@@ -283,6 +285,48 @@ attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const
                               int causal, int window_left, int window_right,
                               attn_dtype_t dtype, void* workspace, size_t workspace_bytes,
                               void* stream);
+
+/*
+ * attn_fwd_paged_prefill -- prefill attention over a paged KV cache: each sequence's
+ * chunk of queries attends to its keys in the cache, resolved block by block through
+ * the block table inside the kernel ("Fast attention kernels and operator fusion"
+ * (the-ai.news), section on FlashAttention-style and paged attention: long prefill,
+ * and a paged cache whose positions the kernel translates through the table). Runs
+ * the tcgen05 prefill kernel of attn_fwd with its K/V tiles gathered from 16-token
+ * blocks.
+ *
+ *   q            [num_seqs, H_q, Lq, D] dtype, strides as attn_fwd_strided (q_strides
+ *                NULL: contiguous); sequence s's chunk is its first q_lens[s] rows
+ *   k_cache      [num_blocks, H_kv, block_size, D] dtype, contiguous
+ *   v_cache      [num_blocks, H_kv, block_size, D] dtype, contiguous
+ *   block_table  [num_seqs, max_blocks_per_seq] int32, as attn_fwd_paged
+ *   seq_lens     [num_seqs] int32: keys of sequence s, 0 <= seq_lens[s] <=
+ *                max_blocks_per_seq * block_size (they include the chunk's own keys)
+ *   q_lens       [num_seqs] int32, 0 <= q_lens[s] <= Lq, or NULL for all Lq
+ *   out          [num_seqs, H_q, Lq, D] dtype, written (every element; out_strides as
+ *                q_strides)
+ *   lse          [num_seqs, H_q, Lq] fp32, contiguous, written if non-NULL
+ *
+ *   The chunk's queries are the sequence's last q_lens[s] positions: with causal != 0,
+ *   query i sees keys j <= i + seq_lens[s] - q_lens[s] (attn_fwd's bottom-right mask
+ *   with Lq = q_lens[s], Lk = seq_lens[s]); without it every query sees all
+ *   seq_lens[s] keys. Rows i >= q_lens[s], and rows that see no key, get O = 0 and
+ *   lse = -inf. block_size must be 16; H_q a multiple of H_kv; D in {64, 128}.
+ *   Table entries past ceil(seq_lens[s] / 16) are never read. A length out of range is
+ *   clamped, an entry outside [0, num_blocks) is replaced by block 0, and both are
+ *   reported as ATTN_ERR_BAD_INDEX by attn_get_device_status(). The cache rows of a
+ *   sequence's last block past seq_lens[s] are read but weigh nothing; they must hold
+ *   finite values (a NaN there would reach the output through 0 * NaN).
+ *   num_seqs == 0 or Lq == 0 is a no-op (pointers may be NULL).
+ */
+attn_status_t attn_fwd_paged_prefill(const void* q, const attn_strides_t* q_strides,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens,
+                                     const int32_t* q_lens, int block_size, void* out,
+                                     const attn_strides_t* out_strides, float* lse, int num_seqs,
+                                     int H_q, int H_kv, int Lq, int D, int max_blocks_per_seq,
+                                     int num_blocks, float scale, int causal, attn_dtype_t dtype,
+                                     void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* attn_error_string(attn_status_t status);

@@ -246,3 +246,25 @@ def test_attn_fwd_strided_validation():
     assert call(ks=S(-8, 512, 64), B=2) == -1                    # negative stride of a used dim
     assert call(os_=S(1 << 38, 512, 64), B=2) == -1              # oversized
     assert call(qs=S(0, 0, 0), B=1, Hq=1, Hkv=1, Lq=1, D=96) == -2  # unused strides; D refused
+
+
+def test_attn_fwd_paged_prefill_validation():
+    lib = ta.load()
+
+    def call(**kw):
+        a = dict(q=P, kc=P, vc=P, bt=P, sl=P, ql=None, bs=16, out=P, lse=P, S=2, Hq=4, Hkv=2,
+                 Lq=64, D=128, MB=8, NB=16, scale=0.088, causal=1, dtype=1)
+        a.update(kw)
+        return lib.attn_fwd_paged_prefill(a["q"], None, a["kc"], a["vc"], a["bt"], a["sl"], a["ql"],
+                                          a["bs"], a["out"], None, a["lse"], a["S"], a["Hq"],
+                                          a["Hkv"], a["Lq"], a["D"], a["MB"], a["NB"], a["scale"],
+                                          a["causal"], a["dtype"], None)
+    assert call(sl=None) == -1
+    assert call(bt=None) == -1
+    assert call(Hq=3) == -1
+    assert call(NB=0) == -1
+    assert call(bs=32) == -2
+    assert call(D=80) == -2
+    assert call(bt=P + 2) == -3
+    assert call(ql=P + 1) == -3
+    assert call(S=0, q=None, out=None) == 0      # nothing to do: NULL pointers allowed

@@ -44,6 +44,8 @@ SIGNATURES = {
                              _vp]),
     "attn_fwd_strided": (_i, [_vp, _sp, _vp, _sp, _vp, _sp, _vp, _sp, _vp, _i, _i, _i, _i, _i, _i,
                               _f, _i, _i, _i, _i, _vp]),
+    "attn_fwd_paged_prefill": (_i, [_vp, _sp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sp, _vp, _i, _i,
+                                    _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                             _i, _vp, _sz, _vp]),
@@ -269,6 +271,39 @@ def fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                S, Hq, Hkv, D, MB, NB, float(scale), _dtype_code(q.dtype), ws_ptr,
                                ws_n, _stream(stream))
     _check(rc, "attn_fwd_paged")
+    return out, lse
+
+
+def fwd_paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      block_table: torch.Tensor, seq_lens: torch.Tensor,
+                      q_lens: torch.Tensor | None = None, causal: bool = True,
+                      scale: float | None = None, out: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Prefill over a paged cache. q [S,Hq,Lq,D] (any view with contiguous D): sequence
+    s's chunk is its first q_lens[s] rows (all Lq if q_lens is None), at the sequence's
+    last positions; caches [NB,Hkv,16,D]; block_table [S,MB] int32; seq_lens [S] int32
+    (keys, including the chunk's). Returns (out [S,Hq,Lq,D], lse [S,Hq,Lq])."""
+    S, Hq, Lq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("cache shape mismatch")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32 or \
+            (q_lens is not None and q_lens.dtype != torch.int32):
+        raise TypeError("block_table, seq_lens and q_lens must be int32")
+    MB = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((S, Hq, Lq), dtype=torch.float32, device=q.device)
+    rc = load().attn_fwd_paged_prefill(
+        q.data_ptr(), _strides(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_table, "block_table"), _dev(seq_lens, "seq_lens"),
+        _dev(q_lens, "q_lens") if q_lens is not None else None, bs, out.data_ptr(),
+        _strides(out, "out"), _dev(lse, "lse") if lse is not None else None, S, Hq, Hkv, Lq, D, MB,
+        NB, float(scale), int(bool(causal)), _dtype_code(q.dtype), _stream(stream))
+    _check(rc, "attn_fwd_paged_prefill")
     return out, lse
 
 

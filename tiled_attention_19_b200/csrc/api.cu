@@ -144,10 +144,10 @@ __global__ void zero_rows_kernel(uint16_t* out, long long sb, long long sh, long
 }
 
 // ------------------------------------------------------------------ launchers
-template <int D, bool BF16, int MASK>
+template <int D, bool BF16, int MASK, bool PAGED = false>
 attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const PrefillArgs& args, int planes, cudaStream_t stream) {
-    auto kern = attn::prefill_fwd_kernel<D, BF16, MASK>;
+    auto kern = attn::prefill_fwd_kernel<D, BF16, MASK, PAGED>;
     constexpr int smem = PrefillCfg<D>::kSmemBytes;
     static std::once_flag once;
     static attn_status_t setup = ATTN_OK;
@@ -468,9 +468,109 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
                 : dispatch_bwd<128, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
 }
 
+// Prefill over a paged cache: the dense forward kernel with its K/V tiles gathered
+// block by block through the table.
+attn_status_t paged_prefill(const void* q, const attn_strides_t* q_st, const void* k_cache,
+                            const void* v_cache, const int32_t* block_table,
+                            const int32_t* seq_lens, const int32_t* q_lens, int block_size,
+                            void* out, const attn_strides_t* o_st, float* lse, int num_seqs,
+                            int H_q, int H_kv, int Lq, int D, int max_blocks, int num_blocks,
+                            float scale, int causal, attn_dtype_t dtype, void* stream_) {
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || max_blocks < 0 || num_blocks < 0)
+        return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (Lq > kMaxSeq || static_cast<long long>(max_blocks) * attn::kPageSize > kMaxSeq)
+        return ATTN_ERR_UNSUPPORTED;
+    const long long planes_q = static_cast<long long>(num_seqs) * H_q;
+    if (planes_q > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || Lq == 0) return ATTN_OK;  // nothing to write; pointers may be NULL
+    if (q == nullptr || out == nullptr || seq_lens == nullptr ||
+        (max_blocks > 0 && (block_table == nullptr || k_cache == nullptr || v_cache == nullptr)))
+        return ATTN_ERR_INVALID;
+    if (max_blocks > 0 && num_blocks < 1) return ATTN_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(q_lens, 4) ||
+        (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    Strides sq, so;
+    attn_status_t st = take_strides(q_st, num_seqs, H_q, Lq, D, &sq);
+    if (st == ATTN_OK) st = take_strides(o_st, num_seqs, H_q, Lq, D, &so);
+    if (st != ATTN_OK) return st;
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool bf16 = dtype == ATTN_BF16;
+    if (max_blocks == 0) {  // every sequence is empty: O = 0, lse = -inf
+        const long long rows = planes_q * Lq;
+        zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(out), so.b, so.h, so.l,
+                                                   H_q, Lq, D, rows);
+        if (lse != nullptr)
+            attn::fill_empty_kernel<true><<<1184, 256, 0, stream>>>(nullptr, lse, 0,
+                                                                    static_cast<size_t>(rows));
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
+
+    alignas(64) CUtensorMap tq, tk, tv;
+    const long long cache_rows = static_cast<long long>(num_blocks) * H_kv * attn::kPageSize;
+    if (!encode_strided_map(&tq, q, bf16, D, Lq, H_q, num_seqs, sq, attn::kBM) ||
+        !encode_cache_map(&tk, k_cache, bf16, D, cache_rows) ||
+        !encode_cache_map(&tv, v_cache, bf16, D, cache_rows))
+        return ATTN_ERR_CUDA;
+    PrefillArgs args{};
+    args.out = out;
+    args.out_sb = so.b;
+    args.out_sh = so.h;
+    args.out_sl = so.l;
+    args.lse = lse;
+    args.Hq = H_q;
+    args.Hkv = H_kv;
+    args.group = H_q / H_kv;
+    args.Lq = Lq;
+    args.Lk = max_blocks * attn::kPageSize;  // replaced per sequence by seq_lens[b]
+    args.n_q_blocks = (Lq + 2 * attn::kBM - 1) / (2 * attn::kBM);
+    args.win_left = -1;
+    args.win_right = causal ? 0 : -1;
+    args.scale_log2 = scale * attn::kLog2e;
+    args.block_table = block_table;
+    args.seq_lens = seq_lens;
+    args.q_lens = q_lens;
+    args.max_blocks = max_blocks;
+    args.num_blocks = num_blocks;
+    const int planes = static_cast<int>(planes_q);
+    if (D == 64) {
+        if (bf16)
+            return causal ? launch_prefill<64, true, attn::kMaskCausal, true>(tq, tk, tv, args, planes, stream)
+                          : launch_prefill<64, true, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
+        return causal ? launch_prefill<64, false, attn::kMaskCausal, true>(tq, tk, tv, args, planes, stream)
+                      : launch_prefill<64, false, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
+    }
+    if (bf16)
+        return causal ? launch_prefill<128, true, attn::kMaskCausal, true>(tq, tk, tv, args, planes, stream)
+                      : launch_prefill<128, true, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
+    return causal ? launch_prefill<128, false, attn::kMaskCausal, true>(tq, tk, tv, args, planes, stream)
+                  : launch_prefill<128, false, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
+}
+
 }  // namespace
 
 extern "C" {
+
+attn_status_t attn_fwd_paged_prefill(const void* q, const attn_strides_t* q_strides,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* block_table, const int32_t* seq_lens,
+                                     const int32_t* q_lens, int block_size, void* out,
+                                     const attn_strides_t* out_strides, float* lse, int num_seqs,
+                                     int H_q, int H_kv, int Lq, int D, int max_blocks_per_seq,
+                                     int num_blocks, float scale, int causal, attn_dtype_t dtype,
+                                     void* stream) {
+    return paged_prefill(q, q_strides, k_cache, v_cache, block_table, seq_lens, q_lens,
+                         block_size, out, out_strides, lse, num_seqs, H_q, H_kv, Lq, D,
+                         max_blocks_per_seq, num_blocks, scale, causal, dtype, stream);
+}
 
 size_t attn_bwd_workspace_size(int B, int H_q, int Lq) {
     if (B < 0 || H_q < 1 || Lq < 0) return 0;

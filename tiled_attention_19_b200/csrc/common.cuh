@@ -71,6 +71,8 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
     }
 }
 
+constexpr int kPageSize = 16;  // tokens per block of a paged KV cache
+
 // Mask modes, fixed at compile time so the common cases carry no window arithmetic.
 enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
 

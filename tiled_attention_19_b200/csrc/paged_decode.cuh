@@ -34,7 +34,6 @@
 
 namespace attn {
 
-constexpr int kPageSize = 16;
 constexpr int kMaxGroup = 16;
 constexpr int kDecConsumers = 4;                      // consumer warps
 constexpr int kDecThreads = (kDecConsumers + 1) * 32;  // + the producer warp
@@ -104,15 +103,6 @@ inline PagedLayout paged_layout(int num_seqs, int Hq, int Hkv, int D, int max_bl
 }
 
 // 2-D TMA load (x = column, y = row) into shared memory, completion counted on `bar`.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x,
-                                            int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(tmap), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])

@@ -90,6 +90,13 @@ struct PrefillArgs {
     int win_left;      // band: keys >= i' - win_left visible (-1: unbounded)
     int win_right;     // band: keys <= i' + win_right visible (-1: unbounded; causal: 0)
     float scale_log2;  // scale * log2(e)
+    // Paged keys (prefill over a paged cache): K and V of sequence b are rows
+    // (block_table[b][t / 16] * Hkv + h_kv) * 16 + t % 16 of the caches, seq_lens[b] keys;
+    // its chunk of queries is the first q_lens[b] rows (all Lq if q_lens is NULL).
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    const int32_t* q_lens;
+    int max_blocks, num_blocks;
 };
 
 // First and one-past-last visible key of query row i (empty if hi <= lo).
@@ -136,7 +143,7 @@ __device__ __forceinline__ void key_tiles_for(int row0, const PrefillArgs& a, in
     t1 = last / kBN + 1;
 }
 
-template <int D, bool BF16, int MASK>
+template <int D, bool BF16, int MASK, bool PAGED>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -177,17 +184,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int b = bh / args.Hq;
     const int hkv = h / args.group;  // grouped-query head mapping
     const int q0 = qb * 2 * kBM;
+    // The lengths the masks see: the problem's, or with paged keys the sequence's own
+    // (seq_lens[b] keys, q_lens[b] queries at its last positions). Out-of-range values
+    // are clamped and reported.
+    PrefillArgs a = args;
+    if constexpr (PAGED) {
+        int len = args.seq_lens[b];
+        const int cap = args.max_blocks * kPageSize;
+        int ql = args.q_lens != nullptr ? args.q_lens[b] : args.Lq;
+        if (len < 0 || len > cap || ql < 0 || ql > args.Lq) {
+            if (threadIdx.x == 0) report_status(ATTN_ERR_BAD_INDEX);
+            len = min(max(len, 0), cap);
+            ql = min(max(ql, 0), args.Lq);
+        }
+        a.Lk = len;
+        a.Lq = ql;
+    }
     // key-tile ranges of the two query tiles and of the CTA (their union, no gaps:
     // the band edges are monotone in the row)
     int a0 = 0, b0, a1 = 0, b1;
     if constexpr (MASK == kMaskWindow) {
-        key_tiles_for<MASK>(q0, args, a0, b0);
-        key_tiles_for<MASK>(q0 + kBM, args, a1, b1);
+        key_tiles_for<MASK>(q0, a, a0, b0);
+        key_tiles_for<MASK>(q0 + kBM, a, a1, b1);
     } else {  // every query tile starts at key tile 0
         int unused;
-        key_tiles_for<MASK>(q0, args, unused, b0);
-        key_tiles_for<MASK>(q0 + kBM, args, unused, b1);
+        key_tiles_for<MASK>(q0, a, unused, b0);
+        key_tiles_for<MASK>(q0 + kBM, a, unused, b1);
     }
+    if (PAGED && q0 >= a.Lq) a0 = b0 = a1 = b1 = 0;  // every row past the sequence's chunk
     const int jlo = (MASK != kMaskWindow) ? 0 : ((b0 > a0) ? a0 : a1);
     const int jhi = max(b0, b1);
     const int n_all = (b1 > a1 || b0 > a0) ? jhi - jlo : 0;  // key tiles this CTA loads
@@ -240,22 +264,57 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, h, b);
                 tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, h, b);
             }
+            constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
             for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile jlo + n
                 const int j = jlo + n;
                 const int sk = n % NK, sv = n % NV;
+                // Paged keys: the tile's rows come from kBlocks cache blocks; a block past
+                // the sequence loads its first block instead (finite rows, masked), and an
+                // entry outside the pool is reported and replaced by block 0.
+                int rows[PAGED ? kBlocks : 1];
+                if constexpr (PAGED) {
+                    const int32_t* tbl = args.block_table + static_cast<size_t>(b) * args.max_blocks;
+                    const int nblk = (a.Lk + kPageSize - 1) / kPageSize;
+#pragma unroll
+                    for (int k = 0; k < kBlocks; ++k) {
+                        const int bi = j * kBlocks + k;
+                        int e = __ldg(tbl + (bi < nblk ? bi : 0));
+                        if (e < 0 || e >= args.num_blocks) {
+                            report_status(ATTN_ERR_BAD_INDEX);
+                            e = 0;
+                        }
+                        rows[k] = (e * args.Hkv + hkv) * kPageSize;
+                    }
+                }
                 if (n >= NK && !wait_phase(bar(K_EMPTY + sk), ((n / NK) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_4d(sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_k,
-                                bar(K_FULL + sk), c * 64, j * kBN, hkv, b);
+                for (int c = 0; c < Cfg::kChunks; ++c) {
+                    const uint32_t dst = sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes;
+                    if constexpr (PAGED) {
+#pragma unroll
+                        for (int k = 0; k < kBlocks; ++k)
+                            tma_load_2d(dst + k * kPageSize * 128, &tm_k, bar(K_FULL + sk), c * 64,
+                                        rows[k]);
+                    } else {
+                        tma_load_4d(dst, &tm_k, bar(K_FULL + sk), c * 64, j * kBN, hkv, b);
+                    }
+                }
                 k_issued = n + 1;
                 if (n >= NV && !wait_phase(bar(V_EMPTY + sv), ((n / NV) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(V_FULL + sv), Cfg::kTileBytes);
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c)
-                    tma_load_4d(sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes, &tm_v,
-                                bar(V_FULL + sv), c * 64, j * kBN, hkv, b);
+                for (int c = 0; c < Cfg::kChunks; ++c) {
+                    const uint32_t dst = sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes;
+                    if constexpr (PAGED) {
+#pragma unroll
+                        for (int k = 0; k < kBlocks; ++k)
+                            tma_load_2d(dst + k * kPageSize * 128, &tm_v, bar(V_FULL + sv), c * 64,
+                                        rows[k]);
+                    } else {
+                        tma_load_4d(dst, &tm_v, bar(V_FULL + sv), c * 64, j * kBN, hkv, b);
+                    }
+                }
                 v_issued = n + 1;
             }
         }
@@ -386,12 +445,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t o_col = tile == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
         const float c = args.scale_log2;
         int row_lo, row_hi;  // this row's visible keys [row_lo, row_hi)
-        row_keys<MASK>(row, args, row_lo, row_hi);
+        row_keys<MASK>(row, a, row_lo, row_hi);
         // band edges of the tile: the largest first key and the smallest end
         const int tile_row0 = q0 + tile * kBM;
         int edge_lo, edge_hi, unused;
-        row_keys<MASK>(min(tile_row0 + kBM - 1, args.Lq - 1), args, edge_lo, unused);
-        row_keys<MASK>(tile_row0, args, unused, edge_hi);
+        row_keys<MASK>(min(tile_row0 + kBM - 1, a.Lq - 1), a, edge_lo, unused);
+        row_keys<MASK>(tile_row0, a, unused, edge_hi);
         float m_ref = -INFINITY;  // reference max, log2 units
         float l = 0.f;            // running sum of 2^(s*c - m_ref)
         bool ok = true;
@@ -412,7 +471,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int x = 0; x < kBN; ++x) s[x] = __uint_as_float(sr[x]);
 
             const int kbase = j * kBN;
-            const bool need_mask = (kbase + kBN > args.Lk) ||
+            const bool need_mask = (kbase + kBN > a.Lk) ||
                                    (MASK != kMaskNone && (kbase < edge_lo || kbase + kBN > edge_hi));
             if (need_mask) {
                 const int lo = row_lo - kbase, hi = row_hi - kbase;
@@ -478,7 +537,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (ok) {
             // ------------------------------------------------------------ epilogue
-            const bool has = l > 0.f;
+            // rows past a paged sequence's chunk are written as rows with no key
+            const bool real = !PAGED || row < a.Lq;
+            const bool has = real && l > 0.f;
             const float inv_l = has ? 1.f / l : 0.f;
             uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) + b * args.out_sb +
                                 h * args.out_sh + static_cast<long long>(row) * args.out_sl;
@@ -488,6 +549,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if (n_kv > 0) {
                     tmem_ld32(lane_base + o_col + d0, o);
                     tmem_wait_ld();
+                    if (!has) {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) o[x] = 0u;
+                    }
                 } else {
 #pragma unroll
                     for (int x = 0; x < 32; ++x) o[x] = 0u;
