@@ -8,9 +8,11 @@ prefill kernel's device time; the decode's HBM GB/s is reported beside it. Both 
 are timed with CUDA events on the stream they run on. Inputs rotate over enough copies
 that every step reads data that is not in L2.
 
-After the step's timed region, the backward pass of the same prefill workload (attn_bwd)
-is timed on its own and reported in the line's ``backward`` object (--no-backward skips
-it); it is not part of ``value``.
+After the step's timed region, two more calls on the same prefill workload are timed on
+their own and reported beside ``value`` (not part of it): the backward pass (attn_bwd,
+the ``backward`` object; --no-backward skips it) and the same prefill with K/V read
+through a paged cache (attn_fwd_paged_prefill, the ``paged_prefill`` object;
+--no-paged-prefill skips it).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -267,6 +269,12 @@ def run_ours(args, ws, rank, local):
         bwd_ms = measure_backward(w, ta, stream, device, steps=max(3, min(100, args.steps)),
                                   warmup=args.warmup, ws=ws, window=args.window)
 
+    pp_ms = None
+    if args.paged_prefill and do_pre and args.window is None and PREFILL.Lq == PREFILL.Lk \
+            and PREFILL.Lk % 16 == 0:
+        pp_ms = measure_paged_prefill(w, ta, stream, device, steps=max(3, min(300, args.steps)),
+                                      warmup=args.warmup, ws=ws)
+
     if args.e2e:
         e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)), window=args.window)
     else:
@@ -354,6 +362,24 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": (int(do_pre) + int(do_dec)) * args.steps,
         "clocks": clocks.summary(),
     }
+    if pp_ms is not None:
+        pp_tf = job_rate(w.prefill_flops, pp_ms, ws, 1e12) / ws
+        line["paged_prefill"] = {
+            "what": "attn_fwd_paged_prefill on the prefill workload with K/V scattered over a "
+                    "paged cache (16-token blocks, seeded permutation), the whole sequence as "
+                    "the chunk",
+            "kernel": f"prefill_fwd_kernel<{PREFILL.D},paged>",
+            "value": r2(pp_tf * ws, 2),
+            "unit": "TFLOP/s",
+            "bound": "tensor",
+            "achieved": r2(pp_tf, 2),
+            "peak": pk_t,
+            "frac": r2(pp_tf / pk_t, 4),
+            "vs_dense": r2(pre_avg / pp_ms, 4),
+            "avg_call_ms": round(pp_ms, 5),
+            "steps": max(3, min(300, args.steps)),
+            "gpu_launches": max(3, min(300, args.steps)),
+        }
     if bwd_ms is not None:
         bwd_flops = 2.5 * w.prefill_flops
         bwd_tf = job_rate(bwd_flops, bwd_ms, ws, 1e12) / ws
@@ -421,6 +447,53 @@ def measure_backward(w, ta, stream, device, steps: int, warmup: int, ws: int, wi
     return reduce_max(ms, ws, device)
 
 
+def measure_paged_prefill(w, ta, stream, device, steps: int, warmup: int, ws: int):
+    """The same prefill through a paged cache (attn_fwd_paged_prefill), timed on its own:
+    each input copy's K and V are cut into 16-token blocks and scattered over the pool by
+    one seeded permutation; the chunk is the whole sequence. Returns ms per call."""
+    B, H, L, D = PREFILL.B, PREFILL.Hkv, PREFILL.Lk, PREFILL.D
+    nblk = L // 16
+    g = torch.Generator().manual_seed(PREFILL.seed + 17)
+    perm = torch.randperm(B * nblk, generator=g).to(device)
+    table = perm.view(B, nblk).to(torch.int32)
+    seq_lens = torch.full((B,), L, dtype=torch.int32, device=device)
+    sets = []
+    for p in w.pf:
+        caches = []
+        for t in (p["k"], p["v"]):
+            blocks = t.view(B, H, nblk, 16, D).permute(0, 2, 1, 3, 4).reshape(B * nblk, H, 16, D)
+            c = torch.empty((B * nblk, H, 16, D), dtype=t.dtype, device=t.device)
+            c[perm] = blocks
+            caches.append(c)
+        sets.append((p["q"], caches[0], caches[1]))
+    out = torch.empty_like(w.pf[0]["q"])
+    lse = torch.empty(B, PREFILL.Hq, PREFILL.Lq, device=device)
+
+    def call(i):
+        q, kc, vc = sets[i % len(sets)]
+        ta.fwd_paged_prefill(q, kc, vc, table, seq_lens, causal=PREFILL.causal,
+                             scale=PREFILL.scale, out=out, lse=lse, stream=stream)
+
+    for i in range(warmup):
+        call(i)
+    torch.cuda.synchronize()
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set by the paged-prefill warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        call(warmup + i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set during the paged-prefill timing")
+    return reduce_max(sum(a.elapsed_time(b) for a, b in ev) / steps, ws, device)
+
+
 def measure_e2e(w, ta, stream, device, steps: int, window=None):
     """Same metric through the public API with host buffers: H2D of the step's inputs
     from pinned memory, the call, D2H of its outputs, all inside the timed region."""
@@ -477,17 +550,28 @@ def oracle_sample(seconds: float):
         g = torch.Generator().manual_seed(7)
         heads = torch.randint(0, PREFILL.Hq, (n,), generator=g)
         pos = torch.randint(0, L, (n,), generator=g)
-        return (heads * L + pos).tolist(), int((pos + 1).sum())
+        if PREFILL.causal:
+            vis = torch.clamp(pos + 1 + (PREFILL.Lk - PREFILL.Lq), min=0, max=PREFILL.Lk)
+        else:
+            vis = torch.full_like(pos, PREFILL.Lk)
+        return (heads * L + pos).tolist(), int(vis.sum())
 
-    # calibrate, then size the sample to about `seconds` of prefill work
-    rows, keys = rows_for(64)
-    t = time.perf_counter()
-    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, True, threads)
-    dt = time.perf_counter() - t
-    n = int(max(64, min(200000, 64 * (0.7 * seconds) / max(dt, 1e-3))))
+    # calibrate on samples that double until one takes a tenth of the budget, then size
+    # the sample to about `seconds` of prefill work
+    n = 64
+    while True:
+        rows, keys = rows_for(n)
+        t = time.perf_counter()
+        oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, PREFILL.causal,
+                             threads)
+        dt = time.perf_counter() - t
+        if dt >= 0.1 * seconds or n >= 100000:
+            break
+        n *= 2
+    n = int(max(64, min(400000, n * (0.9 * seconds) / max(dt, 1e-3))))
     rows, keys = rows_for(n)
     t = time.perf_counter()
-    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, True, threads)
+    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, PREFILL.causal, threads)
     t_pre = time.perf_counter() - t
     flops = 4.0 * D * keys
     t = time.perf_counter()
@@ -557,6 +641,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false",
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--no-paged-prefill", dest="paged_prefill", action="store_false",
+                    help="skip the separately timed paged-cache prefill of the prefill workload")
     ap.add_argument("--no-backward", dest="backward", action="store_false",
                     help="skip the separately timed backward pass of the prefill workload")
     ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",
