@@ -287,6 +287,30 @@ attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const
                               void* stream);
 
 /*
+ * attn_fwd_fp8 -- dense attention forward on 8-bit inputs: q, k and v in FP8 E4M3, the
+ * tensor-core products in 8 bits (tcgen05 kind::f8f6f4), softmax and accumulation in
+ * fp32, O in bf16 ("Flash Attention" skill page (hermes-agent-app.ru), Scenario 3: the
+ * FP8 forward of FlashAttention-3, for maximum performance, on inputs cast to
+ * float8_e4m3fn; forward only).
+ *
+ *   q, k, v  e4m3 bytes, shapes and strides as attn_fwd_strided (strides in elements =
+ *            bytes, multiples of 16); the values they stand for are q * descale_q,
+ *            k * descale_k and v * descale_v (pass 1 for plain casts)
+ *   out      [B, H_q, Lq, D] bf16, strides as attn_fwd_strided; lse as attn_fwd
+ *
+ *   The attention weights P are rounded to e4m3 before P.V (relative error up to 2^-4
+ *   per weight; the normaliser and lse use the unrounded fp32 weights). D must be 128;
+ *   causal as attn_fwd (no window). scale and the three descale factors must be finite
+ *   and > 0. Other arguments, results and errors as attn_fwd_strided.
+ */
+attn_status_t attn_fwd_fp8(const void* q, const attn_strides_t* q_strides, const void* k,
+                           const attn_strides_t* k_strides, const void* v,
+                           const attn_strides_t* v_strides, void* out,
+                           const attn_strides_t* out_strides, float* lse, int B, int H_q, int H_kv,
+                           int Lq, int Lk, int D, float scale, float descale_q, float descale_k,
+                           float descale_v, int causal, void* stream);
+
+/*
  * attn_fwd_paged_prefill -- prefill attention over a paged KV cache: each sequence's
  * chunk of queries attends to its keys in the cache, resolved block by block through
  * the block table inside the kernel ("Fast attention kernels and operator fusion"

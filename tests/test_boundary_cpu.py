@@ -268,3 +268,19 @@ def test_attn_fwd_paged_prefill_validation():
     assert call(bt=P + 2) == -3
     assert call(ql=P + 1) == -3
     assert call(S=0, q=None, out=None) == 0      # nothing to do: NULL pointers allowed
+
+
+def test_attn_fwd_fp8_validation():
+    lib = ta.load()
+    S = ta.Strides
+
+    def call(qs=None, D=128, scale=0.088, dq=1.0, dk=1.0, dv=1.0, **kw):
+        a = fwd_args(**kw)
+        return lib.attn_fwd_fp8(a["q"], qs, a["k"], None, a["v"], None, a["out"], None, a["lse"],
+                                a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"], D, scale, dq, dk, dv,
+                                a["causal"], None)
+    assert call(D=64) == -2                        # 8-bit path: D = 128 only
+    assert call(dv=0.0) == -1
+    assert call(dq=float("nan")) == -1
+    assert call(q=None) == -1
+    assert call(qs=S(16 * 128, 8 * 128, 136)) == -3  # 136-byte rows: not a multiple of 16

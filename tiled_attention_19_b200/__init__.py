@@ -46,6 +46,8 @@ SIGNATURES = {
                               _f, _i, _i, _i, _i, _vp]),
     "attn_fwd_paged_prefill": (_i, [_vp, _sp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _sp, _vp, _i, _i,
                                     _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_fwd_fp8": (_i, [_vp, _sp, _vp, _sp, _vp, _sp, _vp, _sp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                          _f, _f, _f, _i, _vp]),
     "attn_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                             _i, _vp, _sz, _vp]),
@@ -215,6 +217,34 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                                     _dev(workspace, "workspace"), ws_n, _stream(stream))
         _check(rc, "attn_bwd_window")
     return dq, dk, dv
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+            scale: float | None = None, descale=(1.0, 1.0, 1.0), out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Attention on e4m3 inputs (torch.float8_e4m3fn views [B,H,L,D] with contiguous D);
+    the values are q*descale[0], k*descale[1], v*descale[2]. Returns (out bf16, lse)."""
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if not all(t.dtype == torch.float8_e4m3fn for t in (q, k, v)):
+        raise TypeError("q, k, v must be float8_e4m3fn")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Hq, Lq, D), dtype=torch.bfloat16, device=q.device)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bfloat16")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    rc = load().attn_fwd_fp8(q.data_ptr(), _strides(q, "q"), k.data_ptr(), _strides(k, "k"),
+                             v.data_ptr(), _strides(v, "v"), out.data_ptr(), _strides(out, "out"),
+                             _dev(lse, "lse") if lse is not None else None, B, Hq, Hkv, Lq, Lk, D,
+                             float(scale), float(descale[0]), float(descale[1]), float(descale[2]),
+                             int(bool(causal)), _stream(stream))
+    _check(rc, "attn_fwd_fp8")
+    return out, lse
 
 
 def paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, D: int, max_blocks_per_seq: int,

@@ -96,9 +96,10 @@ Strides contiguous_strides(int H, int L, int D) {
 }
 
 // Caller strides (NULL: contiguous [B, H, L, D]). Each stride of a dimension longer than
-// 1 must be a positive multiple of 8 elements (16 bytes, the TMA and vector-store unit)
-// below 2^38; the stride of a dimension of length 1 is never used and is replaced.
-attn_status_t take_strides(const attn_strides_t* in, int B, int H, int L, int D, Strides* out) {
+// 1 must be positive, a multiple of 16 bytes (the TMA and vector-store unit) and below
+// 2^38 elements; the stride of a dimension of length 1 is never used and is replaced.
+attn_status_t take_strides(const attn_strides_t* in, int B, int H, int L, int D, Strides* out,
+                           int elem_bytes = 2) {
     *out = contiguous_strides(H, L, D);
     if (in == nullptr) return ATTN_OK;
     const long long v[3] = {in->batch, in->head, in->seq};
@@ -107,25 +108,31 @@ attn_status_t take_strides(const attn_strides_t* in, int B, int H, int L, int D,
     for (int i = 0; i < 3; ++i) {
         if (ext[i] <= 1) continue;  // keep the contiguous value
         if (v[i] <= 0 || v[i] >= (1LL << 38)) return ATTN_ERR_INVALID;
-        if (v[i] % 8 != 0) return ATTN_ERR_MISALIGNED;
+        if ((v[i] * elem_bytes) % 16 != 0) return ATTN_ERR_MISALIGNED;
         *dst[i] = v[i];
     }
     return ATTN_OK;
 }
 
 // 4-D view (D, L, H, B) of a tensor with element strides (l, h, b) and contiguous D;
-// box 64 x box_rows x 1 x 1 with 128-byte swizzle. Rows past L read as zero.
+// box (128 bytes of D) x box_rows x 1 x 1 with 128-byte swizzle. Rows past L read as zero.
+// u8: 8-bit elements (the bytes of e4m3 values).
 bool encode_strided_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, int H, int B,
-                        const Strides& st, int box_rows) {
+                        const Strides& st, int box_rows, bool u8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
+    const cuuint64_t el = u8 ? 1 : 2;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                                 static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.l) * 2, static_cast<cuuint64_t>(st.h) * 2,
-                                   static_cast<cuuint64_t>(st.b) * 2};
-    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.l) * el, static_cast<cuuint64_t>(st.h) * el,
+                                   static_cast<cuuint64_t>(st.b) * el};
+    // one 128-byte swizzle row per box row: 64 16-bit or 128 8-bit elements
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / el), static_cast<cuuint32_t>(box_rows), 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+    const CUtensorMapDataType dt = u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                      : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    return fn(tm, dt, 4,
               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -144,11 +151,11 @@ __global__ void zero_rows_kernel(uint16_t* out, long long sb, long long sh, long
 }
 
 // ------------------------------------------------------------------ launchers
-template <int D, bool BF16, int MASK, bool PAGED = false>
+template <int D, bool BF16, int MASK, bool PAGED = false, bool FP8 = false>
 attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const PrefillArgs& args, int planes, cudaStream_t stream) {
-    auto kern = attn::prefill_fwd_kernel<D, BF16, MASK, PAGED>;
-    constexpr int smem = PrefillCfg<D>::kSmemBytes;
+    auto kern = attn::prefill_fwd_kernel<D, BF16, MASK, PAGED, FP8>;
+    constexpr int smem = PrefillCfg<D, FP8>::kSmemBytes;
     static std::once_flag once;
     static attn_status_t setup = ATTN_OK;
     std::call_once(once, [&] {
@@ -468,6 +475,72 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
                 : dispatch_bwd<128, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
 }
 
+// Dense forward on e4m3 inputs (8-bit tensor-core products), bf16 output.
+attn_status_t fwd_fp8(const void* q, const attn_strides_t* q_st, const void* k,
+                      const attn_strides_t* k_st, const void* v, const attn_strides_t* v_st,
+                      void* out, const attn_strides_t* o_st, float* lse, int B, int H_q, int H_kv,
+                      int Lq, int Lk, int D, float scale, float descale_q, float descale_k,
+                      float descale_v, int causal, void* stream_) {
+    if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    const float sc = scale * descale_q * descale_k;
+    if (!std::isfinite(scale) || !(scale > 0.f) || !std::isfinite(sc) || !(sc > 0.f) ||
+        !std::isfinite(descale_v) || !(descale_v > 0.f))
+        return ATTN_ERR_INVALID;
+    if (D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (Lq > kMaxSeq || Lk > kMaxSeq) return ATTN_ERR_UNSUPPORTED;
+    const long long planes_q = static_cast<long long>(B) * H_q;
+    if (planes_q > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || Lq == 0) return ATTN_OK;  // nothing to compute; pointers may be NULL
+    if (q == nullptr || out == nullptr || (Lk > 0 && (k == nullptr || v == nullptr)))
+        return ATTN_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    Strides sq, sk, sv, so;
+    attn_status_t st = take_strides(q_st, B, H_q, Lq, D, &sq, 1);
+    if (st == ATTN_OK) st = take_strides(k_st, B, H_kv, Lk, D, &sk, 1);
+    if (st == ATTN_OK) st = take_strides(v_st, B, H_kv, Lk, D, &sv, 1);
+    if (st == ATTN_OK) st = take_strides(o_st, B, H_q, Lq, D, &so, 2);
+    if (st != ATTN_OK) return st;
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (Lk == 0) {  // no keys: O = 0, lse = -inf
+        const long long rows = planes_q * Lq;
+        zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(out), so.b, so.h, so.l,
+                                                   H_q, Lq, D, rows);
+        if (lse != nullptr)
+            attn::fill_empty_kernel<true><<<1184, 256, 0, stream>>>(nullptr, lse, 0,
+                                                                    static_cast<size_t>(rows));
+        return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    }
+    alignas(64) CUtensorMap tq, tk, tv;
+    if (!encode_strided_map(&tq, q, false, D, Lq, H_q, B, sq, attn::kBM, true) ||
+        !encode_strided_map(&tk, k, false, D, Lk, H_kv, B, sk, attn::kBN, true) ||
+        !encode_strided_map(&tv, v, false, D, Lk, H_kv, B, sv, attn::kBN, true))
+        return ATTN_ERR_CUDA;
+    PrefillArgs args{};
+    args.out = out;
+    args.out_sb = so.b;
+    args.out_sh = so.h;
+    args.out_sl = so.l;
+    args.lse = lse;
+    args.Hq = H_q;
+    args.Hkv = H_kv;
+    args.group = H_q / H_kv;
+    args.Lq = Lq;
+    args.Lk = Lk;
+    args.n_q_blocks = (Lq + 2 * attn::kBM - 1) / (2 * attn::kBM);
+    args.win_left = -1;
+    args.win_right = causal ? 0 : -1;
+    args.scale_log2 = sc * attn::kLog2e;
+    args.o_scale = descale_v;
+    const int planes = static_cast<int>(planes_q);
+    return causal ? launch_prefill<128, true, attn::kMaskCausal, false, true>(tq, tk, tv, args, planes, stream)
+                  : launch_prefill<128, true, attn::kMaskNone, false, true>(tq, tk, tv, args, planes, stream);
+}
+
 // Prefill over a paged cache: the dense forward kernel with its K/V tiles gathered
 // block by block through the table.
 attn_status_t paged_prefill(const void* q, const attn_strides_t* q_st, const void* k_cache,
@@ -558,6 +631,16 @@ attn_status_t paged_prefill(const void* q, const attn_strides_t* q_st, const voi
 }  // namespace
 
 extern "C" {
+
+attn_status_t attn_fwd_fp8(const void* q, const attn_strides_t* q_strides, const void* k,
+                           const attn_strides_t* k_strides, const void* v,
+                           const attn_strides_t* v_strides, void* out,
+                           const attn_strides_t* out_strides, float* lse, int B, int H_q, int H_kv,
+                           int Lq, int Lk, int D, float scale, float descale_q, float descale_k,
+                           float descale_v, int causal, void* stream) {
+    return fwd_fp8(q, q_strides, k, k_strides, v, v_strides, out, out_strides, lse, B, H_q, H_kv,
+                   Lq, Lk, D, scale, descale_q, descale_k, descale_v, causal, stream);
+}
 
 attn_status_t attn_fwd_paged_prefill(const void* q, const attn_strides_t* q_strides,
                                      const void* k_cache, const void* v_cache,

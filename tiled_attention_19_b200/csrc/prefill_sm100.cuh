@@ -64,13 +64,19 @@ constexpr int kOtherRegs = 80;
 constexpr int kRegBudget = 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs;  // 61,440
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D>
+template <int D, bool FP8 = false>
 struct PrefillCfg {
-    static constexpr int kChunks = D / 64;             // 64-element (128-byte) column chunks
+    static constexpr int kElem = FP8 ? 1 : 2;           // bytes per Q/K/V element
+    static constexpr int kRowBytes = D * kElem;
+    static constexpr int kChunks = kRowBytes / 128;    // 128-byte column chunks
+    static constexpr int kChunkElems = 128 / kElem;    // elements per chunk row
     static constexpr int kChunkBytes = kBM * 128;      // one chunk of a 128-row tile
-    static constexpr int kTileBytes = kBM * D * 2;     // a whole Q, K or V tile
-    static constexpr int kKStages = (D == 64) ? 5 : 3;
-    static constexpr int kVStages = (D == 64) ? 5 : 2;
+    static constexpr int kTileBytes = kBM * kRowBytes; // a whole Q, K or V tile
+    static constexpr int kKSteps = kRowBytes / 32;     // S = Q K^T: 32 bytes of K per MMA
+    static constexpr int kPVKeys = FP8 ? 32 : 16;      // keys per P.V MMA
+    static constexpr int kPCols = kBN * kElem / 4;     // TMEM columns P takes
+    static constexpr int kKStages = (kTileBytes == 16384) ? 5 : 3;
+    static constexpr int kVStages = (kTileBytes == 16384) ? 5 : 2;
     static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 384;
     static constexpr int kTmemCols = 512;
     // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
@@ -89,7 +95,8 @@ struct PrefillArgs {
     int n_q_blocks;    // ceil(Lq / 256): CTAs along the query axis
     int win_left;      // band: keys >= i' - win_left visible (-1: unbounded)
     int win_right;     // band: keys <= i' + win_right visible (-1: unbounded; causal: 0)
-    float scale_log2;  // scale * log2(e)
+    float scale_log2;  // scale * log2(e) (8-bit inputs: times the q and k descale factors)
+    float o_scale;     // 8-bit inputs: the v descale factor, applied to O (else unused)
     // Paged keys (prefill over a paged cache): K and V of sequence b are rows
     // (block_table[b][t / 16] * Hkv + h_kv) * 16 + t % 16 of the caches, seq_lens[b] keys;
     // its chunk of queries is the first q_lens[b] rows (all Lq if q_lens is NULL).
@@ -143,12 +150,13 @@ __device__ __forceinline__ void key_tiles_for(int row0, const PrefillArgs& a, in
     t1 = last / kBN + 1;
 }
 
-template <int D, bool BF16, int MASK, bool PAGED>
+template <int D, bool BF16, int MASK, bool PAGED, bool FP8 = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs args) {
-    using Cfg = PrefillCfg<D>;
+    static_assert(!FP8 || (BF16 && !PAGED), "8-bit inputs: bf16 output, dense keys");
+    using Cfg = PrefillCfg<D, FP8>;
     constexpr int NK = Cfg::kKStages;
     constexpr int NV = Cfg::kVStages;
     constexpr int Q_FULL = 0;
@@ -261,8 +269,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
-                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0, h, b);
-                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * 64, q0 + kBM, h, b);
+                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, q0, h, b);
+                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, q0 + kBM,
+                            h, b);
             }
             constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
             for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile jlo + n
@@ -297,7 +306,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             tma_load_2d(dst + k * kPageSize * 128, &tm_k, bar(K_FULL + sk), c * 64,
                                         rows[k]);
                     } else {
-                        tma_load_4d(dst, &tm_k, bar(K_FULL + sk), c * 64, j * kBN, hkv, b);
+                        tma_load_4d(dst, &tm_k, bar(K_FULL + sk), c * Cfg::kChunkElems, j * kBN, hkv, b);
                     }
                 }
                 k_issued = n + 1;
@@ -312,7 +321,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             tma_load_2d(dst + k * kPageSize * 128, &tm_v, bar(V_FULL + sv), c * 64,
                                         rows[k]);
                     } else {
-                        tma_load_4d(dst, &tm_v, bar(V_FULL + sv), c * 64, j * kBN, hkv, b);
+                        tma_load_4d(dst, &tm_v, bar(V_FULL + sv), c * Cfg::kChunkElems, j * kBN, hkv, b);
                     }
                 }
                 v_issued = n + 1;
@@ -322,30 +331,41 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ---------------------------------------------------------- MMA issuer
         regs_decrease<kOtherRegs>();
         if (lane == 0 && n_all > 0) {
-            constexpr uint32_t kIdescQK = idesc_f16(BF16, kBM, kBN, false, false);
-            constexpr uint32_t kIdescPV = idesc_f16(BF16, kBM, D, false, true);
+            // 8-bit inputs: format code 0 is E4M3 under kind::f8f6f4
+            constexpr uint32_t kIdescQK = idesc_f16(BF16 && !FP8, kBM, kBN, false, false);
+            constexpr uint32_t kIdescPV = idesc_f16(BF16 && !FP8, kBM, D, false, true);
             mma_started = true;
             // S_t = Q_t K_j^T into TMEM columns s_col (K-major operands: 16 elements =
             // 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
             auto issue_s = [&](uint32_t sQ, uint32_t s_col, int n) {
                 const uint32_t sK = sK0 + (n % NK) * Cfg::kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
                     const uint32_t koff = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
-                    mma_ss(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
-                           sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                    if constexpr (FP8)
+                        mma_ss_f8(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
+                                  sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
+                               sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_t += P_t V_j: P from TMEM (16 keys = 8 columns per step), V MN-major
-            // (16 keys = two 8-row swizzle atoms, 2048 bytes; D chunks 16 KiB apart).
-            // `first` starts the accumulator (the query tile's first key tile).
+            // O_t += P_t V_j: P from TMEM (kPVKeys keys = 8 columns per step), V MN-major
+            // (kPVKeys keys = 8-row swizzle atoms of 128 bytes, kPVKeys * 128 bytes per step;
+            // D chunks 16 KiB apart). `first` starts the accumulator (the query tile's first
+            // key tile).
             auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int n, bool first) {
                 const uint32_t sV = sV0 + (n % NV) * Cfg::kTileBytes;
 #pragma unroll
-                for (int ks = 0; ks < kBN / 16; ++ks)
-                    mma_ts(tmem + o_col, tmem + p_col + ks * 8,
-                           sdesc_sw128(sV + ks * 2048, Cfg::kChunkBytes, 1024), kIdescPV,
-                           (!first || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < kBN / Cfg::kPVKeys; ++ks) {
+                    const uint64_t bd = sdesc_sw128(sV + ks * Cfg::kPVKeys * 128, Cfg::kChunkBytes, 1024);
+                    if constexpr (FP8)
+                        mma_ts_f8(tmem + o_col, tmem + p_col + ks * 8, bd, kIdescPV,
+                                  (!first || ks > 0) ? 1u : 0u);
+                    else
+                        mma_ts(tmem + o_col, tmem + p_col + ks * 8, bd, kIdescPV,
+                               (!first || ks > 0) ? 1u : 0u);
+                }
             };
             bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
             if constexpr (MASK != kMaskWindow) {
@@ -496,20 +516,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const float alpha = (m_new == m_ref) ? 1.f : ex2_approx(m_ref - m_new);
             const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
 
-            uint32_t pk[kBN / 2];
             float rs0 = 0.f, rs1 = 0.f;
+            if constexpr (FP8) {
+                // P in e4m3, four keys per column (the lowest key in the lowest byte);
+                // p <= 2^8 < 448 under the lazy rescale, so it never saturates
+                uint32_t pk[kBN / 4];
 #pragma unroll
-            for (int x = 0; x < kBN; x += 2) {
-                const float p0 = ex2_approx(fmaf(s[x], c, neg_m));
-                const float p1 = ex2_approx(fmaf(s[x + 1], c, neg_m));
-                rs0 += p0;
-                rs1 += p1;
-                pk[x / 2] = pack2<BF16>(p0, p1);
+                for (int x = 0; x < kBN; x += 4) {
+                    const float p0 = ex2_approx(fmaf(s[x], c, neg_m));
+                    const float p1 = ex2_approx(fmaf(s[x + 1], c, neg_m));
+                    const float p2 = ex2_approx(fmaf(s[x + 2], c, neg_m));
+                    const float p3 = ex2_approx(fmaf(s[x + 3], c, neg_m));
+                    rs0 += p0 + p2;
+                    rs1 += p1 + p3;
+                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+                    pk[x / 4] = lo | (hi << 16);
+                }
+                // P overwrites the first 32 columns of this tile's S buffer.
+                tmem_st32(lane_base + s_col, pk);
+            } else {
+                uint32_t pk[kBN / 2];
+#pragma unroll
+                for (int x = 0; x < kBN; x += 2) {
+                    const float p0 = ex2_approx(fmaf(s[x], c, neg_m));
+                    const float p1 = ex2_approx(fmaf(s[x + 1], c, neg_m));
+                    rs0 += p0;
+                    rs1 += p1;
+                    pk[x / 2] = pack2<BF16>(p0, p1);
+                }
+                // P overwrites the first 64 columns of this tile's S buffer (16-bit pairs).
+                tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             }
-
-            // P overwrites the first 64 columns of this tile's S buffer (16-bit pairs).
-            tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             // Correct O when the reference max moved. S_t(j) completing implies the
             // P·V of tile j-1 (issued before it) has completed too.
             if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -540,7 +579,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // rows past a paged sequence's chunk are written as rows with no key
             const bool real = !PAGED || row < a.Lq;
             const bool has = real && l > 0.f;
-            const float inv_l = has ? 1.f / l : 0.f;
+            const float inv_l = has ? (FP8 ? args.o_scale : 1.f) / l : 0.f;
             uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) + b * args.out_sb +
                                 h * args.out_sh + static_cast<long long>(row) * args.out_sl;
 #pragma unroll
