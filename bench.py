@@ -12,7 +12,8 @@ After the step's timed region, two more calls on the same prefill workload are t
 their own and reported beside ``value`` (not part of it): the backward pass (attn_bwd,
 the ``backward`` object; --no-backward skips it) and the same prefill with K/V read
 through a paged cache (attn_fwd_paged_prefill, the ``paged_prefill`` object;
---no-paged-prefill skips it).
+--no-paged-prefill skips it), and the same prefill on e4m3 inputs (attn_fwd_fp8, the
+``fp8`` object; --no-fp8 skips it).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -275,6 +276,11 @@ def run_ours(args, ws, rank, local):
         pp_ms = measure_paged_prefill(w, ta, stream, device, steps=max(3, min(300, args.steps)),
                                       warmup=args.warmup, ws=ws)
 
+    fp8_ms = None
+    if args.fp8 and do_pre and args.window is None and PREFILL.D == 128:
+        fp8_ms = measure_fp8(w, ta, stream, device, steps=max(3, min(300, args.steps)),
+                             warmup=args.warmup, ws=ws)
+
     if args.e2e:
         e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)), window=args.window)
     else:
@@ -377,6 +383,24 @@ def run_ours(args, ws, rank, local):
             "frac": r2(pp_tf / pk_t, 4),
             "vs_dense": r2(pre_avg / pp_ms, 4),
             "avg_call_ms": round(pp_ms, 5),
+            "steps": max(3, min(300, args.steps)),
+            "gpu_launches": max(3, min(300, args.steps)),
+        }
+    if fp8_ms is not None:
+        f8_tf = job_rate(w.prefill_flops, fp8_ms, ws, 1e12) / ws
+        pk_f8 = 2 * pk_t  # the fp8 tensor rate is twice the bf16 rate (nominal 4.5 vs 2.25 PFLOP/s)
+        line["fp8"] = {
+            "what": "attn_fwd_fp8 on the prefill workload with q, k, v cast to e4m3 (bf16 output)",
+            "kernel": f"prefill_fwd_kernel<{PREFILL.D},e4m3>",
+            "value": r2(f8_tf * ws, 2),
+            "unit": "TFLOP/s",
+            "bound": "tensor",
+            "achieved": r2(f8_tf, 2),
+            "peak": pk_f8,
+            "peak_source": f"{peaks_src} bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio)",
+            "frac": r2(f8_tf / pk_f8, 4),
+            "vs_bf16": r2(pre_avg / fp8_ms, 4),
+            "avg_call_ms": round(fp8_ms, 5),
             "steps": max(3, min(300, args.steps)),
             "gpu_launches": max(3, min(300, args.steps)),
         }
@@ -491,6 +515,39 @@ def measure_paged_prefill(w, ta, stream, device, steps: int, warmup: int, ws: in
     barrier(ws)
     if ta.device_status() != 0:
         raise RuntimeError("device status set during the paged-prefill timing")
+    return reduce_max(sum(a.elapsed_time(b) for a, b in ev) / steps, ws, device)
+
+
+def measure_fp8(w, ta, stream, device, steps: int, warmup: int, ws: int):
+    """The same prefill on e4m3 inputs (attn_fwd_fp8), timed on its own: each input
+    copy's q, k, v are cast to float8_e4m3fn once. Returns ms per call."""
+    sets = [tuple(p[n].to(torch.float8_e4m3fn) for n in ("q", "k", "v")) for p in w.pf]
+    out = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Lq, PREFILL.D, dtype=torch.bfloat16,
+                      device=device)
+    lse = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Lq, device=device)
+
+    def call(i):
+        q, k, v = sets[i % len(sets)]
+        ta.fwd_fp8(q, k, v, causal=PREFILL.causal, scale=PREFILL.scale, out=out, lse=lse,
+                   stream=stream)
+
+    for i in range(warmup):
+        call(i)
+    torch.cuda.synchronize()
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set by the fp8 warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        call(warmup + i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    if ta.device_status() != 0:
+        raise RuntimeError("device status set during the fp8 timing")
     return reduce_max(sum(a.elapsed_time(b) for a, b in ev) / steps, ws, device)
 
 
@@ -641,6 +698,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false",
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--no-fp8", dest="fp8", action="store_false",
+                    help="skip the separately timed e4m3 forward of the prefill workload")
     ap.add_argument("--no-paged-prefill", dest="paged_prefill", action="store_false",
                     help="skip the separately timed paged-cache prefill of the prefill workload")
     ap.add_argument("--no-backward", dest="backward", action="store_false",
