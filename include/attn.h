@@ -175,8 +175,8 @@ size_t attn_paged_workspace_size(int num_seqs, int H_q, int H_kv, int D,
  *
  *   block_size must be 16; H_q / H_kv <= 16; D in {64, 128}. Entries of
  *   block_table past ceil(seq_lens[s] / 16) are never read. The cache rows of a
- *   sequence's last block past seq_lens[s] are read but weigh nothing; they must hold
- *   finite values (a NaN there would reach the output through 0 * NaN). An entry outside
+ *   sequence's last block past seq_lens[s] may hold anything (even NaN): they are
+ *   masked out of both products. An entry outside
  *   [0, num_blocks), or a seq_len past the table, is skipped on the device and
  *   reported as ATTN_ERR_BAD_INDEX by attn_get_device_status(). A sequence of
  *   length 0 gets O = 0 and lse = -inf. num_seqs == 0 is a no-op (every

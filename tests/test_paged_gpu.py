@@ -133,3 +133,21 @@ def test_decode_many_units_one_cta_each():
     ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
                                x["seq_lens"], s.scale)
     check_parity(out, lse, ro, rl, s.dtype, "many units")
+
+
+def test_rows_past_the_sequence_end_are_masked_even_if_nan():
+    """Cache rows of a sequence's last block past its length are read with the block but
+    must weigh nothing, whatever they hold: fill them with NaN in K and V."""
+    s = inputs.PagedSpec("t", 4, 12, 2, 128, 16, 512, torch.bfloat16, 1 / math.sqrt(128), seed=31,
+                         fixed_lens=(1, 17, 130, 511))
+    x = inputs.make(s)
+    for sq, n in enumerate(s.fixed_lens):
+        blk = int(x["block_table"][sq][(n - 1) // 16])
+        x["k_cache"][blk, :, n % 16 or 16:] = float("nan")
+        x["v_cache"][blk, :, n % 16 or 16:] = float("nan")
+    out, lse = run_paged(to_dev(x), s.scale)
+    torch.cuda.synchronize()
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out.cpu(), lse.cpu(), ro, rl, s.dtype, "nan rows past the end")

@@ -436,10 +436,24 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 m1 = mn1;
                 const uint32_t pa[4] = {pack2<BF16>(p[0][0], p[0][1]), pack2<BF16>(p[0][2], p[0][3]),
                                         pack2<BF16>(p[1][0], p[1][1]), pack2<BF16>(p[1][2], p[1][3])};
+                // A block that crosses the sequence end: its rows past len weigh nothing,
+                // and zeroing them keeps whatever they hold (even NaN) out of P.V. In the
+                // B fragments, the low and high halves of b0 are tokens 2t and 2t+1, those
+                // of b1 tokens 8+2t and 9+2t.
+                uint32_t vm0 = 0xFFFFFFFFu, vm1 = 0xFFFFFFFFu;
+                if (tok0 + kPageSize > len) {
+                    vm0 = (tok0 + 2 * t < len ? 0x0000FFFFu : 0u) | (tok0 + 2 * t + 1 < len ? 0xFFFF0000u : 0u);
+                    vm1 = (tok0 + 8 + 2 * t < len ? 0x0000FFFFu : 0u) |
+                          (tok0 + 9 + 2 * t < len ? 0xFFFF0000u : 0u);
+                }
 #pragma unroll
                 for (int pp = 0; pp < NT / 2; ++pp) {
                     uint32_t vf[4];
                     ldsm_x4_t(vb + swz<D>(v_tok, 2 * pp + v_sub), vf);
+                    vf[0] &= vm0;
+                    vf[1] &= vm1;
+                    vf[2] &= vm0;
+                    vf[3] &= vm1;
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         float* o = oacc[2 * pp + h2];

@@ -521,30 +521,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 // P in e4m3, four keys per column (the lowest key in the lowest byte);
                 // p <= 2^8 < 448 under the lazy rescale, so it never saturates
                 uint32_t pk[kBN / 4];
+                const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
+                uint64_t rs2 = f2pack(0.f, 0.f);
 #pragma unroll
                 for (int x = 0; x < kBN; x += 4) {
-                    const float p0 = ex2_approx(fmaf(s[x], c, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[x + 1], c, neg_m));
-                    const float p2 = ex2_approx(fmaf(s[x + 2], c, neg_m));
-                    const float p3 = ex2_approx(fmaf(s[x + 3], c, neg_m));
-                    rs0 += p0 + p2;
-                    rs1 += p1 + p3;
+                    float t0, t1, t2, t3;
+                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
+                    f2unpack(fma2(f2pack(s[x + 2], s[x + 3]), c2, nm2), t2, t3);
+                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+                    rs2 = add2(rs2, add2(f2pack(p0, p1), f2pack(p2, p3)));
                     const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
                     const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
                     pk[x / 4] = lo | (hi << 16);
                 }
+                f2unpack(rs2, rs0, rs1);
                 // P overwrites the first 32 columns of this tile's S buffer.
                 tmem_st32(lane_base + s_col, pk);
             } else {
+                // exponent arguments and row sums two at a time (f32x2 instructions)
                 uint32_t pk[kBN / 2];
+                const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
+                uint64_t rs2 = f2pack(0.f, 0.f);
 #pragma unroll
                 for (int x = 0; x < kBN; x += 2) {
-                    const float p0 = ex2_approx(fmaf(s[x], c, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[x + 1], c, neg_m));
-                    rs0 += p0;
-                    rs1 += p1;
+                    float t0, t1;
+                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
+                    const float p0 = ex2_approx(t0);
+                    const float p1 = ex2_approx(t1);
+                    rs2 = add2(rs2, f2pack(p0, p1));
                     pk[x / 2] = pack2<BF16>(p0, p1);
                 }
+                f2unpack(rs2, rs0, rs1);
                 // P overwrites the first 64 columns of this tile's S buffer (16-bit pairs).
                 tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
                 tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
