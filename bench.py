@@ -265,6 +265,27 @@ def run_ours(args, ws, rank, local):
     pre_avg = reduce_max(sum(pre_ms) / len(pre_ms), ws, device)
     dec_avg = reduce_max(sum(dec_ms) / len(dec_ms), ws, device)
 
+    # The same calls replayed from CUDA graphs: device time per launch without the
+    # host's launch latency (matters for microsecond kernels such as the decode).
+    g_pre = g_dec = None
+    if args.graphs:
+        if do_pre:
+            g_pre = graph_launch_ms(
+                lambda i: ta.fwd(w.pf[i % w.p_copies]["q"], w.pf[i % w.p_copies]["k"],
+                                 w.pf[i % w.p_copies]["v"], causal=PREFILL.causal,
+                                 scale=PREFILL.scale, out=w.p_out, lse=w.p_lse,
+                                 window=args.window),
+                n_calls=2 * w.p_copies, replays=max(1, min(100, args.steps) // (2 * w.p_copies)),
+                ws=ws, device=device)
+        if do_dec:
+            g_dec = graph_launch_ms(
+                lambda i: ta.fwd_paged(w.dc[i % copies]["q"], w.dc[i % copies]["k_cache"],
+                                       w.dc[i % copies]["v_cache"], w.dc[i % copies]["block_table"],
+                                       w.dc[i % copies]["seq_lens"], scale=DECODE.scale,
+                                       out=w.d_out, lse=w.d_lse, workspace=ws_buf),
+                n_calls=4 * copies, replays=max(1, min(1000, args.steps) // (4 * copies)),
+                ws=ws, device=device)
+
     bwd_ms = None
     if args.backward and do_pre:
         bwd_ms = measure_backward(w, ta, stream, device, steps=max(3, min(100, args.steps)),
@@ -343,6 +364,8 @@ def run_ours(args, ws, rank, local):
             "frac_of_burst_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops"], 4),
             "traffic": None if args.window else profiled_traffic("prefill", PREFILL.name),
             "avg_launch_ms": round(pre_avg, 5),
+            "graph_avg_launch_ms": None if g_pre is None else round(g_pre, 5),
+            "graph_frac": None if g_pre is None else r2(w.prefill_flops / (g_pre * 1e-3) / 1e12 / pk_t, 4),
         },
         "paged_decode": {
             "kernel": "paged_decode_kernel<128,bf16>",
@@ -355,6 +378,12 @@ def run_ours(args, ws, rank, local):
             "frac": r2(per_gpu_gbs and per_gpu_gbs / pk_h, 4),
             "traffic": profiled_traffic("decode", DECODE.name),
             "avg_launch_ms": round(dec_avg, 5),
+            "graph_avg_launch_ms": None if g_dec is None else round(g_dec, 5),
+            "graph_value": None if g_dec is None else r2(w.decode_bytes / (g_dec * 1e-3) / 1e9, 1),
+            "graph_frac": None if g_dec is None else r2(w.decode_bytes / (g_dec * 1e-3) / 1e9 / pk_h, 4),
+            "graph_note": "the same calls replayed back to back from a CUDA graph (no host work "
+                          "between launches); avg_launch_ms above includes the host's launch "
+                          "latency whenever it exceeds the kernel's time",
         },
         "e2e": {
             "value": r2(e2e_tf, 3),
@@ -468,6 +497,41 @@ def measure_backward(w, ta, stream, device, steps: int, warmup: int, ws: int, wi
     if ta.device_status() != 0:
         raise RuntimeError("device status set during the backward timing")
     ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    return reduce_max(ms, ws, device)
+
+
+def graph_launch_ms(call, n_calls: int, replays: int, ws: int, device):
+    """Per-launch device time of `call` from a CUDA graph of n_calls back-to-back calls,
+    replayed `replays` times between two events: no host work between launches, so a
+    kernel of a few microseconds is timed without the host's launch latency. None if the
+    capture fails."""
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for i in range(3):
+                call(i)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n_calls):
+                call(i)
+        g.replay()
+        torch.cuda.synchronize()
+    except RuntimeError:
+        return None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = e0.elapsed_time(e1) / (replays * n_calls)
+    del g
     return reduce_max(ms, ws, device)
 
 
@@ -705,6 +769,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false",
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--no-graphs", dest="graphs", action="store_false",
+                    help="skip the CUDA-graph replay timing of the step's two calls")
     ap.add_argument("--no-fp8", dest="fp8", action="store_false",
                     help="skip the separately timed e4m3 forward of the prefill workload")
     ap.add_argument("--no-paged-prefill", dest="paged_prefill", action="store_false",

@@ -564,6 +564,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // The partial outputs of this thread's first output slice, chunks 0..7, are loaded
+    // now, so their round trip overlaps the one for the log2-sum-exp values below.
+    const size_t step = static_cast<size_t>(G) * D / 4;  // float4 stride between chunks
+    float4 pre[8];
+    if (tid < G * (D / 4)) {
+        const float4* src = reinterpret_cast<const float4*>(
+            a.ws_o + (static_cast<size_t>(chunk0) * G + tid / (D / 4)) * D + (tid % (D / 4)) * 4);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            pre[u] = (u < nchunk) ? __ldcg(src + u * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     // All chunks' log2-sum-exp in shared memory at once (one round of parallel loads),
     // then per row the maximum, the total weight and each chunk's normalised weight.
     float* s_w = sm_o;  // [nchunk][G], reused
@@ -598,13 +609,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
         const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
         const float4* src = reinterpret_cast<const float4*>(a.ws_o + (static_cast<size_t>(chunk0) * G + r) * D + d);
-        const size_t step = static_cast<size_t>(G) * D / 4;  // float4 stride between chunks
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < nchunk; k += 8) {
             float4 v[8];
+            if (k == 0 && i4 == tid) {  // prefetched above
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                v[u] = (k + u < nchunk) ? __ldcg(src + (k + u) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int u = 0; u < 8; ++u) v[u] = pre[u];
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    v[u] = (k + u < nchunk) ? __ldcg(src + (k + u) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const float w = (k + u < nchunk) ? s_w[(k + u) * G + r] : 0.f;
