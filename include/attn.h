@@ -287,6 +287,31 @@ attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const
                               void* stream);
 
 /*
+ * attn_bwd_strided -- attn_bwd_window on tensors of any layout with a contiguous last
+ * dimension (for example the [B, L, H, D] layout: batch stride L*H*D, head stride D,
+ * row stride H*D). Each of q, k, v, out, dout, dq, dk, dv takes its own
+ * attn_strides_t (in elements; each stride times the element size a multiple of 16
+ * bytes), or NULL for the contiguous [B, H, L, D] layout; lse stays [B, H_q, Lq]
+ * contiguous. Gradients are written through their strides, every element of the
+ * described views and nothing else. causal, window_left and window_right as
+ * attn_fwd_window (pass -1, -1 with causal = 0 for dense attention); all other
+ * arguments and errors as attn_bwd, plus ATTN_ERR_MISALIGNED for a stride that breaks
+ * the 16-byte rule. The results are bit-identical to attn_bwd_window on contiguous
+ * copies of the same values.
+ */
+attn_status_t attn_bwd_strided(const void* q, const attn_strides_t* q_strides, const void* k,
+                               const attn_strides_t* k_strides, const void* v,
+                               const attn_strides_t* v_strides, const void* out,
+                               const attn_strides_t* out_strides, const void* dout,
+                               const attn_strides_t* dout_strides, const float* lse, void* dq,
+                               const attn_strides_t* dq_strides, void* dk,
+                               const attn_strides_t* dk_strides, void* dv,
+                               const attn_strides_t* dv_strides, int B, int H_q, int H_kv, int Lq,
+                               int Lk, int D, float scale, int causal, int window_left,
+                               int window_right, attn_dtype_t dtype, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * attn_fwd_fp8 -- dense attention forward on 8-bit inputs: q, k and v in FP8 E4M3, the
  * tensor-core products in 8 bits (tcgen05 kind::f8f6f4), softmax and accumulation in
  * fp32, O in bf16 ("Flash Attention" skill page (hermes-agent-app.ru), Scenario 3: the

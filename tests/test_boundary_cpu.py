@@ -219,6 +219,28 @@ def test_attn_bwd_window_validation():
     assert call_bwd(bwd_args(D=80), window=(3, 3)) == -2
 
 
+def test_attn_bwd_strided_validation():
+    lib = ta.load()
+    S = ta.Strides
+
+    def call(st=(None,) * 8, **kw):
+        a = bwd_args(**kw)
+        return lib.attn_bwd_strided(a["q"], st[0], a["k"], st[1], a["v"], st[2], a["out"], st[3],
+                                    a["dout"], st[4], a["lse"], a["dq"], st[5], a["dk"], st[6],
+                                    a["dv"], st[7], a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"],
+                                    a["D"], a["scale"], a["causal"], -1, -1, a["dtype"], a["ws"],
+                                    a["ws_n"], a["stream"])
+    bad_row = S(8 * 64 * 2, 64, 64 * 2 + 4)                       # 16-byte rule broken
+    for i in range(8):                                            # every tensor's strides checked
+        st = [None] * 8
+        st[i] = bad_row
+        assert call(st=st) == -3, i
+    assert call(st=[None] * 6 + [S(-8, 512, 64), None], B=2) == -1   # negative dk stride
+    assert call(st=[S(1 << 38, 512, 64)] + [None] * 7, B=2) == -1    # oversized q view
+    assert call(ws_n=16) == -7                                       # strides do not excuse it
+    assert call(st=[S(0, 0, 0)] * 8, B=1, Hq=1, Hkv=1, Lq=1, Lk=1, D=96) == -2
+
+
 def test_bwd_empty_problems_and_workspace_size():
     lib = ta.load()
     # B == 0, or no queries and no keys: nothing to write, pointers may be NULL

@@ -58,6 +58,9 @@ SIGNATURES = {
                       _i, _vp, _sz, _vp]),
     "attn_bwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                              _f, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "attn_bwd_strided": (_i, [_vp, _sp, _vp, _sp, _vp, _sp, _vp, _sp, _vp, _sp, _vp, _vp, _sp,
+                              _vp, _sp, _vp, _sp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _i,
+                              _vp, _sz, _vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_get_device_status": (_i, [_vp]),
     "attn_selftest_bounded_wait": (_i, [_vp]),
@@ -186,7 +189,8 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
     """Gradients (dq, dk, dv) of attention given dout = dLoss/dO, from the forward pass's
     inputs, output and lse (fwd with the same causal / window / scale). dk, dv have the
     K/V heads' shape. The workspace (attn_bwd_workspace_size bytes) is allocated when not
-    given."""
+    given. Tensors may be any views with a contiguous last dimension (as fwd); those go
+    through attn_bwd_strided, and default gradients take their inputs' strides."""
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
     if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape or out.shape != q.shape or \
@@ -201,10 +205,26 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape or \
+            len({q.dtype, dq.dtype, dk.dtype, dv.dtype}) != 1:
+        raise ValueError("dq, dk, dv must match q, k, v in shape and dtype")
     n = bwd_workspace_size(B, Hq, Lq)
     if workspace is None:
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
     ws_n = workspace.numel() * workspace.element_size()
+    if not all(t.is_contiguous() for t in (q, k, v, out, dout, dq, dk, dv)):
+        names = ("q", "k", "v", "out", "dout", "dq", "dk", "dv")
+        st = [_strides(t, n) for t, n in zip((q, k, v, out, dout, dq, dk, dv), names)]
+        w = window if window is not None else (-1, -1)
+        rc = load().attn_bwd_strided(q.data_ptr(), st[0], k.data_ptr(), st[1], v.data_ptr(), st[2],
+                                     out.data_ptr(), st[3], dout.data_ptr(), st[4],
+                                     _dev(lse, "lse"), dq.data_ptr(), st[5], dk.data_ptr(), st[6],
+                                     dv.data_ptr(), st[7], B, Hq, Hkv, Lq, Lk, D, float(scale),
+                                     int(bool(causal)), int(w[0]), int(w[1]),
+                                     _dtype_code(q.dtype), _dev(workspace, "workspace"), ws_n,
+                                     _stream(stream))
+        _check(rc, "attn_bwd_strided")
+        return dq, dk, dv
     args = (_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), _dev(dout, "dout"),
             _dev(lse, "lse"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"), B, Hq, Hkv, Lq, Lk,
             D, float(scale), int(bool(causal)))

@@ -347,18 +347,25 @@ attn_status_t launch_bwd(const CUtensorMap& tx, const CUtensorMap& tw, const CUt
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Strides of the backward pass's tensors: q, k, v, out, dout (dq, dk, dv go in the args).
+struct BwdStrides {
+    Strides q, k, v, o, d;
+};
+
 template <int D, bool BF16, int MASK>
 attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* out,
                       const void* dout, const float* lse, const attn::BwdArgs& args,
-                      long long planes_q, long long planes_kv, cudaStream_t stream) {
+                      long long planes_q, long long planes_kv, const BwdStrides& st,
+                      cudaStream_t stream) {
     // dK, dV: fixed K and V, streamed Q and dO; dQ: fixed Q and dO, streamed K and V
     // (128-row boxes throughout).
     static_assert(attn::kBwdFix == attn::kBwdSub, "one box height for fixed and streamed tiles");
     alignas(64) CUtensorMap tk, tv, tq, tdo;
-    if (!encode_tile_map(&tk, k, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
-        !encode_tile_map(&tv, v, BF16, D, args.Lk, planes_kv, attn::kBwdFix) ||
-        !encode_tile_map(&tq, q, BF16, D, args.Lq, planes_q, attn::kBwdFix) ||
-        !encode_tile_map(&tdo, dout, BF16, D, args.Lq, planes_q, attn::kBwdFix))
+    const int B = static_cast<int>(planes_q / args.Hq);
+    if (!encode_strided_map(&tk, k, BF16, D, args.Lk, args.Hkv, B, st.k, attn::kBwdFix) ||
+        !encode_strided_map(&tv, v, BF16, D, args.Lk, args.Hkv, B, st.v, attn::kBwdFix) ||
+        !encode_strided_map(&tq, q, BF16, D, args.Lq, args.Hq, B, st.q, attn::kBwdFix) ||
+        !encode_strided_map(&tdo, dout, BF16, D, args.Lq, args.Hq, B, st.d, attn::kBwdFix))
         return ATTN_ERR_CUDA;
     const long long rows_pad = planes_q * args.Lq_pad;  // a multiple of 128: whole warps
     const long long blocks = rows_pad * 8 / 256;
@@ -366,11 +373,11 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
     attn::bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const uint16_t*>(out), static_cast<const uint16_t*>(dout), lse,
         const_cast<float*>(args.nlse2), const_cast<float*>(args.delta), args.Lq, args.Lq_pad,
-        rows_pad);
+        rows_pad, args.Hq, st.o.b, st.o.h, st.o.l, st.d.b, st.d.h, st.d.l);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    attn_status_t st = launch_bwd<D, BF16, MASK, attn::kDKDV>(
+    const attn_status_t rc = launch_bwd<D, BF16, MASK, attn::kDKDV>(
         tk, tv, tq, tdo, args, planes_kv, (args.Lk + attn::kBwdFix - 1) / attn::kBwdFix, stream);
-    if (st != ATTN_OK) return st;
+    if (rc != ATTN_OK) return rc;
     return launch_bwd<D, BF16, MASK, attn::kDQ>(tq, tdo, tk, tv, args, planes_q,
                                                 (args.Lq + attn::kBwdFix - 1) / attn::kBwdFix,
                                                 stream);
@@ -380,15 +387,15 @@ template <int D, bool BF16>
 attn_status_t dispatch_bwd(int mask, const void* q, const void* k, const void* v,
                            const void* out, const void* dout, const float* lse,
                            const attn::BwdArgs& args, long long planes_q, long long planes_kv,
-                           cudaStream_t stream) {
+                           const BwdStrides& st, cudaStream_t stream) {
     if (mask == attn::kMaskCausal)
         return run_bwd<D, BF16, attn::kMaskCausal>(q, k, v, out, dout, lse, args, planes_q,
-                                                   planes_kv, stream);
+                                                   planes_kv, st, stream);
     if (mask == attn::kMaskWindow)
         return run_bwd<D, BF16, attn::kMaskWindow>(q, k, v, out, dout, lse, args, planes_q,
-                                                   planes_kv, stream);
+                                                   planes_kv, st, stream);
     return run_bwd<D, BF16, attn::kMaskNone>(q, k, v, out, dout, lse, args, planes_q, planes_kv,
-                                             stream);
+                                             st, stream);
 }
 
 size_t bwd_workspace_bytes(long long planes_q, int Lq) {
@@ -397,15 +404,11 @@ size_t bwd_workspace_bytes(long long planes_q, int Lq) {
     return static_cast<size_t>(planes_q) * static_cast<size_t>(pad) * 2 * sizeof(float);
 }
 
-template <bool BF16>
-void fill_zero(void* p, size_t n, cudaStream_t stream) {
-    attn::fill_empty_kernel<BF16><<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(p), nullptr, n, 0);
-}
-
 attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* out,
                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                        int H_q, int H_kv, int Lq, int Lk, int D, float scale, int left, int right,
-                       attn_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream_) {
+                       attn_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream_,
+                       const attn_strides_t* const* strides = nullptr) {
     if (B < 0 || H_q < 1 || H_kv < 1 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID;
     if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -425,6 +428,17 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4))
         return ATTN_ERR_MISALIGNED;
+    // strides: q, k, v, out, dout, dq, dk, dv (NULL array or entry: contiguous)
+    Strides sts[8];
+    {
+        const int hs[8] = {H_q, H_kv, H_kv, H_q, H_q, H_q, H_kv, H_kv};
+        const int ls[8] = {Lq, Lk, Lk, Lq, Lq, Lq, Lk, Lk};
+        for (int i = 0; i < 8; ++i) {
+            const attn_status_t st = take_strides(strides ? strides[i] : nullptr, B, hs[i], ls[i], D,
+                                                  &sts[i]);
+            if (st != ATTN_OK) return st;
+        }
+    }
     if (have_q && have_k) {
         if (workspace == nullptr || workspace_bytes < bwd_workspace_bytes(planes_q, Lq))
             return ATTN_ERR_WORKSPACE;
@@ -436,13 +450,13 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
     const bool bf16 = dtype == ATTN_BF16;
     if (!have_q || !have_k) {  // no queries: dK = dV = 0; no keys: dQ = 0
         if (!have_q) {
-            const size_t n = static_cast<size_t>(planes_kv) * Lk * D;
-            if (bf16) { fill_zero<true>(dk, n, stream); fill_zero<true>(dv, n, stream); }
-            else { fill_zero<false>(dk, n, stream); fill_zero<false>(dv, n, stream); }
+            zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(dk), sts[6].b, sts[6].h,
+                                                       sts[6].l, H_kv, Lk, D, planes_kv * Lk);
+            zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(dv), sts[7].b, sts[7].h,
+                                                       sts[7].l, H_kv, Lk, D, planes_kv * Lk);
         } else {
-            const size_t n = static_cast<size_t>(planes_q) * Lq * D;
-            if (bf16) fill_zero<true>(dq, n, stream);
-            else fill_zero<false>(dq, n, stream);
+            zero_rows_kernel<<<1184, 256, 0, stream>>>(static_cast<uint16_t*>(dq), sts[5].b, sts[5].h,
+                                                       sts[5].l, H_q, Lq, D, planes_q * Lq);
         }
         return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
     }
@@ -456,6 +470,14 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
     args.dq = dq;
     args.dk = dk;
     args.dv = dv;
+    const Strides* outs[3] = {&sts[5], &sts[6], &sts[7]};
+    long long* dst[3] = {args.dq_s, args.dk_s, args.dv_s};
+    for (int i = 0; i < 3; ++i) {
+        dst[i][0] = outs[i]->b;
+        dst[i][1] = outs[i]->h;
+        dst[i][2] = outs[i]->l;
+    }
+    const BwdStrides bst{sts[0], sts[1], sts[2], sts[3], sts[4]};
     args.Hq = H_q;
     args.Hkv = H_kv;
     args.group = H_q / H_kv;
@@ -469,10 +491,10 @@ attn_status_t bwd_band(const void* q, const void* k, const void* v, const void* 
                   : (left < 0 && right == 0) ? attn::kMaskCausal
                                              : attn::kMaskWindow;
     if (D == 64)
-        return bf16 ? dispatch_bwd<64, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream)
-                    : dispatch_bwd<64, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
-    return bf16 ? dispatch_bwd<128, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream)
-                : dispatch_bwd<128, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, stream);
+        return bf16 ? dispatch_bwd<64, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, bst, stream)
+                    : dispatch_bwd<64, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, bst, stream);
+    return bf16 ? dispatch_bwd<128, true>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, bst, stream)
+                : dispatch_bwd<128, false>(m, q, k, v, out, dout, lse, args, planes_q, planes_kv, bst, stream);
 }
 
 // Dense forward on e4m3 inputs (8-bit tensor-core products), bf16 output.
@@ -666,6 +688,25 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        attn_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
     return bwd_band(q, k, v, out, dout, lse, dq, dk, dv, B, H_q, H_kv, Lq, Lk, D, scale, -1,
                     causal ? 0 : -1, dtype, workspace, workspace_bytes, stream);
+}
+
+attn_status_t attn_bwd_strided(const void* q, const attn_strides_t* q_strides, const void* k,
+                               const attn_strides_t* k_strides, const void* v,
+                               const attn_strides_t* v_strides, const void* out,
+                               const attn_strides_t* out_strides, const void* dout,
+                               const attn_strides_t* dout_strides, const float* lse, void* dq,
+                               const attn_strides_t* dq_strides, void* dk,
+                               const attn_strides_t* dk_strides, void* dv,
+                               const attn_strides_t* dv_strides, int B, int H_q, int H_kv, int Lq,
+                               int Lk, int D, float scale, int causal, int window_left,
+                               int window_right, attn_dtype_t dtype, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID;
+    const attn_strides_t* st[8] = {q_strides, k_strides,  v_strides,  out_strides,
+                                   dout_strides, dq_strides, dk_strides, dv_strides};
+    return bwd_band(q, k, v, out, dout, lse, dq, dk, dv, B, H_q, H_kv, Lq, Lk, D, scale,
+                    window_left, causal ? 0 : window_right, dtype, workspace, workspace_bytes,
+                    stream, st);
 }
 
 attn_status_t attn_bwd_window(const void* q, const void* k, const void* v, const void* out,

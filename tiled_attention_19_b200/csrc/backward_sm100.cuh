@@ -89,9 +89,10 @@ struct BwdCfg {
 struct BwdArgs {
     const float* nlse2;  // [B*Hq][Lq_pad] -lse * log2(e) (-inf: row sees no key / padding)
     const float* delta;  // [B*Hq][Lq_pad] dO . O
-    void* dq;            // [B, Hq, Lq, D]
-    void* dk;            // [B, Hkv, Lk, D]
-    void* dv;            // [B, Hkv, Lk, D]
+    void* dq;            // [B, Hq, Lq, D] through dq_s
+    void* dk;            // [B, Hkv, Lk, D] through dk_s
+    void* dv;            // [B, Hkv, Lk, D] through dv_s
+    long long dq_s[3], dk_s[3], dv_s[3];  // element strides over (batch, head, row)
     int Hq, Hkv, group, Lq, Lk, Lq_pad;
     int win_left, win_right;  // band as in the forward pass (-1: unbounded; causal: right 0)
     float scale;              // applied to dQ and dK
@@ -155,7 +156,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        const float* __restrict__ lse,
                                                        float* __restrict__ nlse2,
                                                        float* __restrict__ delta, int Lq,
-                                                       int Lq_pad, long long rows_pad) {
+                                                       int Lq_pad, long long rows_pad, int Hq,
+                                                       long long o_sb, long long o_sh,
+                                                       long long o_sl, long long d_sb,
+                                                       long long d_sh, long long d_sl) {
     constexpr int kPer = D / 8;  // elements per thread: 16 (D = 128) or 8 (D = 64)
     const long long r = (blockIdx.x * 256LL + threadIdx.x) >> 3;
     const int sub = threadIdx.x & 7;
@@ -164,9 +168,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
     const int i = static_cast<int>(r % Lq_pad);
     float acc = 0.f;
     if (i < Lq) {
-        const size_t e = (static_cast<size_t>(plane) * Lq + i) * D + sub * kPer;
-        const uint4* po = reinterpret_cast<const uint4*>(out + e);
-        const uint4* pd = reinterpret_cast<const uint4*>(dout + e);
+        const long long bb = plane / Hq, hh = plane % Hq;
+        const uint4* po = reinterpret_cast<const uint4*>(out + bb * o_sb + hh * o_sh + i * o_sl + sub * kPer);
+        const uint4* pd = reinterpret_cast<const uint4*>(dout + bb * d_sb + hh * d_sh + i * d_sl + sub * kPer);
 #pragma unroll
         for (int c = 0; c < kPer / 8; ++c) {
             const uint4 a = po[c], b = pd[c];
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int n_all = (KIND == kDKDV) ? n_sub * args.group : n_sub;
     const int b = (KIND == kDKDV) ? plane / args.Hkv : plane / args.Hq;
     const int kv_plane = (KIND == kDKDV) ? plane : b * args.Hkv + (plane % args.Hq) / args.group;
+    const int h_fix = (KIND == kDKDV) ? plane % args.Hkv : plane % args.Hq;  // head of the fixed pair
 
     if (threadIdx.x == 0) {
         mbar_init(bar(FIX_FULL), 1);
@@ -295,21 +300,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ------------------------------------------------------------ producer
         regs_decrease<kBwdOtherRegs>();
         if (lane == 0 && n_all > 0) {
-            const int fix_plane = (KIND == kDKDV) ? kv_plane : plane;
             mbar_arrive_expect_tx(bar(FIX_FULL), 2 * Cfg::kFixBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
-                tma_load_3d(sX + c * Cfg::kFixChunk, &tm_x, bar(FIX_FULL), c * 64, base, fix_plane);
-                tma_load_3d(sW + c * Cfg::kFixChunk, &tm_w, bar(FIX_FULL), c * 64, base, fix_plane);
+                tma_load_4d(sX + c * Cfg::kFixChunk, &tm_x, bar(FIX_FULL), c * 64, base, h_fix, b);
+                tma_load_4d(sW + c * Cfg::kFixChunk, &tm_w, bar(FIX_FULL), c * 64, base, h_fix, b);
             }
             for (int n = 0; n < n_all; ++n) {
-                int sub, y_plane;
+                int sub, y_plane, h_y;  // the streamed pair's (batch * heads + head) and head
                 if (KIND == kDKDV) {
                     const int g = n / n_sub;
                     sub = s_lo + n % n_sub;
-                    y_plane = b * args.Hq + (kv_plane % args.Hkv) * args.group + g;
+                    h_y = (kv_plane % args.Hkv) * args.group + g;
+                    y_plane = b * args.Hq + h_y;
                 } else {
                     sub = s_lo + n;
+                    h_y = kv_plane % args.Hkv;
                     y_plane = kv_plane;
                 }
                 const int row = sub * kBwdSub;
@@ -322,8 +328,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mbar_arrive_expect_tx(bar(Z_FULL + zs), Cfg::kSubBytes);
 #pragma unroll
                     for (int c = 0; c < Cfg::kChunks; ++c)
-                        tma_load_3d(sZ(n) + c * Cfg::kSubChunk, &tm_z, bar(Z_FULL + zs), c * 64, row,
-                                    y_plane);
+                        tma_load_4d(sZ(n) + c * Cfg::kSubChunk, &tm_z, bar(Z_FULL + zs), c * 64, row,
+                                    h_y, b);
                     z_issued = n + 1;
                     return true;
                 };
@@ -334,8 +340,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                           Cfg::kSubBytes + (KIND == kDKDV ? 2 * kBwdSub * 4 : 0));
 #pragma unroll
                     for (int c = 0; c < Cfg::kChunks; ++c)
-                        tma_load_3d(sY(n) + c * Cfg::kSubChunk, &tm_y, bar(Y_FULL + ys), c * 64, row,
-                                    y_plane);
+                        tma_load_4d(sY(n) + c * Cfg::kSubChunk, &tm_y, bar(Y_FULL + ys), c * 64, row,
+                                    h_y, b);
                     if (KIND == kDKDV) {
                         const size_t so = static_cast<size_t>(y_plane) * args.Lq_pad + row;
                         bulk_load(smem_u32(stats + ys * 2 * kBwdSub), args.nlse2 + so, kBwdSub * 4,
@@ -572,15 +578,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             uint32_t g_col;
             float mul;
             if (KIND == kDKDV) {
-                dst = static_cast<uint16_t*>(wg == 0 ? args.dv : args.dk) +
-                      (static_cast<size_t>(plane) * args.Lk + r) * D;
+                const long long* st = wg == 0 ? args.dv_s : args.dk_s;
+                dst = static_cast<uint16_t*>(wg == 0 ? args.dv : args.dk) + b * st[0] + h_fix * st[1] +
+                      static_cast<long long>(r) * st[2];
                 col0 = 0;
                 ncols = D;
                 g_col = G_COL + wg * D;
                 mul = wg == 0 ? 1.f : args.scale;
                 valid = r < args.Lk;
             } else {
-                dst = static_cast<uint16_t*>(args.dq) + (static_cast<size_t>(plane) * args.Lq + r) * D;
+                dst = static_cast<uint16_t*>(args.dq) + b * args.dq_s[0] + h_fix * args.dq_s[1] +
+                      static_cast<long long>(r) * args.dq_s[2];
                 col0 = wg * (D / 2);
                 ncols = D / 2;
                 g_col = G_COL + col0;
