@@ -75,9 +75,9 @@ struct BwdCfg {
     static constexpr int kTileRegion = 2 * kFixBytes + (kYStages + kZStages) * kSubBytes;
     // kDKDV: -lse*log2(e) and delta of the 128 query rows of each Y stage
     static constexpr int kStatBytes = (KIND == kDKDV) ? kYStages * 2 * kBwdSub * 4 : 0;
-    // barriers: FIX_FULL, FULL/EMPTY per Y and per Z stage, S_FULL, DP_FULL, DP_FREE, P_FULL,
-    // DONE, DRAIN
-    static constexpr int kNumBars = 1 + 2 * (kYStages + kZStages) + 6;
+    // barriers: FIX_FULL, FULL/EMPTY per Y and per Z stage, S_FULL, DP_FULL, DP_FREE, two
+    // P_FULL, DONE, DRAIN
+    static constexpr int kNumBars = 1 + 2 * (kYStages + kZStages) + 7;
     static constexpr int kSmemBytes = 1024 + kTileRegion + kStatBytes + kNumBars * 8 + 16;
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
     // TMEM: kDQ: S of even / odd sub-tiles at 0 / 128, dP at 256, dQ at 384;
@@ -212,8 +212,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr int S_FULL = Z_EMPTY + NZ;   // S of the next sub-tile is in TMEM
     constexpr int DP_FULL = S_FULL + 1;    // dP of the next sub-tile is in TMEM
     constexpr int DP_FREE = DP_FULL + 1;   // the softmax warps hold S and dP in registers
-    constexpr int P_FULL = DP_FREE + 1;    // P / dS of the sub-tile are in TMEM
-    constexpr int DONE = P_FULL + 1;
+    // P / dS of sub-tile n are in TMEM: barrier P_FULL + (n & 1). The 256 softmax threads
+    // arrive once per sub-tile, and for kDQ a fast warp can arrive for n + 1 (S and dP of
+    // n + 1 are issued as soon as every warp holds those of n) while a slow one is still
+    // writing dS(n); on a single barrier that early arrival would complete phase n before
+    // dS(n) is whole. Alternating barriers keep each phase's arrivals apart: no warp can
+    // reach n + 2 before every warp has finished n, since S(n + 2) waits for DP_FREE(n + 1).
+    constexpr int P_FULL = DP_FREE + 1;
+    constexpr int DONE = P_FULL + 2;
     constexpr int DRAIN = DONE + 1;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
     constexpr uint32_t G_COL = (KIND == kDKDV) ? 256 : 384;
@@ -271,6 +277,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar(DP_FULL), 1);
         mbar_init(bar(DP_FREE), 256);
         mbar_init(bar(P_FULL), 256);
+        mbar_init(bar(P_FULL + 1), 256);
         mbar_init(bar(DONE), 1);
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
@@ -420,7 +427,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         mma_commit(bar(Z_EMPTY + m % NZ));
                     }
                 }
-                ok = wait_phase(bar(P_FULL), n & 1, abort_flag);
+                ok = wait_phase(bar(P_FULL + (n & 1)), (n >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 if (KIND == kDKDV) {
@@ -562,7 +569,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_FULL));
+            mbar_arrive(bar(P_FULL + (n & 1)));
         }
         if (ok && n_all > 0) {
             const bool w = wait_phase(bar(DONE), 0, abort_flag);
