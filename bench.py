@@ -182,7 +182,11 @@ class Workload:
         per_copy = sum(v.numel() * v.element_size() for v in xp.values())
         self.p_copies = max(copies, -(-2 * L2_BYTES // per_copy)) if copies > 1 else 1
         self.pf = [{k: v.to(device) for k, v in xp.items()} for _ in range(self.p_copies)]
-        self.dc = [{k: v.to(device) for k, v in xd.items()} for _ in range(copies)]
+        # and enough decode copies that the bytes one rotation's calls touch (the valid
+        # tokens' K/V rows, not the whole pool) also span more than twice the L2
+        self.decode_bytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
+        self.d_copies = max(copies, -(-2 * L2_BYTES // self.decode_bytes)) if copies > 1 else 1
+        self.dc = [{k: v.to(device) for k, v in xd.items()} for _ in range(self.d_copies)]
         self.copies = copies
         self.p_out = torch.empty_like(self.pf[0]["q"])
         self.p_lse = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Lq, device=device)
@@ -190,7 +194,6 @@ class Workload:
         self.d_out = torch.empty_like(self.dc[0]["q"])
         self.d_lse = torch.empty(DECODE.num_seqs, DECODE.Hq, device=device)
         self.prefill_flops = PREFILL.flops() if window is None else windowed_flops(PREFILL, window)
-        self.decode_bytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
 
 
 def windowed_flops(spec, window) -> float:
@@ -211,7 +214,7 @@ def run_ours(args, ws, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     ta.load()
-    copies = args.copies  # default 4: 4 x 96 MiB prefill inputs, 4 x 67 MB decode pool > L2
+    copies = args.copies  # at least this many copies of each input (more where L2 needs it)
     w = Workload(device, copies, args.window)
     do_pre = args.only in ("both", "prefill")
     do_dec = args.only in ("both", "decode")
@@ -221,7 +224,7 @@ def run_ours(args, ws, rank, local):
 
     def step(i, ev=None):
         p = w.pf[i % w.p_copies]
-        d = w.dc[i % copies]
+        d = w.dc[i % w.d_copies]
         if ev is not None:
             ev[0].record(stream)
         if do_pre:
@@ -281,11 +284,11 @@ def run_ours(args, ws, rank, local):
                 ws=ws, device=device)
         if do_dec:
             g_dec = graph_launch_ms(
-                lambda i: ta.fwd_paged(w.dc[i % copies]["q"], w.dc[i % copies]["k_cache"],
-                                       w.dc[i % copies]["v_cache"], w.dc[i % copies]["block_table"],
-                                       w.dc[i % copies]["seq_lens"], scale=DECODE.scale,
+                lambda i: ta.fwd_paged(w.dc[i % w.d_copies]["q"], w.dc[i % w.d_copies]["k_cache"],
+                                       w.dc[i % w.d_copies]["v_cache"], w.dc[i % w.d_copies]["block_table"],
+                                       w.dc[i % w.d_copies]["seq_lens"], scale=DECODE.scale,
                                        out=w.d_out, lse=w.d_lse, workspace=ws_buf),
-                n_calls=4 * copies, replays=max(1, min(1000, args.steps) // (4 * copies)),
+                n_calls=2 * w.d_copies, replays=max(1, min(1000, args.steps) // (2 * w.d_copies)),
                 ws=ws, device=device)
 
     bwd_ms = None
@@ -351,7 +354,8 @@ def run_ours(args, ws, rank, local):
                        "bytes": w.decode_bytes},
             "l2": f"inputs rotate over device copies larger than the 126 MB L2: prefill "
                   f"{w.p_copies} x {sum(v.numel() * v.element_size() for v in w.xp_host.values()) / 1e6:.1f} MB, "
-                  f"decode pool {copies} x 67 MB",
+                  f"decode {w.d_copies} x {w.decode_bytes / 1e6:.1f} MB touched per call (pools of "
+                  f"{sum(v.numel() * v.element_size() for v in w.xd_host.values()) / 1e6:.0f} MB)",
             "parallelism": f"replicas x{ws} (independent problems per GPU)",
             "window": args.window,
         },

@@ -46,10 +46,11 @@ struct DecodeCfg {
     static constexpr int kTileBytes = kPageSize * 128;          // one 16-row x 64-column swizzled tile
     static constexpr int kKBytes = kPageSize * D * 2;           // one block's K rows (D/64 tiles)
     static constexpr int kStageBytes = 2 * kKBytes;             // K and V
-    // merge buffers, reusing the ring: per-warp O with padded rows plus the factors, or
-    // the chunk weights of one unit. A unit has at most (P - U) + 1 <= kDecMaxUnits + 1
-    // chunks, since P = max(kDecCtas, 2U) and U <= kDecMaxUnits.
-    static constexpr int kMergeBytes = kDecConsumers * kMaxGroup * (D + 8) * 4 + kDecConsumers * kMaxGroup * 4;
+    // merge buffers, reusing the ring: per-warp O with padded rows; the chunk weights of
+    // one unit (a unit has at most (P - U) + 1 <= kDecMaxUnits + 1 chunks, since
+    // P = max(kDecCtas, 2U) and U <= kDecMaxUnits); and, when they fit, a unit's partial
+    // outputs staged for its merge, with their weights.
+    static constexpr int kMergeBytes = kDecConsumers * kMaxGroup * (D + 8) * 4;
     static constexpr int kWeightBytes = (kDecMaxUnits + 1) * kMaxGroup * 4;
     static constexpr int kRingBytes = kDecStages * kStageBytes;
     static constexpr int kBufBytes = kRingBytes > kMergeBytes
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     constexpr int NT = D / 8;   // output n-tiles
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
+    __shared__ uint64_t merge_bar;  // the bulk copy of a unit's partials (last chunk only)
     __shared__ int stage_skip[kDecStages];
     __shared__ int s_nb[kDecMaxUnits];   // blocks per unit
     __shared__ int s_pre[kDecMaxUnits];  // first chunk index of each unit
@@ -304,6 +306,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
+        mbar_init(smem_u32(&merge_bar), 1);
         s_abort = 0;
         fence_barrier_init();
     }
@@ -485,10 +488,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
     // ---------------------------------------------------- merge this CTA's warps
     // Per-warp outputs in shared memory (row stride D + 8 floats keeps the fragment
-    // stores at most two-way bank conflicted), then one scale factor per (warp, row).
+    // stores at most two-way bank conflicted) with each warp's row maximum and sum.
     constexpr int kRow = D + 8;
     float* sm_o = reinterpret_cast<float*>(smem);  // [kDecConsumers][16][kRow]
-    float* sm_f = sm_o + kDecConsumers * kMaxGroup * kRow;  // [kDecConsumers][16] factors
     if (warp < kDecConsumers) {
         if (t == 0) {
             sm_m[warp][g] = m0;
@@ -507,41 +509,35 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         }
     }
     __syncthreads();
-    __shared__ float s_rowM[kMaxGroup], s_rowL[kMaxGroup];
-    if (tid < G) {
-        const int r = tid;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kDecConsumers; ++w) M = fmaxf(M, sm_m[w][r]);
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecConsumers; ++w) {
-            const float f = (M == -INFINITY) ? 0.f : ex2_approx(sm_m[w][r] - M);
-            sm_f[w * kMaxGroup + r] = f;
-            L += f * sm_l[w][r];
-        }
-        s_rowM[r] = M;
-        s_rowL[r] = L;
-    }
-    __syncthreads();
+    __shared__ float s_rowM[kMaxGroup], s_rowL[kMaxGroup];  // the unit merge's row statistics
 
+    // Each thread forms its row's combined maximum and weight from the four warps' (m, l)
+    // itself (no further barrier) and writes one 4-float slice of the normalised output.
     const bool direct = nchunk == 1;
     const int cidx = blockIdx.x;  // chunk index (balanced schedule; unused when direct)
     for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
         const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
-        const float L = s_rowL[r];
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) M = fmaxf(M, sm_m[w][r]);
+        float f[kDecConsumers], L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) {
+            f[w] = (M == -INFINITY) ? 0.f : ex2_approx(sm_m[w][r] - M);
+            L += f[w] * sm_l[w][r];
+        }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kDecConsumers; ++w) {
-            const float f = sm_f[w * kMaxGroup + r] * inv;
+            const float fw = f[w] * inv;
             const float4 v = *reinterpret_cast<const float4*>(sm_o + (w * kMaxGroup + r) * kRow + d);
-            o.x += f * v.x;
-            o.y += f * v.y;
-            o.z += f * v.z;
-            o.w += f * v.w;
+            o.x += fw * v.x;
+            o.y += fw * v.y;
+            o.z += fw * v.z;
+            o.w += fw * v.w;
         }
-        const float lse2 = L > 0.f ? s_rowM[r] + log2f(L) : -INFINITY;
+        const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
         if (direct) {
             const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
             uint2 pk;
@@ -558,29 +554,33 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (direct) return;
 
     // ---------------------------------------------- the last chunk merges the unit
-    __threadfence();
+    // One gpu-scope acquire-release add by thread 0 after the CTA barrier: its release
+    // publishes the partial stores of every thread (the barrier orders them before it),
+    // its acquire makes the other chunks' partials visible here.
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&a.ws_count[unit], 1) == nchunk - 1;
+    if (tid == 0) s_last = atom_add_acq_rel_gpu(&a.ws_count[unit], 1) == nchunk - 1;
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    // The partial outputs of this thread's first output slice, chunks 0..7, are loaded
-    // now, so their round trip overlaps the one for the log2-sum-exp values below.
-    const size_t step = static_cast<size_t>(G) * D / 4;  // float4 stride between chunks
-    float4 pre[8];
-    if (tid < G * (D / 4)) {
-        const float4* src = reinterpret_cast<const float4*>(
-            a.ws_o + (static_cast<size_t>(chunk0) * G + tid / (D / 4)) * D + (tid % (D / 4)) * 4);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            pre[u] = (u < nchunk) ? __ldcg(src + u * step) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // All chunks' log2-sum-exp in shared memory at once (one round of parallel loads),
-    // then per row the maximum, the total weight and each chunk's normalised weight.
-    float* s_w = sm_o;  // [nchunk][G], reused
+    const float* part = a.ws_o + static_cast<size_t>(chunk0) * G * D;  // [nchunk][G][D]
+    const float* plse = a.ws_lse + static_cast<size_t>(chunk0) * G;     // [nchunk][G]
     const int nw = nchunk * G;
-    for (int i = tid; i < nw; i += blockDim.x)
-        s_w[i] = __ldcg(a.ws_lse + static_cast<size_t>(chunk0) * G + i);
+    const uint32_t part_bytes = static_cast<uint32_t>(nw) * D * sizeof(float);
+    // The unit's partials are contiguous: when they fit the ring they arrive by one bulk
+    // copy (one round trip), else every thread loads its slices from L2.
+    const bool staged = static_cast<size_t>(nw) * (D + 1) * sizeof(float) <= Cfg::kBufBytes;
+    float* s_part = reinterpret_cast<float*>(smem);
+    float* s_w = staged ? s_part + static_cast<size_t>(nw) * D : reinterpret_cast<float*>(smem);
+    if (staged && tid == 0) {
+        // the copy reads what the acquire made visible, and writes ring bytes the
+        // barrier above ordered after their last generic use
+        fence_proxy_async_global();
+        fence_proxy_async_shared();
+        mbar_arrive_expect_tx(smem_u32(&merge_bar), part_bytes);
+        bulk_load(smem_u32(s_part), part, part_bytes, smem_u32(&merge_bar));
+    }
+    // All chunks' log2-sum-exp in shared memory (one round of parallel loads), then per
+    // row the maximum, the total weight and each chunk's normalised weight.
+    for (int i = tid; i < nw; i += blockDim.x) s_w[i] = __ldcg(plse + i);
     __syncthreads();
     for (int r = warp; r < G; r += kDecThreads / 32) {
         float M = -INFINITY;
@@ -603,30 +603,54 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const float M = s_rowM[r], W = s_rowL[r];
         s_w[i] = (M == -INFINITY || !(W > 0.f)) ? 0.f : ex2_approx(s_w[i] - M) / W;
     }
+    if (staged && tid == 0 && !wait_phase(smem_u32(&merge_bar), 0, abort_flag))
+        drain_phase(smem_u32(&merge_bar), 0);  // gave up (reported): let the copy land
     __syncthreads();
-    // Each thread owns one 4-float slice of the output and sums it over the chunks,
-    // eight independent loads in flight at a time.
+    if (*abort_flag) return;
+    // Each thread owns 4-float slices of the output and sums them over the chunks.
     for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
         const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
-        const float4* src = reinterpret_cast<const float4*>(a.ws_o + (static_cast<size_t>(chunk0) * G + r) * D + d);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < nchunk; k += 8) {
-            float4 v[8];
-            if (k == 0 && i4 == tid) {  // prefetched above
+        if (staged) {
+            // four independent sums over the chunks keep four loads in flight
+            const float4* src = reinterpret_cast<const float4*>(s_part + r * D + d);
+            const int step = G * D / 4;  // float4 stride between chunks
+            float4 part4[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = pre[u];
-            } else {
+            for (int u = 0; u < 4; ++u) part4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k < nchunk; k += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (k + u < nchunk) {
+                        const float w = s_w[(k + u) * G + r];
+                        const float4 v = src[(k + u) * step];
+                        part4[u].x += w * v.x;
+                        part4[u].y += w * v.y;
+                        part4[u].z += w * v.z;
+                        part4[u].w += w * v.w;
+                    }
+                }
+            }
+            acc.x = (part4[0].x + part4[1].x) + (part4[2].x + part4[3].x);
+            acc.y = (part4[0].y + part4[1].y) + (part4[2].y + part4[3].y);
+            acc.z = (part4[0].z + part4[1].z) + (part4[2].z + part4[3].z);
+            acc.w = (part4[0].w + part4[1].w) + (part4[2].w + part4[3].w);
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(part + r * D + d);
+            const size_t step = static_cast<size_t>(G) * D / 4;
+            for (int k = 0; k < nchunk; k += 8) {
+                float4 v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     v[u] = (k + u < nchunk) ? __ldcg(src + (k + u) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float w = (k + u < nchunk) ? s_w[(k + u) * G + r] : 0.f;
-                acc.x += w * v[u].x;
-                acc.y += w * v[u].y;
-                acc.z += w * v[u].z;
-                acc.w += w * v[u].w;
+                for (int u = 0; u < 8; ++u) {
+                    const float w = (k + u < nchunk) ? s_w[(k + u) * G + r] : 0.f;
+                    acc.x += w * v[u].x;
+                    acc.y += w * v[u].y;
+                    acc.z += w * v[u].z;
+                    acc.w += w * v[u].w;
+                }
             }
         }
         const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
