@@ -122,6 +122,22 @@ def test_decode_skewed_lengths_balanced_schedule():
     check_parity(out, lse, ro, rl, s.dtype, "skewed")
 
 
+def test_decode_one_sequence_of_a_million_tokens():
+    """One sequence of 2^20 tokens (65,536 blocks through the table) and one of 5 tokens,
+    H_q 8 / H_kv 1: the long unit is cut into about 290 chunks, too many partial outputs
+    to stage in shared memory, so its merge reads them from L2; the other unit has one
+    chunk and writes directly."""
+    lens = (1 << 20, 5)
+    s = inputs.PagedSpec("t", 2, 8, 1, 128, 16, 1 << 20, torch.bfloat16, 1 / math.sqrt(128),
+                         seed=33, fixed_lens=lens)
+    x = inputs.make(s)
+    out, lse = run_paged(x, s.scale, guard=True)
+    assert ta.device_status() == 0
+    ro, rl = oracle.attn_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
+                               x["seq_lens"], s.scale)
+    check_parity(out, lse, ro, rl, s.dtype, "one long sequence")
+
+
 def test_decode_many_units_one_cta_each():
     # more than 1024 (sequence, K/V head) units: each CTA takes a whole unit, no split
     s = inputs.PagedSpec("t", 520, 4, 2, 64, 16, 160, torch.float16, 0.125, seed=32, min_len=0)

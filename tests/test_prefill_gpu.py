@@ -160,3 +160,33 @@ def test_long_prefill_sampled_rows():
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
     vmax = x["v"].float().abs().amax(dim=(2, 3)).view(1, s.Hq, 1, 1)
     assert torch.all(out.float().abs() <= vmax * (1 + 2 ** -7) + 1e-6)
+
+
+@pytest.mark.parametrize("Lq,Lk,causal", [(256, 1 << 22, False), (1 << 22, 384, False),
+                                          (1 << 22, 384, True)],
+                         ids=["max_keys", "max_queries", "max_queries_causal"])
+def test_maximum_sequence_lengths_sampled_rows(Lq, Lk, causal):
+    """The longest sequences attn_fwd accepts (2^22 queries or keys; one head, D 64, bf16):
+    32k key tiles streamed by one CTA, or 16k query tiles. With Lq > Lk the causal band
+    is bottom-right aligned, so all but the last Lk rows see no key (O = 0, lse = -inf).
+    The oracle checks sampled rows, including both sides of that edge."""
+    s = inputs.DenseSpec("maxlen", 1, 1, 1, Lq, Lk, 64, torch.bfloat16, causal, 0.125,
+                         seed=Lq % 1000 + Lk % 1000)
+    x = inputs.make(s)
+    out, lse = run(x["q"], x["k"], x["v"], causal, s.scale)
+    g = torch.Generator().manual_seed(5)
+    edge = Lq - Lk  # first row that sees a key under the causal mask
+    picks = {0, 1, 127, 128, Lq - 1} | set(torch.randint(0, Lq, (3,), generator=g).tolist())
+    if causal:
+        picks |= {edge - 1, edge, edge + 1, edge + 127, edge + 128}
+    rows = sorted(picks)
+    ro, rl = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, s.scale, causal)
+    rows_t = torch.tensor(rows)
+    check_parity(out.reshape(-1, 64)[rows_t], lse.reshape(-1)[rows_t], ro, rl, s.dtype,
+                 f"Lq {Lq} Lk {Lk} causal {causal}")
+    if causal:
+        assert torch.count_nonzero(out[0, 0, :edge]) == 0
+        assert torch.all(lse[0, 0, :edge] == -math.inf)
+        assert torch.isfinite(lse[0, 0, edge:]).all()
+    else:
+        assert torch.isfinite(lse).all()
