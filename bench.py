@@ -311,9 +311,11 @@ def run_ours(args, ws, rank, local):
         e2e = measure_e2e(w, ta, stream, device, steps=max(3, min(20, args.steps)), window=args.window)
     else:
         e2e = {"prefill_ms": float("nan"), "decode_ms": float("nan"), "h2d_bytes": 0,
-               "d2h_bytes": 0}
+               "d2h_bytes": 0, "serial_prefill_ms": float("nan"), "serial_decode_ms": float("nan")}
     e2e_pre = reduce_max(e2e["prefill_ms"], ws, device)
     e2e_dec = reduce_max(e2e["decode_ms"], ws, device)
+    e2e_pre_serial = reduce_max(e2e["serial_prefill_ms"], ws, device)
+    e2e_dec_serial = reduce_max(e2e["serial_decode_ms"], ws, device)
 
     if rank != 0:
         return None
@@ -326,6 +328,8 @@ def run_ours(args, ws, rank, local):
     r2 = lambda x, n: None if x is None else round(x, n)  # noqa: E731
     e2e_tf = job_rate(w.prefill_flops, e2e_pre, ws, 1e12) if do_pre else None
     e2e_gb = job_rate(w.decode_bytes, e2e_dec, ws, 1e9) if do_dec else None
+    e2e_tf_serial = job_rate(w.prefill_flops, e2e_pre_serial, ws, 1e12) if do_pre else None
+    e2e_gb_serial = job_rate(w.decode_bytes, e2e_dec_serial, ws, 1e9) if do_dec else None
     pk_t = peaks["bf16_tflops_sustained"]
     pk_h = peaks["hbm_gbs"]
     line = {
@@ -398,8 +402,13 @@ def run_ours(args, ws, rank, local):
             "h2d_bytes_per_step": e2e["h2d_bytes"],
             "d2h_bytes_per_step": e2e["d2h_bytes"],
             "paged_decode_gbs": r2(e2e_gb, 2),
-            "how": "pinned host inputs copied to the device, the C-ABI call, outputs copied back, "
-                   "all on one stream inside the timed region",
+            "how": "every step copies its inputs from pinned host memory to the device, makes the "
+                   "C-ABI call and copies its outputs back, all inside the timed region; two "
+                   "buffer sets let step i+1's host-to-device copies overlap step i's call and "
+                   "step i-1's device-to-host copies (three streams, event-ordered)",
+            "serial_value": r2(e2e_tf_serial, 3),
+            "serial_paged_decode_gbs": r2(e2e_gb_serial, 2),
+            "serial_how": "the same steps on one stream with a host sync after each step",
         },
         "gpu_launches": (int(do_pre) + int(do_dec)) * args.steps,
         "clocks": clocks.summary(),
@@ -622,44 +631,103 @@ def measure_fp8(w, ta, stream, device, steps: int, warmup: int, ws: int):
     return reduce_max(sum(a.elapsed_time(b) for a, b in ev) / steps, ws, device)
 
 
+def _pipelined_ms(host_in: dict, out_like: dict, call, steps: int, warmup: int, device) -> float:
+    """ms per step of a double-buffered loop through the public API: the H2D copies of
+    step i+1 (one copy stream) overlap the call of step i (a compute stream) and the D2H
+    copies of step i-1 (a second copy stream). Every step's copies are inside the timed
+    region, which runs from the first timed H2D to the last D2H."""
+    sets = 2
+    dev_in = [{k: torch.empty_like(v, device=device) for k, v in host_in.items()} for _ in range(sets)]
+    dev_out = [{k: torch.empty_like(v, device=device) for k, v in out_like.items()} for _ in range(sets)]
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in out_like.items()}
+    s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    n = warmup + steps
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_run = [torch.cuda.Event() for _ in range(n)]
+    ev_out = [torch.cuda.Event() for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    for i in range(n):
+        if i == warmup:  # the timed region starts once the warm-up steps have drained
+            torch.cuda.synchronize()
+            t0.record(s_in)
+        b = i % sets
+        if i >= sets:
+            s_in.wait_event(ev_run[i - sets])   # step i-2's call read input set b
+        with torch.cuda.stream(s_in):
+            for k, v in host_in.items():
+                dev_in[b][k].copy_(v, non_blocking=True)
+        ev_in[i].record(s_in)
+        s_run.wait_event(ev_in[i])
+        if i >= sets:
+            s_run.wait_event(ev_out[i - sets])  # step i-2's D2H read output set b
+        call(dev_in[b], dev_out[b], s_run)
+        ev_run[i].record(s_run)
+        s_out.wait_event(ev_run[i])
+        with torch.cuda.stream(s_out):
+            for k, v in host_out.items():
+                v.copy_(dev_out[b][k], non_blocking=True)
+        ev_out[i].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
 def measure_e2e(w, ta, stream, device, steps: int, window=None):
     """Same metric through the public API with host buffers: H2D of the step's inputs
-    from pinned memory, the call, D2H of its outputs, all inside the timed region."""
+    from pinned memory, the call, D2H of its outputs, all inside the timed region.
+    Reported: a double-buffered loop (copies in both directions overlap the calls, as a
+    serving loop would run them) and, for context, the same steps one after another on
+    one stream with a host sync per step."""
     hp = {k: v.pin_memory() for k, v in w.xp_host.items()}
     hd = {k: v.pin_memory() for k, v in w.xd_host.items()}
-    dp = {k: torch.empty_like(v, device=device) for k, v in hp.items()}
-    dd = {k: torch.empty_like(v, device=device) for k, v in hd.items()}
-    op = torch.empty_like(w.p_out, device="cpu").pin_memory()
-    lp = torch.empty_like(w.p_lse, device="cpu").pin_memory()
-    od = torch.empty_like(w.d_out, device="cpu").pin_memory()
-    ld = torch.empty_like(w.d_lse, device="cpu").pin_memory()
     wsb = ta.paged_workspace(DECODE.num_seqs, DECODE.Hq, DECODE.Hkv, DECODE.D, DECODE.max_blocks,
                              device)
+    p_like = {"out": w.p_out, "lse": w.p_lse}
+    d_like = {"out": w.d_out, "lse": w.d_lse}
     h2d = sum(v.numel() * v.element_size() for v in list(hp.values()) + list(hd.values()))
-    d2h = sum(t.numel() * t.element_size() for t in (op, lp, od, ld))
+    d2h = sum(t.numel() * t.element_size() for t in list(p_like.values()) + list(d_like.values()))
+
+    def pre_call(di, do, st):
+        ta.fwd(di["q"], di["k"], di["v"], causal=PREFILL.causal, scale=PREFILL.scale,
+               out=do["out"], lse=do["lse"], stream=st, window=window)
+
+    def dec_call(di, do, st):
+        ta.fwd_paged(di["q"], di["k_cache"], di["v_cache"], di["block_table"], di["seq_lens"],
+                     scale=DECODE.scale, out=do["out"], lse=do["lse"], workspace=wsb, stream=st)
+
+    pre_ms = _pipelined_ms(hp, p_like, pre_call, steps, 2, device)
+    dec_ms = _pipelined_ms(hd, d_like, dec_call, steps, 2, device)
+
+    # the serial form: one stream, H2D -> call -> D2H, a host sync after every step
+    dp = {k: torch.empty_like(v, device=device) for k, v in hp.items()}
+    dd = {k: torch.empty_like(v, device=device) for k, v in hd.items()}
+    op = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in p_like.items()}
+    od = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in d_like.items()}
     pre, dec = [], []
     for it in range(steps + 1):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record(stream)
-        for k in dp:
-            dp[k].copy_(hp[k], non_blocking=True)
-        ta.fwd(dp["q"], dp["k"], dp["v"], causal=PREFILL.causal, scale=PREFILL.scale, out=w.p_out,
-               lse=w.p_lse, stream=stream, window=window)
-        op.copy_(w.p_out, non_blocking=True)
-        lp.copy_(w.p_lse, non_blocking=True)
+        with torch.cuda.stream(stream):
+            for k in dp:
+                dp[k].copy_(hp[k], non_blocking=True)
+            pre_call(dp, p_like, stream)
+            for k in op:
+                op[k].copy_(p_like[k], non_blocking=True)
         e[1].record(stream)
-        for k in dd:
-            dd[k].copy_(hd[k], non_blocking=True)
-        ta.fwd_paged(dd["q"], dd["k_cache"], dd["v_cache"], dd["block_table"], dd["seq_lens"],
-                     scale=DECODE.scale, out=w.d_out, lse=w.d_lse, workspace=wsb, stream=stream)
-        od.copy_(w.d_out, non_blocking=True)
-        ld.copy_(w.d_lse, non_blocking=True)
+        with torch.cuda.stream(stream):
+            for k in dd:
+                dd[k].copy_(hd[k], non_blocking=True)
+            dec_call(dd, d_like, stream)
+            for k in od:
+                od[k].copy_(d_like[k], non_blocking=True)
         e[2].record(stream)
         torch.cuda.synchronize()
         if it > 0:  # the first pass warms up
             pre.append(e[0].elapsed_time(e[1]))
             dec.append(e[1].elapsed_time(e[2]))
-    return {"prefill_ms": sum(pre) / len(pre), "decode_ms": sum(dec) / len(dec),
+    return {"prefill_ms": pre_ms, "decode_ms": dec_ms,
+            "serial_prefill_ms": sum(pre) / len(pre), "serial_decode_ms": sum(dec) / len(dec),
             "h2d_bytes": h2d, "d2h_bytes": d2h}
 
 
