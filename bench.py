@@ -405,7 +405,10 @@ def run_ours(args, ws, rank, local):
             "how": "every step copies its inputs from pinned host memory to the device, makes the "
                    "C-ABI call and copies its outputs back, all inside the timed region; two "
                    "buffer sets let step i+1's host-to-device copies overlap step i's call and "
-                   "step i-1's device-to-host copies (three streams, event-ordered)",
+                   "step i-1's device-to-host copies (three streams, event-ordered). The prefill "
+                   "and the decode each run such a loop: value is the prefill's TFLOP/s over its "
+                   "loop, paged_decode_gbs the decode's; the byte counts are one whole step's "
+                   "(prefill and decode inputs and outputs)",
             "serial_value": r2(e2e_tf_serial, 3),
             "serial_paged_decode_gbs": r2(e2e_gb_serial, 2),
             "serial_how": "the same steps on one stream with a host sync after each step",
