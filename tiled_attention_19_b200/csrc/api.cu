@@ -68,24 +68,6 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view (D, L, planes) of a contiguous [planes, L, D] tensor; box 64 x box_rows x 1
-// with 128-byte swizzle. Rows past L read as zero and are never written.
-bool encode_tile_map(CUtensorMap* tm, const void* base, bool bf16, int D, int L, long long planes,
-                     int box_rows = attn::kBM) {
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
-                                static_cast<cuuint64_t>(planes)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                                   static_cast<cuuint64_t>(L) * D * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Element strides of a (batch, head, row) tensor with contiguous rows of D elements.
 struct Strides {
     long long b, h, l;
