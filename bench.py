@@ -24,6 +24,7 @@ scaling); rank 0 prints the whole-job throughput over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -864,9 +865,18 @@ def main(argv=None):
     ap.add_argument("--prefill-workload", default=PREFILL_DEFAULT,
                     choices=[n for n, w in inputs.WORKLOADS.items() if w.kind == "dense"],
                     help="dense workload of the prefill call (default: the long causal prefill)")
+    ap.add_argument("--decode-seqs", type=int, default=None,
+                    help="the decode workload with this many sequences instead of 16 (same "
+                         "length distribution, heads and seed): how its GB/s grows with the batch")
     args = ap.parse_args(argv)
-    global PREFILL
+    global PREFILL, DECODE
     PREFILL = inputs.WORKLOADS[args.prefill_workload]
+    if args.decode_seqs is not None:
+        if args.decode_seqs < 1:
+            ap.error("--decode-seqs must be >= 1")
+        DECODE = dataclasses.replace(DECODE, num_seqs=args.decode_seqs,
+                                     name=DECODE.name.replace(f"_s{DECODE.num_seqs}_",
+                                                              f"_s{args.decode_seqs}_"))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()

@@ -11,12 +11,14 @@
 // Work split. A unit is one (sequence, K/V head); its G = H_q / H_kv query heads are
 // the rows of one m16n8k16 tensor-core tile (rows >= G are zero), so every K/V byte is
 // read once. The grid has P = max(kDecCtas, 2U) CTAs for U units. Every CTA reads the
-// sequence lengths and derives the same schedule: the blocks of all units (T in total)
-// are cut into chunks of at most C = ceil(T / (P - U)) blocks, each unit into
-// ceil(blocks / C) near-equal chunks (at least one), which gives at most P chunks; CTA
-// c takes chunk c. One wave of CTAs with equal shares of the bytes: the kernel is bound
-// by HBM bandwidth, not by its longest sequence. (With more than kDecMaxUnits units
-// each CTA takes one whole unit instead.)
+// sequence lengths and derives the same schedule: each unit is cut into
+// max(1, ceil(blocks / C)) near-equal chunks, with C the smallest chunk size whose
+// chunk count over all units fits P (a binary search between ceil(T / P) and
+// ceil(T / (P - U)), which always fits; T = all units' blocks) while P is one wave of
+// kDecCtas, else ceil(T / (P - U)); CTA c takes chunk c.
+// One wave of CTAs with near-equal shares of the bytes: the kernel is bound by HBM
+// bandwidth, not by its longest sequence. (With more than kDecMaxUnits units each CTA
+// takes one whole unit instead.)
 //
 // Per CTA: a producer warp reads the chunk's block-table entries and issues 2-D TMA
 // loads (128-byte swizzle) of each block's K and V rows into a ring of shared-memory
@@ -24,9 +26,9 @@
 // ldmatrix (.trans for V), so the swizzle keeps the reads free of bank conflicts. Each
 // warp keeps its own running max, sum and output; the CTA merges its warps in shared
 // memory. A unit with one chunk writes O and lse directly; otherwise every chunk writes
-// its normalised output and log2-sum-exp to the workspace, fences and bumps the unit's
-// counter, and the CTA that completes the count merges the chunks and resets the
-// counter to zero.
+// its normalised output and log2-sum-exp to the workspace and bumps the unit's counter
+// with an acquire-release atomic, and the CTA that completes the count merges the
+// chunks and resets the counter to zero.
 #pragma once
 #include <cuda.h>
 
@@ -198,7 +200,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
             const int P = gridDim.x;
-            const int C = max(1, (T + (P - U) - 1) / (P - U));
+            // The smallest chunk size C whose chunk count sum_u max(1, ceil(blocks_u / C))
+            // fits the P CTAs: a binary search between ceil(T / P), below which the count
+            // exceeds P, and ceil(T / (P - U)), which always fits. (Here P is one wave.)
+            int C = max(1, (T + (P - U) - 1) / (P - U));
+            for (int lo = max(1, (T + P - 1) / P); lo < C;) {
+                const int mid = (lo + C) >> 1;
+                int cnt = lane < U ? max(1, (nbu + mid - 1) / mid) : 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+                if (cnt <= P) C = mid;
+                else lo = mid + 1;
+            }
             const int v = lane < U ? max(1, (nbu + C - 1) / C) : 0;
             int x = v;
 #pragma unroll
@@ -245,7 +258,26 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         for (int w = 0; w < kDecThreads / 32; ++w) T += s_red[w];
         __syncthreads();
         const int P = gridDim.x;  // P >= 2U, so P - U >= U >= 1
-        const int C = static_cast<int>(max(1LL, (T + (P - U) - 1) / (P - U)));
+        // the smallest feasible chunk size, as in the one-warp schedule above (every
+        // thread takes the same branches: the counts are CTA-wide sums), while the grid
+        // is one wave; a grid of several waves balances itself, and there fewer, larger
+        // chunks cost less
+        int C = static_cast<int>(max(1LL, (T + (P - U) - 1) / (P - U)));
+        for (int lo = P == kDecCtas ? static_cast<int>(max(1LL, (T + P - 1) / P)) : C; lo < C;) {
+            const int mid = (lo + C) >> 1;
+            int cnt = 0;
+            for (int u = tid; u < U; u += blockDim.x) cnt += max(1, (s_nb[u] + mid - 1) / mid);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+            if (lane == 0) s_red[warp] = cnt;
+            __syncthreads();
+            long long total = 0;
+#pragma unroll
+            for (int w = 0; w < kDecThreads / 32; ++w) total += s_red[w];
+            __syncthreads();
+            if (total <= P) C = mid;
+            else lo = mid + 1;
+        }
         // pass 2: exclusive prefix over units of the chunk counts max(1, ceil(blocks / C))
         int carry = 0;
         for (int base = 0; base < U; base += blockDim.x) {
