@@ -64,3 +64,21 @@ def test_reference_arm_prints_only_on_rank_zero(monkeypatch):
     class A:
         steps, warmup, cpu_seconds = 1, 3, 0.1
     assert bench.run_reference(A(), 2, 1) is None   # rank 1: no work, exits quietly
+
+
+def test_decode_seqs_option_scales_the_decode_workload(monkeypatch, capsys):
+    """--decode-seqs N swaps in the decode workload with N sequences (same heads, length
+    distribution and seed); the reference arm, which runs on the host, reports it."""
+    import json
+    monkeypatch.setattr(bench, "DECODE", bench.DECODE)    # main() rebinds the workloads
+    monkeypatch.setattr(bench, "PREFILL", bench.PREFILL)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--impl", "reference", "--decode-seqs", "4", "--steps", "1",
+                       "--warmup", "3", "--cpu-seconds", "0.2"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert "paged_decode_s4_hq12_hkv2_d128_bf16" in line["config"]["workload"]
+    assert bench.DECODE.num_seqs == 4 and bench.DECODE.Hq == 12 and bench.DECODE.seed == 5
+    with pytest.raises(SystemExit):
+        bench.main(["--decode-seqs", "0"])
