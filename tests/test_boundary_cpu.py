@@ -306,3 +306,14 @@ def test_attn_fwd_fp8_validation():
     assert call(dq=float("nan")) == -1
     assert call(q=None) == -1
     assert call(qs=S(16 * 128, 8 * 128, 136)) == -3  # 136-byte rows: not a multiple of 16
+
+
+def test_binding_refuses_tensors_off_the_current_device(monkeypatch):
+    """The library launches on the calling thread's current device: the binding checks
+    every tensor's and stream's device against it before any call."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    ta._on_current_device(torch.device("cuda", 0), "q")          # the current device: fine
+    with pytest.raises(ValueError, match="cuda:1"):
+        ta._on_current_device(torch.device("cuda", 1), "k")
+    with pytest.raises(ValueError, match="CUDA tensor"):        # host tensors never get that far
+        ta.fwd(torch.zeros(1, 1, 8, 64), torch.zeros(1, 1, 8, 64), torch.zeros(1, 1, 8, 64))

@@ -108,12 +108,25 @@ def _dtype_code(dt: torch.dtype) -> int:
 def _stream(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
-    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+    if isinstance(stream, torch.cuda.Stream):
+        _on_current_device(stream.device, "stream")
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _on_current_device(device: torch.device, name: str) -> None:
+    """The library launches its kernels on the calling thread's current CUDA device, so
+    every tensor and stream of a call must live there."""
+    cur = torch.cuda.current_device()
+    if device.index != cur:
+        raise ValueError(f"{name} is on {device} but the current CUDA device is cuda:{cur} "
+                         "(select it with torch.cuda.set_device or torch.cuda.device)")
 
 
 def _dev(t: torch.Tensor, name: str) -> int:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    _on_current_device(t.device, name)
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
@@ -127,6 +140,7 @@ def _check(rc: int, what: str) -> None:
 def _strides(t: torch.Tensor, name: str) -> Strides:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    _on_current_device(t.device, name)
     if t.dim() != 4 or t.stride(3) != 1:
         raise ValueError(f"{name} must be a 4-D view [B, H, L, D] with contiguous D")
     return Strides(t.stride(0), t.stride(1), t.stride(2))
@@ -313,7 +327,7 @@ def fwd_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = paged_workspace(S, Hq, Hkv, D, MB, q.device, bs)
-    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
     ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
     rc = load().attn_fwd_paged(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                                _dev(block_table, "block_table"), _dev(seq_lens, "seq_lens"), bs,
