@@ -26,7 +26,7 @@ P = 0x10000  # a 16-byte-aligned fake address (never dereferenced: every call is
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
 
 
 def test_header_declares_expected_entry_points():
@@ -41,6 +41,26 @@ def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
         assert name in ta.SIGNATURES, f"{name} has no binding signature"
+
+
+def declared_arities():
+    """Parameter count of every attn_* function the header declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(attn_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Each ctypes signature has as many arguments as the C declaration: a parameter
+    added to the header without the binding (or the reverse) fails here, on the CPU."""
+    arity = declared_arities()
+    assert set(arity) == set(declared_functions())
+    for name, n in arity.items():
+        assert len(ta.SIGNATURES[name][1]) == n, (name, n, len(ta.SIGNATURES[name][1]))
 
 
 def test_error_strings():
