@@ -88,56 +88,127 @@ def profiled_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks, power and clock-event (throttle) reasons, polled through NVML every
+    few milliseconds from a background thread for the whole measurement, each sample
+    stamped with the host clock; summary() keeps the samples inside a host-time window
+    (the timed region), so even a region of a few milliseconds gets samples. Falls back
+    to `nvidia-smi -lms` (50 ms period) where NVML cannot be loaded. Reads only."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    SMI_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int, period_ms: int = 50):
-        self.index, self.period, self.rows, self.proc = index, period_ms, [], None
+    def __init__(self, device, period_ms: float = 2.0):
+        self.device, self.period = device, period_ms / 1e3
+        self.samples = []  # (host time, sm MHz, max sm MHz, power W, [reasons])
+        self.stop = threading.Event()
+        self.thread = None
+        self.proc = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except pynvml.NVMLError:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = self.device.index or 0
+        if vis:
+            idx = int(vis.split(",")[idx])
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", f"-lms={self.period}"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-            # nvidia-smi takes a moment to start: begin the timed region once it samples
-            t0 = time.perf_counter()
-            while not self.rows and time.perf_counter() - t0 < 5.0 and self.proc.poll() is None:
-                time.sleep(0.01)
-            self.rows.clear()
-        except (OSError, ValueError):
-            self.proc = None
+            nv, h = self._nvml_handle()
+            masks = [(n, getattr(nv, c)) for n, c in self.REASONS]
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+            def poll():
+                while not self.stop.is_set():
+                    t = time.perf_counter()
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1e3
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except nv.NVMLError:
+                        break
+                    self.samples.append((t, float(sm), float(mx), pw,
+                                         [n for n, m in masks if r & m]))
+                    time.sleep(self.period)
+
+            self.source = f"NVML, every {self.period * 1e3:.0f} ms"
+        except Exception:  # no NVML: nvidia-smi at its shortest period
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.device.index or 0}", f"--query-gpu={self.SMI_Q}",
+                     "--format=csv,noheader,nounits", "-lms=50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, ValueError):
+                return self
+            names = [n for n, _ in self.REASONS]
+
+            def poll():
+                for line in self.proc.stdout:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                        self.samples.append((time.perf_counter(), float(p[1]), float(p[2]),
+                                             float(p[3]) if p[3].replace(".", "").isdigit() else None,
+                                             [n for n, v in zip(names, p[5:9]) if v == "Active"]))
+
+            self.source = "nvidia-smi -lms 50"
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        t0 = time.perf_counter()  # start measuring once the sampler delivers
+        while not self.samples and time.perf_counter() - t0 < 5.0:
+            time.sleep(0.005)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
-
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
             self.thread.join(timeout=5)
 
-    def summary(self):
-        if not self.rows:
+    def summary(self, t_from: float, t_to: float):
+        """Samples taken between host times t_from and t_to; if none fell inside (a
+        region shorter than the period), the nearest sample on each side."""
+        inside = [x for x in self.samples if t_from <= x[0] <= t_to]
+        how = "inside the timed region"
+        if not inside and self.samples:
+            before = [x for x in self.samples if x[0] < t_from][-1:]
+            after = [x for x in self.samples if x[0] > t_to][:1]
+            inside = before + after
+            how = "nearest samples on either side of the timed region"
+        if not inside:
             return None
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.rows)}
+        sm = [x[1] for x in inside]
+        pw = [x[3] for x in inside if x[3] is not None]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[2] for x in inside),
+                "sm_min_mhz": min(sm), "power_w": round(statistics.median(pw), 1) if pw else None,
+                "reasons": sorted({r for x in inside for r in x[4]}), "samples": len(inside),
+                "source": f"{self.source}; {how}"}
+
+
+def tensor_peak(peaks: dict, region_ms: float):
+    """The measured tensor peak that applies to a kernel timed over `region_ms`: the
+    burst GEMM rate below one second of timed work, the sustained (power-capped) rate
+    above it."""
+    if region_ms < 1000.0:
+        return peaks["bf16_tflops"], "bf16_tflops (burst: the timed region is under 1 s)"
+    return peaks["bf16_tflops_sustained"], "bf16_tflops_sustained (the timed region is over 1 s)"
 
 
 def dist_env():
@@ -210,11 +281,24 @@ def windowed_flops(spec, window) -> float:
     return 4.0 * spec.D * spec.B * spec.Hq * pairs
 
 
+SMALL_CONFIGS = ("sdpa_b1_h8_l512_d64_f16", "vit_b32_h12_n196_d64_f16",
+                 "sdpa_causal_b2_h8_l2048_d64_f16")
+
+
 def run_ours(args, ws, rank, local):
     import tiled_attention_19_b200 as ta
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     ta.load()
+    clocks = ClockSampler(device)
+    clocks.__enter__()  # samples the whole run; each timed region picks its own window
+    try:
+        return _run_ours(args, ws, rank, ta, device, clocks)
+    finally:
+        clocks.__exit__(None, None, None)
+
+
+def _run_ours(args, ws, rank, ta, device, clocks):
     copies = args.copies  # at least this many copies of each input (more where L2 needs it)
     w = Workload(device, copies, args.window)
     do_pre = args.only in ("both", "prefill")
@@ -252,15 +336,16 @@ def run_ours(args, ws, rank, local):
     t1 = torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize()
-    with ClockSampler(device.index if device.index is not None else 0) as clocks:
-        t0.record(stream)
-        h0 = time.perf_counter()
-        for i in range(args.steps):
-            step(args.warmup + i, evs[i])
-        host_ms = (time.perf_counter() - h0) * 1e3  # host time to enqueue the K steps
-        t1.record(stream)
-        torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    host_ms = (time.perf_counter() - h0) * 1e3  # host time to enqueue the K steps
+    t1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.perf_counter()
     barrier(ws)
+    region_clocks = clocks.summary(h0, h1)
     total_ms = t0.elapsed_time(t1)
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
@@ -291,6 +376,11 @@ def run_ours(args, ws, rank, local):
                                        out=w.d_out, lse=w.d_lse, workspace=ws_buf),
                 n_calls=2 * w.d_copies, replays=max(1, min(1000, args.steps) // (2 * w.d_copies)),
                 ws=ws, device=device)
+
+    cfg = None
+    if args.configs and args.window is None:
+        cfg = measure_configs(ta, device, ws, steps=max(20, min(200, args.steps)),
+                              warmup=args.warmup, clocks=clocks)
 
     bwd_ms = None
     if args.backward and do_pre:
@@ -331,7 +421,7 @@ def run_ours(args, ws, rank, local):
     e2e_gb = job_rate(w.decode_bytes, e2e_dec, ws, 1e9) if do_dec else None
     e2e_tf_serial = job_rate(w.prefill_flops, e2e_pre_serial, ws, 1e12) if do_pre else None
     e2e_gb_serial = job_rate(w.decode_bytes, e2e_dec_serial, ws, 1e9) if do_dec else None
-    pk_t = peaks["bf16_tflops_sustained"]
+    pk_t, pk_t_src = tensor_peak(peaks, total_ms)
     pk_h = peaks["hbm_gbs"]
     line = {
         "metric": METRIC,
@@ -370,11 +460,12 @@ def run_ours(args, ws, rank, local):
             "bound": "tensor",
             "achieved": r2(per_gpu_tflops, 2),
             "peak": pk_t,
-            "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long loop)",
+            "peak_source": f"{peaks_src} {pk_t_src}",
             "unit": "TFLOP/s",
             "frac": r2(per_gpu_tflops and per_gpu_tflops / pk_t, 4),
-            "frac_of_burst_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops"], 4),
+            "frac_of_sustained_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops_sustained"], 4),
             "traffic": None if args.window else profiled_traffic("prefill", PREFILL.name),
+            "timed_region_ms": round(total_ms, 3),
             "avg_launch_ms": round(pre_avg, 5),
             "graph_avg_launch_ms": None if g_pre is None else round(g_pre, 5),
             "graph_frac": None if g_pre is None else r2(w.prefill_flops / (g_pre * 1e-3) / 1e12 / pk_t, 4),
@@ -415,10 +506,42 @@ def run_ours(args, ws, rank, local):
             "serial_how": "the same steps on one stream with a host sync after each step",
         },
         "gpu_launches": (int(do_pre) + int(do_dec)) * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": region_clocks,
     }
+    if cfg is not None:
+        line["configs"] = {}
+        for name, c in cfg.items():
+            spec = inputs.WORKLOADS[name]
+            pk, pk_src = tensor_peak(peaks, c["region_ms"])
+            tf = spec.flops() / (c["ms"] * 1e-3) / 1e12
+            gtf = None if c["graph_ms"] is None else spec.flops() / (c["graph_ms"] * 1e-3) / 1e12
+            nbytes = inputs.dense_bytes(spec)
+            line["configs"][name] = {
+                "kernel": f"prefill_fwd_kernel<{spec.D},{'bf16' if spec.dtype == torch.bfloat16 else 'f16'},"
+                          f"{'causal' if spec.causal else 'full'}>",
+                "flops": spec.flops(),
+                "bytes": nbytes,
+                "avg_launch_ms": round(c["ms"], 5),
+                "value": r2(tf, 2),
+                "unit": "TFLOP/s",
+                "bound": "tensor",
+                "peak": pk,
+                "peak_source": f"{peaks_src} {pk_src}",
+                "frac": r2(tf / pk, 4),
+                "graph_avg_launch_ms": None if c["graph_ms"] is None else round(c["graph_ms"], 5),
+                "graph_value": r2(gtf, 2),
+                "graph_frac": None if gtf is None else r2(gtf / pk, 4),
+                "graph_gbs": None if c["graph_ms"] is None else r2(nbytes / (c["graph_ms"] * 1e-3) / 1e9, 1),
+                "graph_hbm_frac": None if c["graph_ms"] is None else
+                r2(nbytes / (c["graph_ms"] * 1e-3) / 1e9 / pk_h, 4),
+                "launches": c["launches"],
+                "copies": c["copies"],
+                "clocks": c["clocks"],
+                "bar": "tensor >= 0.60 of peak (L >= 2048)" if spec.Lq >= 2048 else None,
+            }
     if pp_ms is not None:
         pp_tf = job_rate(w.prefill_flops, pp_ms, ws, 1e12) / ws
+        pk_pp, pk_pp_src = tensor_peak(peaks, pp_ms * max(3, min(300, args.steps)))
         line["paged_prefill"] = {
             "what": "attn_fwd_paged_prefill on the prefill workload with K/V scattered over a "
                     "paged cache (16-token blocks, seeded permutation), the whole sequence as "
@@ -428,8 +551,9 @@ def run_ours(args, ws, rank, local):
             "unit": "TFLOP/s",
             "bound": "tensor",
             "achieved": r2(pp_tf, 2),
-            "peak": pk_t,
-            "frac": r2(pp_tf / pk_t, 4),
+            "peak": pk_pp,
+            "peak_source": f"{peaks_src} {pk_pp_src}",
+            "frac": r2(pp_tf / pk_pp, 4),
             "vs_dense": r2(pre_avg / pp_ms, 4),
             "avg_call_ms": round(pp_ms, 5),
             "steps": max(3, min(300, args.steps)),
@@ -437,7 +561,8 @@ def run_ours(args, ws, rank, local):
         }
     if fp8_ms is not None:
         f8_tf = job_rate(w.prefill_flops, fp8_ms, ws, 1e12) / ws
-        pk_f8 = 2 * pk_t  # the fp8 tensor rate is twice the bf16 rate (nominal 4.5 vs 2.25 PFLOP/s)
+        pk_b, pk_b_src = tensor_peak(peaks, fp8_ms * max(3, min(300, args.steps)))
+        pk_f8 = 2 * pk_b  # the fp8 tensor rate is twice the bf16 rate (nominal 4.5 vs 2.25 PFLOP/s)
         line["fp8"] = {
             "what": "attn_fwd_fp8 on the prefill workload with q, k, v cast to e4m3 (bf16 output)",
             "kernel": f"prefill_fwd_kernel<{PREFILL.D},e4m3>",
@@ -446,7 +571,7 @@ def run_ours(args, ws, rank, local):
             "bound": "tensor",
             "achieved": r2(f8_tf, 2),
             "peak": pk_f8,
-            "peak_source": f"{peaks_src} bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio)",
+            "peak_source": f"{peaks_src} {pk_b_src} x 2 (nominal fp8/bf16 ratio)",
             "frac": r2(f8_tf / pk_f8, 4),
             "vs_bf16": r2(pre_avg / fp8_ms, 4),
             "avg_call_ms": round(fp8_ms, 5),
@@ -456,6 +581,7 @@ def run_ours(args, ws, rank, local):
     if bwd_ms is not None:
         bwd_flops = 2.5 * w.prefill_flops
         bwd_tf = job_rate(bwd_flops, bwd_ms, ws, 1e12) / ws
+        pk_bw, pk_bw_src = tensor_peak(peaks, bwd_ms * max(3, min(100, args.steps)))
         line["backward"] = {
             "what": "attn_bwd of the prefill workload: dQ, dK, dV from O, lse and a seeded dO",
             "kernels": "bwd_prep_kernel + bwd_kernel<dK,dV> + bwd_kernel<dQ>",
@@ -467,15 +593,73 @@ def run_ours(args, ws, rank, local):
                           "the dK/dV and the dQ kernel), so 5/7 of the peak is their ceiling",
             "bound": "tensor",
             "achieved": r2(bwd_tf, 2),
-            "peak": pk_t,
-            "frac": r2(bwd_tf / pk_t, 4),
+            "peak": pk_bw,
+            "peak_source": f"{peaks_src} {pk_bw_src}",
+            "frac": r2(bwd_tf / pk_bw, 4),
             "avg_call_ms": round(bwd_ms, 5),
             "steps": max(3, min(100, args.steps)),
             "gpu_launches": 3 * max(3, min(100, args.steps)),
         }
     if args.cpu_baseline and ws == 1:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        gpu = {"prefill": (w.p_out, w.p_lse) if do_pre and args.window is None else None,
+               "decode": (w.d_out, w.d_lse) if do_dec else None,
+               "configs": {n: (c["inputs"], c["out"], c["lse"]) for n, c in (cfg or {}).items()}}
+        line["cpu_baseline"], line["parity"] = cpu_baseline(args.cpu_seconds, gpu)
     return line
+
+
+def measure_configs(ta, device, ws, steps: int, warmup: int, clocks):
+    """The pages' smaller dense workloads (B1 H8 L512, the ViT-B/16 attention, B2 H8 L2048
+    causal; fp16, D = 64), each timed on its own: `steps` back-to-back attn_fwd calls
+    between two CUDA events, and the same calls replayed from a CUDA graph. Inputs rotate
+    over device copies that together exceed twice the L2. Returns per workload the ms per
+    launch, the graph's ms per launch, the clock record of the timed window and the
+    output of one call (for the oracle comparison)."""
+    res = {}
+    stream = torch.cuda.current_stream()
+    for name in SMALL_CONFIGS:
+        spec = inputs.WORKLOADS[name]
+        x = inputs.make(spec)
+        per = sum(t.numel() * t.element_size() for t in x.values())
+        n_copies = max(2, -(-2 * L2_BYTES // per))
+        dev = [{k: v.to(device) for k, v in x.items()} for _ in range(n_copies)]
+        out = torch.empty_like(dev[0]["q"])
+        lse = torch.empty(spec.B, spec.Hq, spec.Lq, device=device)
+
+        def call(i, st=None):
+            c = dev[i % n_copies]
+            ta.fwd(c["q"], c["k"], c["v"], causal=spec.causal, scale=spec.scale, out=out,
+                   lse=lse, stream=st)
+
+        for i in range(warmup):
+            call(i, stream)
+        torch.cuda.synchronize()
+        if ta.device_status() != 0:
+            raise RuntimeError(f"device status set by the {name} warm-up")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        torch.cuda.synchronize()
+        h0 = time.perf_counter()
+        e0.record(stream)
+        for i in range(steps):
+            call(warmup + i, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        h1 = time.perf_counter()
+        barrier(ws)
+        ms = reduce_max(e0.elapsed_time(e1) / steps, ws, device)
+        n_calls = max(2 * n_copies, 64)
+        g_ms = graph_launch_ms(lambda i: call(i), n_calls=n_calls,
+                               replays=max(1, 2000 // n_calls), ws=ws, device=device)
+        if ta.device_status() != 0:
+            raise RuntimeError(f"device status set during the {name} timing")
+        call(0, stream)
+        torch.cuda.synchronize()
+        res[name] = {"ms": ms, "graph_ms": g_ms, "region_ms": ms * steps, "launches": steps,
+                     "copies": n_copies, "clocks": clocks.summary(h0, h1), "inputs": x,
+                     "out": out, "lse": lse}
+        del dev
+    return res
 
 
 def measure_backward(w, ta, stream, device, steps: int, warmup: int, ws: int, window=None):
@@ -739,11 +923,12 @@ def measure_e2e(w, ta, stream, device, steps: int, window=None):
 _ORACLE_INPUTS: dict = {}
 
 
-def oracle_sample(seconds: float):
+def oracle_sample(seconds: float, keep: bool = False):
     """Time the fp64 oracle on a bounded sample of the same step: rows of the long
     prefill spread over heads and positions, and whole decode sequences. Returns the
-    measured TFLOP/s (prefill convention 4*D per visible key per row) and GB/s. The
-    inputs are drawn once per process."""
+    measured TFLOP/s (prefill convention 4*D per visible key per row) and GB/s; with
+    keep=True also the sampled rows and the oracle's outputs for them and for the
+    decode. The inputs are drawn once per process."""
     import oracle
     if PREFILL.name not in _ORACLE_INPUTS:
         _ORACLE_INPUTS[PREFILL.name] = (inputs.make(PREFILL), inputs.make(DECODE))
@@ -776,25 +961,73 @@ def oracle_sample(seconds: float):
     n = int(max(64, min(400000, n * (0.9 * seconds) / max(dt, 1e-4))))
     rows, keys = rows_for(n)
     t = time.perf_counter()
-    oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale, PREFILL.causal, threads)
+    ro, rl = oracle.attn_fwd_rows(xp["q"], xp["k"], xp["v"], rows, PREFILL.scale,
+                                  PREFILL.causal, threads)
     t_pre = time.perf_counter() - t
     flops = 4.0 * D * keys
     t = time.perf_counter()
-    oracle.attn_paged(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"], xd["seq_lens"],
-                      DECODE.scale, threads)
+    do, dl = oracle.attn_paged(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"],
+                               xd["seq_lens"], DECODE.scale, threads)
     t_dec = time.perf_counter() - t
     nbytes = inputs.paged_bytes(DECODE, xd["seq_lens"])
-    return {"tflops": flops / t_pre / 1e12, "gbs": nbytes / t_dec / 1e9, "rows": n,
-            "prefill_s": t_pre, "decode_s": t_dec, "threads": threads}
+    r = {"tflops": flops / t_pre / 1e12, "gbs": nbytes / t_dec / 1e9, "rows": n,
+         "prefill_s": t_pre, "decode_s": t_dec, "threads": threads}
+    if keep:
+        r["prefill_ref"] = (rows, ro, rl)
+        r["decode_ref"] = (do, dl)
+    return r
 
 
-def cpu_baseline(seconds: float):
-    r = oracle_sample(seconds)
-    return {"value": r["tflops"], "unit": "TFLOP/s", "cores": r["threads"], "kind": "oracle",
+O_TOL = {torch.float16: 2e-3, torch.bfloat16: 1.6e-2}
+LSE_REL = 1e-4
+
+
+def compare(out, lse, ro, rl, dtype, rows_note):
+    """max |O err| and max lse error (|d| / max(1, |lse|)) of a GPU result against the
+    oracle's, with the tolerances the parity tests use."""
+    o = out.detach().to("cpu", torch.float64).reshape(ro.shape)
+    err = float((o - ro).abs().max()) if ro.numel() else 0.0
+    lg = lse.detach().to("cpu", torch.float64).reshape(rl.shape)
+    fin = torch.isfinite(rl)
+    same_inf = bool(torch.equal(torch.isfinite(lg), fin))
+    lerr = float(((lg[fin] - rl[fin]).abs() / rl[fin].abs().clamp_min(1.0)).max()) if fin.any() else 0.0
+    tol = O_TOL[dtype]
+    return {"rows": rows_note, "max_abs_err": err, "tol": tol, "max_lse_rel_err": lerr,
+            "lse_tol": LSE_REL, "ok": bool(err <= tol and lerr <= LSE_REL and same_inf)}
+
+
+def cpu_baseline(seconds: float, gpu=None):
+    """The oracle timed on the host cores on a bounded sample of the step (the CPU
+    baseline). With the GPU results of the same inputs (`gpu`), the oracle's outputs for
+    that sample are also compared with them: the long prefill on the sampled rows, the
+    decode on every output, and the small dense workloads (timed in `configs`) on every
+    output."""
+    import oracle
+    r = oracle_sample(seconds, keep=gpu is not None)
+    line = {"value": r["tflops"], "unit": "TFLOP/s", "cores": r["threads"], "kind": "oracle",
             "sample": f"{r['rows']} random query rows of {PREFILL.name} (all their visible keys, "
                       f"{r['prefill_s']:.1f} s) + the whole {DECODE.name} decode "
                       f"({r['decode_s']:.2f} s, {r['gbs']:.3f} GB/s)",
             "paged_decode_gbs": r["gbs"]}
+    if gpu is None:
+        return line, None
+    par = {}
+    if gpu.get("prefill") is not None:
+        rows, ro, rl = r["prefill_ref"]
+        out, lse = gpu["prefill"]
+        idx = torch.tensor(rows)
+        par[PREFILL.name] = compare(out.reshape(-1, PREFILL.D)[idx.to(out.device)],
+                                    lse.reshape(-1)[idx.to(lse.device)], ro, rl, PREFILL.dtype,
+                                    f"{len(rows)} sampled rows (the CPU-baseline sample)")
+    if gpu.get("decode") is not None:
+        do, dl = r["decode_ref"]
+        out, lse = gpu["decode"]
+        par[DECODE.name] = compare(out, lse, do, dl, DECODE.dtype, "every output")
+    for name, (x, out, lse) in gpu.get("configs", {}).items():
+        spec = inputs.WORKLOADS[name]
+        ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], spec.scale, spec.causal)
+        par[name] = compare(out, lse, ro, rl, spec.dtype, "every output")
+    return line, par
 
 
 def run_reference(args, ws, rank):
@@ -854,6 +1087,8 @@ def main(argv=None):
                     help="skip the separately timed e4m3 forward of the prefill workload")
     ap.add_argument("--no-paged-prefill", dest="paged_prefill", action="store_false",
                     help="skip the separately timed paged-cache prefill of the prefill workload")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the separately timed small dense workloads (C1-C3 shapes)")
     ap.add_argument("--no-backward", dest="backward", action="store_false",
                     help="skip the separately timed backward pass of the prefill workload")
     ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",

@@ -218,8 +218,12 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
  *
  * The first call on a device looks up the array's device address with that
  * device current (cudaGetSymbolAddress); make that first call before any
- * stream capture. Each call clears the array's completion counters on `stream`
- * before the kernel.
+ * stream capture. The address is looked up again when the device's current
+ * context changes (after a device reset the library's module, and the array
+ * with it, is loaded anew); the first call after such a reset is then again a
+ * set-up call. Every argument check and the tensor-map encoding run before
+ * anything is enqueued; then each call clears the array's completion counters
+ * on `stream` and launches the kernel.
  *
  * Every call on a device shares the one array, which keeps the last call's
  * contents: calls that overlap on the GPU (different streams, or different

@@ -19,7 +19,6 @@ from __future__ import annotations
 
 import math
 
-import numpy as np
 import pytest
 import torch
 
@@ -109,10 +108,10 @@ def test_backward_empty_sides():
     assert ta.device_status() == 0
 
 
-def test_backward_long_causal_prefill_sampled():
-    """The long causal prefill workload (B1 H16 L8192 D128 bf16) end to end on the GPU;
-    the oracle checks dQ on sampled rows of every head and dK, dV on sampled keys of one
-    head (it recomputes that head's row statistics)."""
+def test_backward_long_causal_prefill_all():
+    """The long causal prefill workload (B1 H16 L8192 D128 bf16) end to end on the GPU:
+    every element of dQ, dK and dV against the oracle's full backward pass (about a
+    minute of host time on 16 cores), under the per-element bound."""
     s = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
     x = inputs.make(s)
     do = inputs.dense_grad_output(s)
@@ -121,18 +120,6 @@ def test_backward_long_causal_prefill_sampled():
     dq, dk, dv = ta.bwd(q, k, v, out, do.to(DEV), lse, causal=True, scale=s.scale)
     torch.cuda.synchronize()
     assert ta.device_status() == 0
-    L, H, D = s.Lq, s.Hq, s.D
-    rng = np.random.default_rng(7)
-    rows = np.concatenate([[0, 63, 64, 127, 128, L - 1], rng.integers(0, L, 42)])
-    heads = rng.integers(0, H, rows.shape[0])
-    ids = heads * L + rows
-    ref_dq, m_dq = oracle.attn_bwd_dq_rows(x["q"], x["k"], x["v"], do, ids, s.scale, True,
-                                           sensitivity=True)
-    check_grad(dq.reshape(-1, D)[torch.as_tensor(ids)].cpu(), ref_dq, m_dq, s.dtype, "dq rows")
-    h = 5
-    keys = np.concatenate([[0, 1, 127, 128, 4095, L - 1], rng.integers(0, L, 26)])
-    kid = h * L + keys
-    ref_dk, ref_dv, m_dk, m_dv = oracle.attn_bwd_dkv_keys(x["q"], x["k"], x["v"], do, kid,
-                                                          s.scale, True, sensitivity=True)
-    check_grad(dk.reshape(-1, D)[torch.as_tensor(kid)].cpu(), ref_dk, m_dk, s.dtype, "dk keys")
-    check_grad(dv.reshape(-1, D)[torch.as_tensor(kid)].cpu(), ref_dv, m_dv, s.dtype, "dv keys")
+    ref = oracle.attn_bwd(x["q"], x["k"], x["v"], do, s.scale, True, sensitivity=True)
+    for i, (name, got) in enumerate((("dq", dq), ("dk", dk), ("dv", dv))):
+        check_grad(got.cpu(), ref[i], ref[3 + i], s.dtype, f"long causal prefill {name}, all")

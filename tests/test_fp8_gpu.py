@@ -98,24 +98,14 @@ def test_fp8_blhd_layout_matches_contiguous():
     assert torch.equal(ob.transpose(1, 2), ref) and torch.equal(lse, ref_lse)
 
 
-def test_fp8_long_causal_prefill_sampled():
-    """The long causal prefill shape (B1 H16 L8192 D128) with e4m3 inputs: sampled rows
-    against the oracle, under the same bound."""
+def test_fp8_long_causal_prefill_all_rows():
+    """The long causal prefill shape (B1 H16 L8192 D128) with e4m3 inputs: every row
+    against the oracle on the exact e4m3 values, under the same element bound, plus the
+    per-head relative Frobenius bound."""
     s = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
     x = inputs.make(s)
     q, k, v = (x[n].to(torch.float32).to(torch.float8_e4m3fn) for n in ("q", "k", "v"))
     out, lse = ta.fwd_fp8(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=s.scale)
     torch.cuda.synchronize()
     assert ta.device_status() == 0
-    g = torch.Generator().manual_seed(11)
-    rows = torch.randint(0, s.Hq * s.Lq, (256,), generator=g)
-    rows[:3] = torch.tensor([0, s.Lq - 1, 5 * s.Lq + 4095])
-    q64, k64, v64 = (t.to(torch.float64) for t in (q, k, v))
-    ro, rl = oracle.attn_fwd_rows(q64, k64, v64, rows, s.scale, True)
-    m, _ = oracle.attn_fwd_rows(q64, k64, v64.abs(), rows, s.scale, True)
-    o = out.reshape(-1, 128)[rows.to(DEV)].cpu().to(torch.float64)
-    err = (o - ro).abs()
-    bound = 2 * U8 * m + 2.0 ** -8 * ro.abs() + 2.0 ** -7
-    assert bool((err <= bound).all()), float((err / bound).max())
-    lg = lse.reshape(-1)[rows.to(DEV)].cpu().to(torch.float64)
-    assert float(((lg - rl).abs() / rl.abs().clamp_min(1.0)).max()) <= 1e-4
+    check_fp8(out, lse, q, k, v, s.scale, True, (1.0, 1.0, 1.0), "long causal prefill, all rows")

@@ -3,8 +3,9 @@
 Every call goes through the C ABI (ctypes) of the in-tree library. Inputs are the
 seeded generators' tensors; the oracle sees the identical f16/bf16 values widened to
 fp64. Small shapes are compared element by element over every output; the full-size
-workloads are run in the benchmark's launch configuration and compared on all outputs
-(when the oracle finishes in seconds) or on sampled rows (long prefill).
+workloads are run in the benchmark's launch configuration and compared on all outputs;
+only the longest sequences the library accepts (2^22 keys or queries) are compared on
+sampled rows.
 """
 from __future__ import annotations
 
@@ -137,27 +138,18 @@ def test_full_workload_all_outputs(name):
     check_parity(out, lse, ro, rl, s.dtype, name)
 
 
-def test_long_prefill_sampled_rows():
+def test_long_prefill_all_rows():
+    """The long causal prefill workload (B1 H16 L8192 D128 bf16) in the benchmark's launch
+    configuration, compared with the oracle on every one of its 131,072 rows: every
+    element of O and every lse (the oracle takes about 15 s of host time on 16 cores)."""
     s = inputs.WORKLOADS["prefill_causal_b1_h16_l8192_d128_bf16"]
     x = inputs.make(s)
     out, lse = run(x["q"], x["k"], x["v"], s.causal, s.scale)
-    g = torch.Generator().manual_seed(123)
-    L = s.Lq
-    rows = []
-    for h in range(s.Hq):
-        # the first rows (few keys, largest outputs), tile edges, the last rows, and a
-        # random sample in between
-        picks = list(range(0, 8)) + [127, 128, 129, 4095, 4096, L - 2, L - 1]
-        picks += torch.randint(0, L, (40,), generator=g).tolist()
-        rows += [h * L + i for i in picks]
-    ro, rl = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, s.scale, s.causal)
-    rows_t = torch.tensor(rows)
-    check_parity(out.reshape(-1, s.D)[rows_t], lse.reshape(-1)[rows_t], ro, rl, s.dtype,
-                 "long prefill sampled rows")
-    # properties that hold at any size: every output and every lse is finite (each row
-    # sees at least key 0), and |O| never exceeds the largest |V| entry (O is a convex
-    # combination of value rows)
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], s.scale, s.causal)
+    mx = check_parity(out, lse, ro, rl, s.dtype, "long prefill, all rows")
+    print(f"long prefill: max |O err| {mx:.3e} over {ro.numel()} elements")
+    # |O| never exceeds the largest |V| entry of its head (a convex combination of
+    # value rows), up to the output rounding
     vmax = x["v"].float().abs().amax(dim=(2, 3)).view(1, s.Hq, 1, 1)
     assert torch.all(out.float().abs() <= vmax * (1 + 2 ** -7) + 1e-6)
 

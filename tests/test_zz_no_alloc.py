@@ -4,7 +4,7 @@ Such a caller (for example a plugin handed only its input and output buffers by 
 framework that owns the allocator) cannot provide the split-KV workspace that
 attn_fwd_paged takes. The no-allocation entry point uses a fixed 4 MiB scratch array
 inside the library instead. These tests call it through the C ABI and check that two
-calls in a row give the same results as attn_fwd_paged with a caller workspace, within
+calls in a row match the fp64 oracle and attn_fwd_paged with a caller workspace, within
 the parity tolerances, and that a problem too large for the fixed array is refused.
 
 This file is collected last on purpose; it must pass both on its own in a fresh
@@ -17,9 +17,10 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import tiled_attention_19_b200 as ta
 from tiled_attention_19_b200 import inputs
-from tests.parity import LSE_REL, O_TOL
+from tests.parity import LSE_REL, O_TOL, check_parity
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -46,7 +47,10 @@ def test_noalloc_matches_workspace_entry_point(name):
         s = inputs.WORKLOADS[name]
     need = ta.paged_workspace_size(s.num_seqs, s.Hq, s.Hkv, s.D, s.max_blocks)
     assert 0 < need <= SCRATCH_LIMIT
-    x = {k: v.to(DEV) for k, v in inputs.make(s).items()}
+    xh = inputs.make(s)
+    x = {k: v.to(DEV) for k, v in xh.items()}
+    oro, orl = oracle.attn_paged(xh["q"], xh["k_cache"], xh["v_cache"], xh["block_table"],
+                                 xh["seq_lens"], s.scale)
     ref_out, ref_lse = ta.fwd_paged(x["q"], x["k_cache"], x["v_cache"], x["block_table"],
                                     x["seq_lens"], scale=s.scale)
     for _ in range(2):  # two calls in a row share (and must leave clean) the scratch
@@ -55,6 +59,7 @@ def test_noalloc_matches_workspace_entry_point(name):
         assert call_noalloc(x, s, out, lse) == 0
         torch.cuda.synchronize()
         assert ta.device_status() == 0
+        check_parity(out, lse, oro, orl, s.dtype, f"{name} no-alloc vs oracle")
         err = (out.double() - ref_out.double()).abs().max().item()
         assert err <= O_TOL[s.dtype], err
         fin = torch.isfinite(ref_lse)

@@ -632,6 +632,133 @@ attn_status_t paged_prefill(const void* q, const attn_strides_t* q_st, const voi
                   : launch_prefill<128, false, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
 }
 
+// Tensor maps of paged caches, cached by what they encode (base address, rows, D,
+// dtype, device): a map holds nothing else, so a cached map is exact even if the
+// memory behind an address was freed and reallocated with the same extent.
+struct CacheMapKey {
+    const void* base;
+    long long rows;
+    int D, bf16, dev;
+    bool operator==(const CacheMapKey& o) const {
+        return base == o.base && rows == o.rows && D == o.D && bf16 == o.bf16 && dev == o.dev;
+    }
+};
+
+bool cached_cache_map(CUtensorMap* tm, const void* base, bool bf16, int D, long long rows) {
+    constexpr int kSlots = 16;
+    static std::mutex mu;
+    static CacheMapKey keys[kSlots];
+    alignas(64) static CUtensorMap maps[kSlots];
+    static int used = 0, next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    const CacheMapKey key{base, rows, D, bf16 ? 1 : 0, dev};
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (keys[i] == key) {
+            *tm = maps[i];
+            return true;
+        }
+    if (!encode_cache_map(tm, base, bf16, D, rows)) return false;
+    const int slot = used < kSlots ? used++ : (next++ % kSlots);
+    keys[slot] = key;
+    maps[slot] = *tm;
+    return true;
+}
+
+// A paged-decode call: paged_prepare checks the arguments and fills in the kernel's
+// arguments, paged_encode checks the device and encodes the cache tensor maps, and
+// paged_launch enqueues the kernel. Nothing is enqueued before paged_launch.
+struct PagedCall {
+    bool empty = false;  // num_seqs == 0: nothing to launch
+    int D = 0;
+    bool bf16 = false;
+    attn::PagedLayout L{};
+    const void* k_cache = nullptr;
+    const void* v_cache = nullptr;
+    long long rows = 1;  // cache rows the tensor maps span
+    alignas(64) CUtensorMap tk, tv;
+    PagedArgs a{};
+};
+
+attn_status_t paged_prepare(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_table, const int32_t* seq_lens, int block_size,
+                            void* out, float* lse, int num_seqs, int H_q, int H_kv, int D,
+                            int max_blocks_per_seq, int num_blocks, float scale,
+                            attn_dtype_t dtype, PagedCall* c) {
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return ATTN_ERR_INVALID;
+    if (num_seqs == 0) {  // nothing to compute; pointers may be NULL
+        c->empty = true;
+        return ATTN_OK;
+    }
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
+        seq_lens == nullptr || out == nullptr)
+        return ATTN_ERR_INVALID;
+    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (H_q / H_kv > attn::kMaxGroup) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long long>(max_blocks_per_seq) * attn::kPageSize > kMaxSeq || num_seqs > 65535 ||
+        H_kv > 65535)
+        return ATTN_ERR_UNSUPPORTED;
+    const long long rows = static_cast<long long>(num_blocks) * H_kv * attn::kPageSize;
+    if (rows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
+        return ATTN_ERR_MISALIGNED;
+    c->D = D;
+    c->bf16 = dtype == ATTN_BF16;
+    c->L = attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq);
+    c->k_cache = k_cache;
+    c->v_cache = v_cache;
+    c->rows = rows > 0 ? rows : 1;
+    PagedArgs& a = c->a;
+    a.q = static_cast<const uint16_t*>(q);
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.out = static_cast<uint16_t*>(out);
+    a.lse = lse;
+    a.num_seqs = num_seqs;
+    a.Hq = H_q;
+    a.Hkv = H_kv;
+    a.G = H_q / H_kv;
+    a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.balanced = c->L.balanced;
+    a.scale_log2 = scale * attn::kLog2e;
+    return ATTN_OK;
+}
+
+attn_status_t paged_encode(PagedCall& c) {
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    if (!cached_cache_map(&c.tk, c.k_cache, c.bf16, c.D, c.rows) ||
+        !cached_cache_map(&c.tv, c.v_cache, c.bf16, c.D, c.rows))
+        return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+// Launches a prepared, encoded call with its split-KV scratch at `workspace` (unused
+// when the layout needs none).
+attn_status_t paged_launch(PagedCall& c, void* workspace, cudaStream_t stream) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const attn::PagedLayout& L = c.L;
+    c.a.ws_count = L.total ? reinterpret_cast<int*>(ws + L.count_off) : nullptr;
+    c.a.ws_lse = L.total ? reinterpret_cast<float*>(ws + L.lse_off) : nullptr;
+    c.a.ws_o = L.total ? reinterpret_cast<float*>(ws + L.o_off) : nullptr;
+    if (c.D == 64)
+        return c.bf16 ? launch_paged<64, true>(c.tk, c.tv, c.a, L.grid, stream)
+                      : launch_paged<64, false>(c.tk, c.tv, c.a, L.grid, stream);
+    return c.bf16 ? launch_paged<128, true>(c.tk, c.tv, c.a, L.grid, stream)
+                  : launch_paged<128, false>(c.tk, c.tv, c.a, L.grid, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -746,62 +873,17 @@ attn_status_t attn_fwd_paged(const void* q, const void* k_cache, const void* v_c
                              int max_blocks_per_seq, int num_blocks, float scale,
                              attn_dtype_t dtype, void* workspace, size_t workspace_bytes,
                              void* stream_) {
-    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
-        return ATTN_ERR_INVALID;
-    if (num_seqs == 0) return ATTN_OK;  // nothing to compute; pointers may be NULL
-    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
-        seq_lens == nullptr || out == nullptr)
-        return ATTN_ERR_INVALID;
-    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
-    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
-    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
-    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-    if (H_q / H_kv > attn::kMaxGroup) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<long long>(max_blocks_per_seq) * attn::kPageSize > kMaxSeq || num_seqs > 65535 ||
-        H_kv > 65535)
-        return ATTN_ERR_UNSUPPORTED;
-    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
-        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
-        return ATTN_ERR_MISALIGNED;
-    const attn::PagedLayout L = attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq);
-    if (L.total > 0 && (workspace == nullptr || workspace_bytes < L.total)) return ATTN_ERR_WORKSPACE;
+    PagedCall c;
+    const attn_status_t st =
+        paged_prepare(q, k_cache, v_cache, block_table, seq_lens, block_size, out, lse, num_seqs,
+                      H_q, H_kv, D, max_blocks_per_seq, num_blocks, scale, dtype, &c);
+    if (st != ATTN_OK || c.empty) return st;
+    if (c.L.total > 0 && (workspace == nullptr || workspace_bytes < c.L.total))
+        return ATTN_ERR_WORKSPACE;
     if (workspace != nullptr && !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
-    const attn_status_t dev = check_device();
-    if (dev != ATTN_OK) return dev;
-
-    const long long rows = static_cast<long long>(num_blocks) * H_kv * attn::kPageSize;
-    if (rows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    const bool bf16 = dtype == ATTN_BF16;
-    alignas(64) CUtensorMap tk, tv;
-    if (!encode_cache_map(&tk, k_cache, bf16, D, rows > 0 ? rows : 1) ||
-        !encode_cache_map(&tv, v_cache, bf16, D, rows > 0 ? rows : 1))
-        return ATTN_ERR_CUDA;
-
-    PagedArgs a{};
-    a.q = static_cast<const uint16_t*>(q);
-    a.block_table = block_table;
-    a.seq_lens = seq_lens;
-    a.out = static_cast<uint16_t*>(out);
-    a.lse = lse;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    a.ws_count = L.total ? reinterpret_cast<int*>(ws + L.count_off) : nullptr;
-    a.ws_lse = L.total ? reinterpret_cast<float*>(ws + L.lse_off) : nullptr;
-    a.ws_o = L.total ? reinterpret_cast<float*>(ws + L.o_off) : nullptr;
-    a.num_seqs = num_seqs;
-    a.Hq = H_q;
-    a.Hkv = H_kv;
-    a.G = H_q / H_kv;
-    a.max_blocks = max_blocks_per_seq;
-    a.num_blocks = num_blocks;
-    a.balanced = L.balanced;
-    a.scale_log2 = scale * attn::kLog2e;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    if (D == 64)
-        return bf16 ? launch_paged<64, true>(tk, tv, a, L.grid, stream)
-                    : launch_paged<64, false>(tk, tv, a, L.grid, stream);
-    return bf16 ? launch_paged<128, true>(tk, tv, a, L.grid, stream)
-                : launch_paged<128, false>(tk, tv, a, L.grid, stream);
+    const attn_status_t enc = paged_encode(c);
+    if (enc != ATTN_OK) return enc;
+    return paged_launch(c, workspace, static_cast<cudaStream_t>(stream_));
 }
 
 // ------------------------------------------------------------ failure detection
@@ -839,8 +921,29 @@ namespace {
 constexpr size_t kStaticScratchBytes = static_cast<size_t>(4) << 20;
 static __device__ __align__(256) uint8_t g_paged_scratch[kStaticScratchBytes];
 
-// Device address of g_paged_scratch on the current device; looked up on the first
-// call made with that device current (nullptr if the lookup fails).
+// The calling thread's current CUDA context (nullptr if none or if the driver entry
+// point is unavailable).
+CUcontext current_context() {
+    using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        cudaGetLastError();
+    });
+    CUcontext ctx = nullptr;
+    if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
+
+// Device address of g_paged_scratch in the current device's context. It is looked up
+// (cudaGetSymbolAddress) by the first call made with that device current, and again
+// whenever the device's current context differs from the one it was looked up in
+// (after a device reset the module is loaded anew, at a new address).
 void* static_scratch_address() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -849,14 +952,17 @@ void* static_scratch_address() {
     }
     static std::mutex mu;
     static void* addr[64] = {nullptr};
+    static CUcontext ctx_of[64] = {nullptr};
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+    const CUcontext ctx = current_context();
+    if (addr[dev] == nullptr || ctx == nullptr || ctx != ctx_of[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_paged_scratch) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
         addr[dev] = p;
+        ctx_of[dev] = current_context();  // the lookup made the device's context current
     }
     return addr[dev];
 }
@@ -869,46 +975,32 @@ attn_status_t attn_fwd_paged_noalloc(const void* q, const void* k_cache, const v
                                      int H_q, int H_kv, int D, int max_blocks_per_seq,
                                      int num_blocks, float scale, attn_dtype_t dtype,
                                      void* stream_) {
-    // Same argument checks as attn_fwd_paged, done here first so that nothing is
-    // enqueued (not even the counter clear) when the call is rejected.
-    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || max_blocks_per_seq < 0 || num_blocks < 0)
-        return ATTN_ERR_INVALID;
-    if (num_seqs == 0) return ATTN_OK;
-    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
-        seq_lens == nullptr || out == nullptr)
-        return ATTN_ERR_INVALID;
-    if (H_q % H_kv != 0) return ATTN_ERR_INVALID;
-    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
-    if (block_size != attn::kPageSize) return ATTN_ERR_UNSUPPORTED;
-    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-    if (H_q / H_kv > attn::kMaxGroup) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<long long>(max_blocks_per_seq) * attn::kPageSize > kMaxSeq || num_seqs > 65535 ||
-        H_kv > 65535)
-        return ATTN_ERR_UNSUPPORTED;
-    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
-        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
-        return ATTN_ERR_MISALIGNED;
-    const attn::PagedLayout L = attn::paged_layout(num_seqs, H_q, H_kv, D, max_blocks_per_seq);
-    if (L.total > kStaticScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
-    const attn_status_t dev = check_device();
-    if (dev != ATTN_OK) return dev;
-    void* scratch = static_scratch_address();
-    if (scratch == nullptr) return ATTN_ERR_CUDA;
+    // Every check and the tensor-map encoding run first, so that a rejected call
+    // enqueues nothing (not even the counter clear).
+    PagedCall c;
+    const attn_status_t st =
+        paged_prepare(q, k_cache, v_cache, block_table, seq_lens, block_size, out, lse, num_seqs,
+                      H_q, H_kv, D, max_blocks_per_seq, num_blocks, scale, dtype, &c);
+    if (st != ATTN_OK || c.empty) return st;
+    if (c.L.total > kStaticScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+    const attn_status_t enc = paged_encode(c);
+    if (enc != ATTN_OK) return enc;
+    void* scratch = nullptr;
+    if (c.L.total > 0) {
+        scratch = static_scratch_address();
+        if (scratch == nullptr) return ATTN_ERR_CUDA;
+    }
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    if (L.total > 0) {
+    if (c.L.total > 0) {
         // The completion counters must start at zero; the partial results need not.
         const size_t counters = static_cast<size_t>(num_seqs) * H_kv * sizeof(int);
-        if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + L.count_off, 0, counters, stream) !=
+        if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + c.L.count_off, 0, counters, stream) !=
             cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_CUDA;
         }
     }
-    return attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, block_size, out, lse,
-                          num_seqs, H_q, H_kv, D, max_blocks_per_seq, num_blocks, scale, dtype,
-                          L.total > 0 ? scratch : nullptr, L.total > 0 ? kStaticScratchBytes : 0,
-                          stream_);
+    return paged_launch(c, scratch, stream);
 }
 
 const char* attn_error_string(attn_status_t status) {
