@@ -27,9 +27,9 @@
 //              was issued, and the commit that signals S0_j also covers PV0_{j-1}: the
 //              softmax may rescale O0 as soon as S0_j is ready.
 //   warps 10-11 idle.
-// Registers: the third warpgroup releases registers (setmaxnreg.dec to 80) and the two
-// softmax warpgroups take them (setmaxnreg.inc to 200): 2x128x200 + 128x80 = 61,440 of
-// the 384 x 168 = 64,512 the CTA is launched with.
+// Registers: the third warpgroup releases registers (setmaxnreg.dec to 72) and the two
+// softmax warpgroups take them (setmaxnreg.inc to 216): 2x128x216 + 128x72 = 64,512, all
+// of the 384 x 168 the CTA is launched with.
 // TMEM (512 columns): S0/P0 at 0, S1/P1 at 128, O0 at 256, O1 at 384.
 //
 // Band masks (the "Flash Attention" skill page, Scenario 2: causal=True for
@@ -59,9 +59,12 @@ constexpr int kPrefillThreads = 384;
 // CTA was launched with cover it; the launcher checks 384 x (registers per thread at
 // launch) >= kRegBudget before the first launch and refuses otherwise, because a
 // setmaxnreg.inc that cannot be satisfied waits forever.
-constexpr int kSoftmaxRegs = 200;
-constexpr int kOtherRegs = 80;
-constexpr int kRegBudget = 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs;  // 61,440
+// ptxas allocates each region for the count its setmaxnreg sets, so these are also the
+// registers the softmax and the other roles are compiled for (216 leaves the softmax
+// without spills; the producer and MMA roles fit in 72).
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
+constexpr int kRegBudget = 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs;  // 64,512
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D, bool FP8 = false>
@@ -79,9 +82,16 @@ struct PrefillCfg {
     static constexpr int kVStages = (kTileBytes == 16384) ? 5 : 2;
     static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 384;
     static constexpr int kTmemCols = 512;
+    // P is handed to the MMA warp in two parts: the first kPSplit keys, then the rest
+    // (kPSplit is a multiple of kPVKeys, so each part is whole P.V instructions).
+    // One pair of exponentials in kPolyEvery is computed on the FMA pipe instead of the
+    // MUFU (0: none).
+    static constexpr int kPolyEvery = 0;
+    static constexpr int kPSplit = 96;  // the softmax's stores below are laid out for 96
+    static_assert(kPSplit == 96 && kBN == 128, "P hand-off layout");
     // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
-    // S_FULL[2], P_FULL[2], O_DONE[2], DRAIN
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 7;
+    // S_FULL[2], P_FULL[2] (first part of P), P_REST[2] (the rest), O_DONE[2], DRAIN
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 9;
     static constexpr int kTileRegion = kTileBytes * (2 + kKStages + kVStages);
     static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTileRegion + kNumBars * 8 + 16;
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
@@ -92,7 +102,9 @@ struct PrefillArgs {
     long long out_sb, out_sh, out_sl;  // element strides of out over (batch, head, row)
     float* lse;
     int Hq, Hkv, group, Lq, Lk;
-    int n_q_blocks;    // ceil(Lq / 256): CTAs along the query axis
+    int n_q_blocks;    // CTAs along the query axis: ceil(Lq / 256), or ceil(ceil(Lq / 128) / 2) paired
+    int paired;        // causal only: CTA y takes query tiles y and T - 1 - y (T = ceil(Lq / 128)),
+                       // so every CTA walks about the same number of key tiles
     int win_left;      // band: keys >= i' - win_left visible (-1: unbounded)
     int win_right;     // band: keys <= i' + win_right visible (-1: unbounded; causal: 0)
     float scale_log2;  // scale * log2(e) (8-bit inputs: times the q and k descale factors)
@@ -165,8 +177,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     constexpr int V_FULL = K_EMPTY + NK;
     constexpr int V_EMPTY = V_FULL + NV;
     constexpr int S_FULL = V_EMPTY + NV;  // [2]
-    constexpr int P_FULL = S_FULL + 2;    // [2]
-    constexpr int O_DONE = P_FULL + 2;    // [2]
+    constexpr int P_FULL = S_FULL + 2;    // [2] the first kPSplit keys of P are in TMEM
+    constexpr int P_REST = P_FULL + 2;    // [2] the rest of P is in TMEM
+    constexpr int O_DONE = P_REST + 2;    // [2]
     constexpr int DRAIN = O_DONE + 2;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
 
@@ -187,11 +200,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int bh = blockIdx.x;                           // b * Hq + h
-    const int qb = args.n_q_blocks - 1 - blockIdx.y;     // longest causal blocks first
     const int h = bh % args.Hq;
     const int b = bh / args.Hq;
     const int hkv = h / args.group;  // grouped-query head mapping
-    const int q0 = qb * 2 * kBM;
+    // First rows of the CTA's two query tiles. Normally two consecutive tiles, the
+    // CTAs with the most key tiles first. Paired (causal grids of at most one wave): a
+    // short tile and a long one, the long one as Q1; the middle tile of an odd count
+    // runs alone as Q1 (Q0 then computes and writes nothing).
+    int qrow0, qrow1;
+    bool has_q0 = true;
+    if (MASK == kMaskCausal && !PAGED && args.paired) {
+        const int T = (args.Lq + kBM - 1) / kBM;
+        qrow0 = blockIdx.y * kBM;
+        qrow1 = (T - 1 - static_cast<int>(blockIdx.y)) * kBM;
+        has_q0 = qrow0 != qrow1;
+    } else {
+        const int qb = args.n_q_blocks - 1 - blockIdx.y;  // longest causal blocks first
+        qrow0 = qb * 2 * kBM;
+        qrow1 = qrow0 + kBM;
+    }
     // The lengths the masks see: the problem's, or with paged keys the sequence's own
     // (seq_lens[b] keys, q_lens[b] queries at its last positions). Out-of-range values
     // are clamped and reported.
@@ -212,14 +239,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // the band edges are monotone in the row)
     int a0 = 0, b0, a1 = 0, b1;
     if constexpr (MASK == kMaskWindow) {
-        key_tiles_for<MASK>(q0, a, a0, b0);
-        key_tiles_for<MASK>(q0 + kBM, a, a1, b1);
+        key_tiles_for<MASK>(qrow0, a, a0, b0);
+        key_tiles_for<MASK>(qrow1, a, a1, b1);
     } else {  // every query tile starts at key tile 0
         int unused;
-        key_tiles_for<MASK>(q0, a, unused, b0);
-        key_tiles_for<MASK>(q0 + kBM, a, unused, b1);
+        key_tiles_for<MASK>(qrow0, a, unused, b0);
+        key_tiles_for<MASK>(qrow1, a, unused, b1);
     }
-    if (PAGED && q0 >= a.Lq) a0 = b0 = a1 = b1 = 0;  // every row past the sequence's chunk
+    if (!has_q0) a0 = b0 = 0;
+    if (PAGED && qrow0 >= a.Lq) a0 = b0 = a1 = b1 = 0;  // every row past the sequence's chunk
     const int jlo = (MASK != kMaskWindow) ? 0 : ((b0 > a0) ? a0 : a1);
     const int jhi = max(b0, b1);
     const int n_all = (b1 > a1 || b0 > a0) ? jhi - jlo : 0;  // key tiles this CTA loads
@@ -237,6 +265,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(S_FULL + t), 1);
             mbar_init(bar(P_FULL + t), kBM);
+            mbar_init(bar(P_REST + t), kBM);
             mbar_init(bar(O_DONE + t), 1);
         }
         mbar_init(bar(DRAIN), 1);
@@ -269,8 +298,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
-                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, q0, h, b);
-                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, q0 + kBM,
+                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow0,
+                            h, b);
+                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow1,
                             h, b);
             }
             constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
@@ -335,118 +365,142 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             constexpr uint32_t kIdescQK = idesc_f16(BF16 && !FP8, kBM, kBN, false, false);
             constexpr uint32_t kIdescPV = idesc_f16(BF16 && !FP8, kBM, D, false, true);
             mma_started = true;
-            // S_t = Q_t K_j^T into TMEM columns s_col (K-major operands: 16 elements =
-            // 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
-            auto issue_s = [&](uint32_t sQ, uint32_t s_col, int n) {
-                const uint32_t sK = sK0 + (n % NK) * Cfg::kTileBytes;
+            // The issue of a tcgen05.mma blocks while the tensor core's queue is full, so
+            // this thread's own work between products is tensor-core idle time: the shared
+            // memory descriptors are built once and offset per product (the start address
+            // is the descriptor's low field, in 16-byte units, and never carries out of it).
+            const uint64_t dq0 = sdesc_sw128(sQ0, 16, 1024), dq1 = sdesc_sw128(sQ1, 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(sK0, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sV0, Cfg::kChunkBytes, 1024);
+            constexpr uint32_t kTileUnits = Cfg::kTileBytes >> 4;
+            // S_t = Q_t K^T into TMEM columns s_col, K from ring stage sk (K-major operands:
+            // 16 elements = 32 bytes per step inside a 128-byte swizzle row, then the next
+            // chunk).
+            auto issue_s = [&](uint64_t dq, uint32_t s_col, int sk) {
+                const uint64_t dk = dk0 + static_cast<uint32_t>(sk) * kTileUnits;
 #pragma unroll
                 for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
+                    constexpr uint32_t kChunkUnits = Cfg::kChunkBytes >> 4;
+                    const uint32_t off = (kk >> 2) * kChunkUnits + (kk & 3) * 2;
                     if constexpr (FP8)
-                        mma_ss_f8(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
-                                  sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                        mma_ss_f8(tmem + s_col, dq + off, dk + off, kIdescQK, kk > 0 ? 1u : 0u);
                     else
-                        mma_ss(tmem + s_col, sdesc_sw128(sQ + koff, 16, 1024),
-                               sdesc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + s_col, dq + off, dk + off, kIdescQK, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_t += P_t V_j: P from TMEM (kPVKeys keys = 8 columns per step), V MN-major
-            // (kPVKeys keys = 8-row swizzle atoms of 128 bytes, kPVKeys * 128 bytes per step;
-            // D chunks 16 KiB apart). `first` starts the accumulator (the query tile's first
+            // O_t += P_t V: P from TMEM (kPVKeys keys = 8 columns per step), V from ring
+            // stage sv, MN-major (kPVKeys keys = 8-row swizzle atoms of 128 bytes,
+            // kPVKeys * 128 bytes per step; D chunks 16 KiB apart). Keys [k0, k1) of the tile
+            // (whole instructions); `first` starts the accumulator (the query tile's first
             // key tile).
-            auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int n, bool first) {
-                const uint32_t sV = sV0 + (n % NV) * Cfg::kTileBytes;
+            auto issue_pv = [&](uint32_t p_col, uint32_t o_col, int sv, bool first, int k0, int k1) {
+                const uint64_t dv = dv0 + static_cast<uint32_t>(sv) * kTileUnits;
 #pragma unroll
-                for (int ks = 0; ks < kBN / Cfg::kPVKeys; ++ks) {
-                    const uint64_t bd = sdesc_sw128(sV + ks * Cfg::kPVKeys * 128, Cfg::kChunkBytes, 1024);
+                for (int ks = k0 / Cfg::kPVKeys; ks < k1 / Cfg::kPVKeys; ++ks) {
+                    const uint32_t off = ks * Cfg::kPVKeys * 8;  // kPVKeys * 128 bytes
                     if constexpr (FP8)
-                        mma_ts_f8(tmem + o_col, tmem + p_col + ks * 8, bd, kIdescPV,
+                        mma_ts_f8(tmem + o_col, tmem + p_col + ks * 8, dv + off, kIdescPV,
                                   (!first || ks > 0) ? 1u : 0u);
                     else
-                        mma_ts(tmem + o_col, tmem + p_col + ks * 8, bd, kIdescPV,
+                        mma_ts(tmem + o_col, tmem + p_col + ks * 8, dv + off, kIdescPV,
                                (!first || ks > 0) ? 1u : 0u);
                 }
             };
+            // O_t += P_t V: the first part of P as soon as it is in TMEM, then the rest.
+            // V is already known to be in stage sv. Returns false if a wait gave up.
+            auto pv_parts = [&](int t, uint32_t p_col, uint32_t o_col, int sv, bool first,
+                                uint32_t parity) -> bool {
+                if (!wait_phase(bar(P_FULL + t), parity, abort_flag)) return false;
+                tc_fence_after();
+                issue_pv(p_col, o_col, sv, first, 0, Cfg::kPSplit);
+                if (!wait_phase(bar(P_REST + t), parity, abort_flag)) return false;
+                tc_fence_after();
+                issue_pv(p_col, o_col, sv, first, Cfg::kPSplit, kBN);
+                return true;
+            };
             bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
+            // ring positions: K of the tile whose S is due, V of the tile whose P.V is due
+            int sk = 0, sv = 0;
+            uint32_t kpar = 0, vpar = 0;
             if constexpr (MASK != kMaskWindow) {
                 // Query tiles both start at key tile 0: n0 = b0 <= n1 = b1.
                 const int n0 = b0, n1 = b1;
                 for (int j = 0; ok && j <= n1; ++j) {
                     const int i = j - 1;  // the key tile whose P·V is due
+                    if (i >= 0) {
+                        ok = wait_phase(bar(V_FULL + sv), vpar, abort_flag);
+                        if (!ok) break;
+                    }
                     // PV0_{j-1}
                     if (i >= 0 && i < n0) {
-                        ok = wait_phase(bar(P_FULL + 0), i & 1, abort_flag) &&
-                             wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                        ok = pv_parts(0, Cfg::kSCol0, Cfg::kOCol0, sv, i == 0, i & 1);
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(Cfg::kSCol0, Cfg::kOCol0, i, i == 0);
                         if (i == n0 - 1) mma_commit(bar(O_DONE + 0));
                     }
                     if (j < n1) {
-                        ok = wait_phase(bar(K_FULL + j % NK), (j / NK) & 1, abort_flag);
+                        ok = wait_phase(bar(K_FULL + sk), kpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         if (j < n0) {
-                            issue_s(sQ0, Cfg::kSCol0, j);
+                            issue_s(dq0, Cfg::kSCol0, sk);
                             mma_commit(bar(S_FULL + 0));
                         }
                     }
                     // PV1_{j-1}
                     if (i >= 0) {
-                        ok = wait_phase(bar(P_FULL + 1), i & 1, abort_flag) &&
-                             wait_phase(bar(V_FULL + i % NV), (i / NV) & 1, abort_flag);
+                        ok = pv_parts(1, Cfg::kSCol1, Cfg::kOCol1, sv, i == 0, i & 1);
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(Cfg::kSCol1, Cfg::kOCol1, i, i == 0);
-                        mma_commit(bar(V_EMPTY + i % NV));
+                        mma_commit(bar(V_EMPTY + sv));
                         if (i == n1 - 1) mma_commit(bar(O_DONE + 1));
+                        if (++sv == NV) sv = 0, vpar ^= 1u;
                     }
                     if (j < n1) {
-                        issue_s(sQ1, Cfg::kSCol1, j);
+                        issue_s(dq1, Cfg::kSCol1, sk);
                         mma_commit(bar(S_FULL + 1));
-                        mma_commit(bar(K_EMPTY + j % NK));
+                        mma_commit(bar(K_EMPTY + sk));
+                        if (++sk == NK) sk = 0, kpar ^= 1u;
                     }
                 }
             } else {
                 for (int n = 0; ok && n <= n_all; ++n) {
                     const int j = jlo + n;  // the key tile whose S is due
                     const int i = j - 1;    // the key tile whose P·V is due
+                    if (n >= 1) {
+                        ok = wait_phase(bar(V_FULL + sv), vpar, abort_flag);
+                        if (!ok) break;
+                    }
                     // PV0_{j-1}
                     if (n >= 1 && i >= a0 && i < b0) {
-                        ok = wait_phase(bar(P_FULL + 0), (i - a0) & 1, abort_flag) &&
-                             wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
+                        ok = pv_parts(0, Cfg::kSCol0, Cfg::kOCol0, sv, i == a0, (i - a0) & 1);
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(Cfg::kSCol0, Cfg::kOCol0, n - 1, i == a0);
                         if (i == b0 - 1) mma_commit(bar(O_DONE + 0));
                     }
                     if (n < n_all) {
-                        ok = wait_phase(bar(K_FULL + n % NK), (n / NK) & 1, abort_flag);
+                        ok = wait_phase(bar(K_FULL + sk), kpar, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         if (j >= a0 && j < b0) {
-                            issue_s(sQ0, Cfg::kSCol0, n);
+                            issue_s(dq0, Cfg::kSCol0, sk);
                             mma_commit(bar(S_FULL + 0));
                         }
                     }
                     // PV1_{j-1}
                     if (n >= 1) {
                         if (i >= a1 && i < b1) {
-                            ok = wait_phase(bar(P_FULL + 1), (i - a1) & 1, abort_flag) &&
-                                 wait_phase(bar(V_FULL + (n - 1) % NV), ((n - 1) / NV) & 1, abort_flag);
+                            ok = pv_parts(1, Cfg::kSCol1, Cfg::kOCol1, sv, i == a1, (i - a1) & 1);
                             if (!ok) break;
-                            tc_fence_after();
-                            issue_pv(Cfg::kSCol1, Cfg::kOCol1, n - 1, i == a1);
                             if (i == b1 - 1) mma_commit(bar(O_DONE + 1));
                         }
-                        mma_commit(bar(V_EMPTY + (n - 1) % NV));  // V_{j-1} is no longer needed
+                        mma_commit(bar(V_EMPTY + sv));  // V_{j-1} is no longer needed
+                        if (++sv == NV) sv = 0, vpar ^= 1u;
                     }
                     if (n < n_all) {
                         if (j >= a1 && j < b1) {
-                            issue_s(sQ1, Cfg::kSCol1, n);
+                            issue_s(dq1, Cfg::kSCol1, sk);
                             mma_commit(bar(S_FULL + 1));
                         }
-                        mma_commit(bar(K_EMPTY + n % NK));  // K_j is no longer needed
+                        mma_commit(bar(K_EMPTY + sk));  // K_j is no longer needed
+                        if (++sk == NK) sk = 0, kpar ^= 1u;
                     }
                 }
             }
@@ -456,7 +510,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         regs_increase<kSoftmaxRegs>();
         const int tile = warp >> 2;          // 0: Q0 (warps 0-3), 1: Q1 (warps 4-7)
         const int t = threadIdx.x & 127;     // query row within the tile == TMEM lane
-        const int row = q0 + tile * kBM + t;
+        const int tile_row0 = tile == 0 ? qrow0 : qrow1;
+        const int row = tile_row0 + t;
         const int ta = tile == 0 ? a0 : a1;  // this query tile's key tiles [ta, tb)
         const int tb = tile == 0 ? b0 : b1;
         const int n_kv = tb > ta ? tb - ta : 0;
@@ -467,7 +522,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         int row_lo, row_hi;  // this row's visible keys [row_lo, row_hi)
         row_keys<MASK>(row, a, row_lo, row_hi);
         // band edges of the tile: the largest first key and the smallest end
-        const int tile_row0 = q0 + tile * kBM;
         int edge_lo, edge_hi, unused;
         row_keys<MASK>(min(tile_row0 + kBM - 1, a.Lq - 1), a, edge_lo, unused);
         row_keys<MASK>(tile_row0, a, unused, edge_hi);
@@ -503,62 +557,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     for (int x = 0; x < kBN; ++x) s[x] = (x < hi) ? s[x] : -INFINITY;
                 }
             }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+            // row maximum: four chains of three-input maxima over 32 scores each
+            float mx[4];
 #pragma unroll
-            for (int x = 4; x < kBN; x += 4) {
-                mx0 = fmaxf(mx0, s[x]);
-                mx1 = fmaxf(mx1, s[x + 1]);
-                mx2 = fmaxf(mx2, s[x + 2]);
-                mx3 = fmaxf(mx3, s[x + 3]);
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float m = fmaxf(s[32 * q4], s[32 * q4 + 1]);
+#pragma unroll
+                for (int x = 2; x < 32; x += 2) m = max3(m, s[32 * q4 + x], s[32 * q4 + x + 1]);
+                mx[q4] = m;
             }
-            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+            const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
             const float m_new = (m_tile > m_ref + kRescaleThreshold) ? m_tile : m_ref;
             const float alpha = (m_new == m_ref) ? 1.f : ex2_approx(m_ref - m_new);
             const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
 
-            float rs0 = 0.f, rs1 = 0.f;
-            if constexpr (FP8) {
-                // P in e4m3, four keys per column (the lowest key in the lowest byte);
-                // p <= 2^8 < 448 under the lazy rescale, so it never saturates
-                uint32_t pk[kBN / 4];
-                const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
-                uint64_t rs2 = f2pack(0.f, 0.f);
-#pragma unroll
-                for (int x = 0; x < kBN; x += 4) {
-                    float t0, t1, t2, t3;
-                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
-                    f2unpack(fma2(f2pack(s[x + 2], s[x + 3]), c2, nm2), t2, t3);
-                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                    const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
-                    rs2 = add2(rs2, add2(f2pack(p0, p1), f2pack(p2, p3)));
-                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
-                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
-                    pk[x / 4] = lo | (hi << 16);
-                }
-                f2unpack(rs2, rs0, rs1);
-                // P overwrites the first 32 columns of this tile's S buffer.
-                tmem_st32(lane_base + s_col, pk);
-            } else {
-                // exponent arguments and row sums two at a time (f32x2 instructions)
-                uint32_t pk[kBN / 2];
-                const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
-                uint64_t rs2 = f2pack(0.f, 0.f);
-#pragma unroll
-                for (int x = 0; x < kBN; x += 2) {
-                    float t0, t1;
-                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
-                    const float p0 = ex2_approx(t0);
-                    const float p1 = ex2_approx(t1);
-                    rs2 = add2(rs2, f2pack(p0, p1));
-                    pk[x / 2] = pack2<BF16>(p0, p1);
-                }
-                f2unpack(rs2, rs0, rs1);
-                // P overwrites the first 64 columns of this tile's S buffer (16-bit pairs).
-                tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-                tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            }
-            // Correct O when the reference max moved. S_t(j) completing implies the
-            // P·V of tile j-1 (issued before it) has completed too.
+            // Correct O when the reference max moved, before any part of this tile's P
+            // is handed over. S_t(j) completing implies the P.V of tile j-1 (issued
+            // before it) has completed too.
             if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 32) {
@@ -570,9 +585,68 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     tmem_st32(lane_base + o_col + d0, o);
                 }
             }
+
+            // P = 2^(s*c - m) in two parts: the first kPSplit keys are stored and handed
+            // to the MMA warp (P_FULL) while the rest are still being exponentiated.
+            float rs0 = 0.f, rs1 = 0.f;
+            const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
+            uint64_t rs2 = f2pack(0.f, 0.f);
+            if constexpr (FP8) {
+                // P in e4m3, four keys per column (the lowest key in the lowest byte);
+                // p <= 2^8 < 448 under the lazy rescale, so it never saturates
+                uint32_t pk[kBN / 4];
+#pragma unroll
+                for (int x = 0; x < kBN; x += 4) {
+                    float t0, t1, t2, t3;
+                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
+                    f2unpack(fma2(f2pack(s[x + 2], s[x + 3]), c2, nm2), t2, t3);
+                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+                    rs2 = add2(rs2, add2(f2pack(p0, p1), f2pack(p2, p3)));
+                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+                    pk[x / 4] = lo | (hi << 16);
+                    if (x + 4 == Cfg::kPSplit) {
+                        // columns [0, 24): keys [0, 96)
+                        tmem_st16(lane_base + s_col, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                        tmem_st8(lane_base + s_col + 16, *reinterpret_cast<uint32_t(*)[8]>(&pk[16]));
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar(P_FULL + tile));
+                    }
+                }
+                tmem_st8(lane_base + s_col + 24, *reinterpret_cast<uint32_t(*)[8]>(&pk[24]));
+            } else {
+                // exponent arguments and row sums two at a time (f32x2 instructions)
+                uint32_t pk[kBN / 2];
+#pragma unroll
+                for (int x = 0; x < kBN; x += 2) {
+                    float t0, t1;
+                    f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
+                    float p0, p1;
+                    if (Cfg::kPolyEvery > 0 && (x / 2) % Cfg::kPolyEvery == Cfg::kPolyEvery - 1) {
+                        ex2_fma2(t0, t1, p0, p1);  // on the FMA pipe
+                    } else {
+                        p0 = ex2_approx(t0);
+                        p1 = ex2_approx(t1);
+                    }
+                    rs2 = add2(rs2, f2pack(p0, p1));
+                    pk[x / 2] = pack2<BF16>(p0, p1);
+                    if (x + 2 == Cfg::kPSplit) {
+                        // 16-bit pairs: columns [0, 48) hold keys [0, 96)
+                        tmem_st32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                        tmem_st16(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[32]));
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar(P_FULL + tile));
+                    }
+                }
+                tmem_st16(lane_base + s_col + 48, *reinterpret_cast<uint32_t(*)[16]>(&pk[48]));
+            }
+            f2unpack(rs2, rs0, rs1);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_FULL + tile));
+            mbar_arrive(bar(P_REST + tile));
             l = l * alpha + (rs0 + rs1);
             m_ref = m_new;
         }
@@ -582,7 +656,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ok = __all_sync(0xffffffffu, w);
             if (ok) tc_fence_after();
         }
-        if (ok) {
+        if (ok && (tile == 1 || has_q0)) {
             // ------------------------------------------------------------ epilogue
             // rows past a paged sequence's chunk are written as rows with no key
             const bool real = !PAGED || row < a.Lq;
