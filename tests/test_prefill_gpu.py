@@ -59,6 +59,10 @@ SWEEP += [
     (1, 2, 2, 300, 100, 128, torch.float16, True),     # Lq > Lk: fully masked rows
     (1, 2, 2, 129, 700, 128, torch.bfloat16, False),   # Lq != Lk, ragged both
     (3, 3, 1, 1, 513, 64, torch.float16, True),        # single query row (decode-like)
+    # grids of more than one wave (two query tiles per CTA); the small problems above run
+    # with one query tile per CTA and the key tiles split between the softmax warpgroups
+    (1, 160, 160, 300, 300, 64, torch.float16, True),
+    (2, 96, 48, 257, 385, 128, torch.bfloat16, False),
 ]
 
 

@@ -68,17 +68,15 @@ int sm_count() {
     return known[dev];
 }
 
-// Causal grids of at most one wave take their query tiles in pairs (a short tile with a
-// long one; see PrefillArgs::paired), so every CTA walks about the same number of key
-// tiles instead of the longest one setting the launch's time. Larger grids keep
-// consecutive tiles, longest CTAs first, which balances across waves.
-void choose_query_pairing(PrefillArgs& args, long long planes) {
-    const int T = (args.Lq + attn::kBM - 1) / attn::kBM;
-    const long long paired_ctas = planes * ((T + 1) / 2);
+// When the usual grid (two query tiles per CTA) would leave SMs idle, each CTA takes one
+// query tile and its two softmax warpgroups split the tile's key tiles between them
+// (PrefillArgs::split_kv): twice the CTAs, each about half as long. Needs at least two
+// key tiles to split.
+void choose_split_kv(PrefillArgs& args, long long planes) {
     const int sms = sm_count();
-    if (sms > 0 && paired_ctas <= sms) {
-        args.paired = 1;
-        args.n_q_blocks = (T + 1) / 2;
+    if (sms > 0 && planes * args.n_q_blocks < sms && args.Lk > attn::kBN) {
+        args.split_kv = 1;
+        args.n_q_blocks = (args.Lq + attn::kBM - 1) / attn::kBM;
     }
 }
 
@@ -323,7 +321,7 @@ attn_status_t fwd_band(const void* q, const void* k, const void* v, void* out, f
     const int m = (left < 0 && right < 0) ? attn::kMaskNone
                   : (left < 0 && right == 0) ? attn::kMaskCausal
                                              : attn::kMaskWindow;
-    if (m == attn::kMaskCausal) choose_query_pairing(args, planes_q);
+    choose_split_kv(args, planes_q);
     if (D == 64)
         return bf16 ? dispatch_mask<64, true>(m, tq, tk, tv, args, planes, stream)
                     : dispatch_mask<64, false>(m, tq, tk, tv, args, planes, stream);
@@ -576,7 +574,7 @@ attn_status_t fwd_fp8(const void* q, const attn_strides_t* q_st, const void* k,
     args.win_right = causal ? 0 : -1;
     args.scale_log2 = sc * attn::kLog2e;
     args.o_scale = descale_v;
-    if (causal) choose_query_pairing(args, planes_q);
+    choose_split_kv(args, planes_q);
     const int planes = static_cast<int>(planes_q);
     return causal ? launch_prefill<128, true, attn::kMaskCausal, false, true>(tq, tk, tv, args, planes, stream)
                   : launch_prefill<128, true, attn::kMaskNone, false, true>(tq, tk, tv, args, planes, stream);

@@ -102,9 +102,9 @@ struct PrefillArgs {
     long long out_sb, out_sh, out_sl;  // element strides of out over (batch, head, row)
     float* lse;
     int Hq, Hkv, group, Lq, Lk;
-    int n_q_blocks;    // CTAs along the query axis: ceil(Lq / 256), or ceil(ceil(Lq / 128) / 2) paired
-    int paired;        // causal only: CTA y takes query tiles y and T - 1 - y (T = ceil(Lq / 128)),
-                       // so every CTA walks about the same number of key tiles
+    int n_q_blocks;    // CTAs along the query axis: ceil(Lq / 256), or ceil(Lq / 128) with split_kv
+    int split_kv;      // one query tile per CTA whose key tiles are split between the two
+                       // softmax warpgroups (the first half and the rest), merged at the end
     int win_left;      // band: keys >= i' - win_left visible (-1: unbounded)
     int win_right;     // band: keys <= i' + win_right visible (-1: unbounded; causal: 0)
     float scale_log2;  // scale * log2(e) (8-bit inputs: times the q and k descale factors)
@@ -203,22 +203,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int h = bh % args.Hq;
     const int b = bh / args.Hq;
     const int hkv = h / args.group;  // grouped-query head mapping
-    // First rows of the CTA's two query tiles. Normally two consecutive tiles, the
-    // CTAs with the most key tiles first. Paired (causal grids of at most one wave): a
-    // short tile and a long one, the long one as Q1; the middle tile of an odd count
-    // runs alone as Q1 (Q0 then computes and writes nothing).
-    int qrow0, qrow1;
-    bool has_q0 = true;
-    if (MASK == kMaskCausal && !PAGED && args.paired) {
-        const int T = (args.Lq + kBM - 1) / kBM;
-        qrow0 = blockIdx.y * kBM;
-        qrow1 = (T - 1 - static_cast<int>(blockIdx.y)) * kBM;
-        has_q0 = qrow0 != qrow1;
-    } else {
-        const int qb = args.n_q_blocks - 1 - blockIdx.y;  // longest causal blocks first
-        qrow0 = qb * 2 * kBM;
-        qrow1 = qrow0 + kBM;
-    }
+    // First rows of the CTA's two query tiles, the CTAs with the most key tiles first:
+    // two consecutive tiles, or with split_kv one tile that both softmax warpgroups
+    // work on (each over its share of the key tiles).
+    const bool split = !PAGED && args.split_kv != 0;
+    const int qb = args.n_q_blocks - 1 - blockIdx.y;
+    const int qrow0 = split ? qb * kBM : qb * 2 * kBM;
+    const int qrow1 = split ? qrow0 : qrow0 + kBM;
     // The lengths the masks see: the problem's, or with paged keys the sequence's own
     // (seq_lens[b] keys, q_lens[b] queries at its last positions). Out-of-range values
     // are clamped and reported.
@@ -246,11 +237,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         key_tiles_for<MASK>(qrow0, a, unused, b0);
         key_tiles_for<MASK>(qrow1, a, unused, b1);
     }
-    if (!has_q0) a0 = b0 = 0;
     if (PAGED && qrow0 >= a.Lq) a0 = b0 = a1 = b1 = 0;  // every row past the sequence's chunk
+    if (split) {  // warpgroup 0 takes the first half of the tile's key tiles, 1 the rest
+        const int t0 = (MASK == kMaskWindow) ? a0 : 0, t1 = b0;
+        a0 = t0;
+        b0 = t1 > t0 ? t0 + (t1 - t0 + 1) / 2 : t0;
+        a1 = b0;
+        b1 = t1 > b0 ? t1 : b0;
+    }
     const int jlo = (MASK != kMaskWindow) ? 0 : ((b0 > a0) ? a0 : a1);
     const int jhi = max(b0, b1);
-    const int n_all = (b1 > a1 || b0 > a0) ? jhi - jlo : 0;  // key tiles this CTA loads
+    // key tiles this CTA loads (with split_kv each is used by one warpgroup)
+    const int n_all = split ? (b0 - a0) + (b1 - a1)
+                            : ((b1 > a1 || b0 > a0) ? jhi - jlo : 0);
+    // split_kv ring order: the two warpgroups' tiles alternate, (a0, a1, a0+1, a1+1, ...),
+    // then the rest of warpgroup 0's (it has at least as many)
+    const int ns0 = b0 - a0, ns1 = b1 - a1;
+    auto split_tile = [&](int n) -> int {
+        return n < 2 * ns1 ? ((n & 1) ? a1 : a0) + (n >> 1) : a0 + (n - ns1);
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(Q_FULL), 1);
@@ -295,17 +300,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ------------------------------------------------------------ producer
         regs_decrease<kOtherRegs>();
         if (lane == 0 && n_all > 0) {
-            mbar_arrive_expect_tx(bar(Q_FULL), 2 * Cfg::kTileBytes);
+            mbar_arrive_expect_tx(bar(Q_FULL), (split ? 1 : 2) * Cfg::kTileBytes);
 #pragma unroll
             for (int c = 0; c < Cfg::kChunks; ++c) {
                 tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow0,
                             h, b);
-                tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow1,
-                            h, b);
+                if (!split)
+                    tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems,
+                                qrow1, h, b);
             }
             constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
-            for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile jlo + n
-                const int j = jlo + n;
+            for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile j
+                const int j = split ? split_tile(n) : jlo + n;
                 const int sk = n % NK, sv = n % NV;
                 // Paged keys: the tile's rows come from kBlocks cache blocks; a block past
                 // the sequence loads its first block instead (finite rows, masked), and an
@@ -422,6 +428,44 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // ring positions: K of the tile whose S is due, V of the tile whose P.V is due
             int sk = 0, sv = 0;
             uint32_t kpar = 0, vpar = 0;
+            if (split) {
+                // Both warpgroups work on Q0 (the only query tile), warpgroup t over its own
+                // key tiles, which sit at ring sequence seq(t, m) in the alternating order.
+                // Per step m: PV0 of its tile m-1, S0 of tile m, then the same for
+                // warpgroup 1. Every ring slot is read by one product only.
+                auto seq0 = [&](int m) { return m + min(m, ns1); };
+                auto ring = [&](int q, int nst, int& st, uint32_t& par) {
+                    st = q % nst;
+                    par = static_cast<uint32_t>(q / nst) & 1u;
+                };
+                for (int m = 0; ok && m <= ns0; ++m) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const int nt = t == 0 ? ns0 : ns1;
+                        const uint32_t s_col = t == 0 ? Cfg::kSCol0 : Cfg::kSCol1;
+                        const uint32_t o_col = t == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
+                        if (m >= 1 && m - 1 < nt) {  // P.V of this warpgroup's tile m-1
+                            const int q = t == 0 ? seq0(m - 1) : 2 * (m - 1) + 1;
+                            ring(q, NV, sv, vpar);
+                            ok = wait_phase(bar(V_FULL + sv), vpar, abort_flag) &&
+                                 pv_parts(t, s_col, o_col, sv, m == 1, (m - 1) & 1);
+                            if (!ok) break;
+                            if (m - 1 == nt - 1) mma_commit(bar(O_DONE + t));
+                            mma_commit(bar(V_EMPTY + sv));
+                        }
+                        if (m < nt) {  // S of its tile m
+                            const int q = t == 0 ? seq0(m) : 2 * m + 1;
+                            ring(q, NK, sk, kpar);
+                            ok = wait_phase(bar(K_FULL + sk), kpar, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_s(dq0, s_col, sk);
+                            mma_commit(bar(S_FULL + t));
+                            mma_commit(bar(K_EMPTY + sk));
+                        }
+                    }
+                }
+            } else
             if constexpr (MASK != kMaskWindow) {
                 // Query tiles both start at key tile 0: n0 = b0 <= n1 = b1.
                 const int n0 = b0, n1 = b1;
@@ -656,7 +700,62 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ok = __all_sync(0xffffffffu, w);
             if (ok) tc_fence_after();
         }
-        if (ok && (tile == 1 || has_q0)) {
+        if (split) {
+            // ------------------------------------------------ split_kv merge epilogue
+            // Each warpgroup holds the row's partial (O_t, m_t, l_t) over its share of
+            // the key tiles: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / L with M the larger
+            // reference max and L = l_0 2^(m_0 - M) + l_1 2^(m_1 - M) (the same
+            // log-sum-exp combine as split-KV decoding). The statistics meet in shared
+            // memory (the unused second Q buffer); every softmax thread reaches the
+            // barrier, also after a wait gave up, so it cannot hang.
+            float* stat = reinterpret_cast<float*>(smem + Cfg::kTileBytes);  // [2][2][128]
+            stat[tile * 256 + t] = m_ref;
+            stat[tile * 256 + 128 + t] = l;
+            tc_fence_before();
+            named_barrier_sync(1, 256);
+            tc_fence_after();
+            if (!*abort_flag) {
+                const float m0 = stat[t], l0 = stat[128 + t];
+                const float m1 = stat[256 + t], l1 = stat[384 + t];
+                const float M = fmaxf(m0, m1);
+                const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M);
+                const float f1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+                const float L = l0 * f0 + l1 * f1;
+                const bool has = L > 0.f;
+                const float inv_l = has ? (FP8 ? args.o_scale : 1.f) / L : 0.f;
+                const float g0 = f0 * inv_l, g1 = f1 * inv_l;
+                uint16_t* out_row = reinterpret_cast<uint16_t*>(args.out) + b * args.out_sb +
+                                    h * args.out_sh + static_cast<long long>(row) * args.out_sl;
+                // warpgroup t writes the columns [t D / 2, (t + 1) D / 2)
+#pragma unroll
+                for (int d0 = tile * (D / 2); d0 < (tile + 1) * (D / 2); d0 += 32) {
+                    uint32_t o0[32], o1[32];
+                    tmem_ld32(lane_base + Cfg::kOCol0 + d0, o0);
+                    if (ns1 > 0) tmem_ld32(lane_base + Cfg::kOCol1 + d0, o1);
+                    tmem_wait_ld();
+                    uint32_t pkd[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        float v0 = __uint_as_float(o0[2 * x]) * g0;
+                        float v1 = __uint_as_float(o0[2 * x + 1]) * g0;
+                        if (ns1 > 0) {
+                            v0 = fmaf(__uint_as_float(o1[2 * x]), g1, v0);
+                            v1 = fmaf(__uint_as_float(o1[2 * x + 1]), g1, v1);
+                        }
+                        pkd[x] = has ? pack2<BF16>(v0, v1) : 0u;
+                    }
+                    if (row < args.Lq) {
+                        uint4* dst = reinterpret_cast<uint4*>(out_row + d0);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+                    }
+                }
+                if (tile == 0 && args.lse != nullptr && row < args.Lq)
+                    args.lse[static_cast<size_t>(bh) * args.Lq + row] =
+                        has ? (M + log2f(L)) * kLn2 : -INFINITY;
+            }
+        } else if (ok) {
             // ------------------------------------------------------------ epilogue
             // rows past a paged sequence's chunk are written as rows with no key
             const bool real = !PAGED || row < a.Lq;

@@ -259,6 +259,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Register reallocation between warpgroups (all warps of a warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void regs_increase() {
