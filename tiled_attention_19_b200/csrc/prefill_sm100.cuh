@@ -412,16 +412,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                (!first || ks > 0) ? 1u : 0u);
                 }
             };
-            // O_t += P_t V: the first part of P as soon as it is in TMEM, then the rest.
-            // V is already known to be in stage sv. Returns false if a wait gave up.
+            // O_t += P_t V. At D = 64 the first part of P goes as soon as it is in TMEM
+            // and the rest after it (there the products wait for the softmax); at D = 128,
+            // where P is always ready first, all of it after both parts (one wait fewer on
+            // the issuing thread: measured about 2 % faster). V is already known to be in
+            // stage sv. Returns false if a wait gave up.
             auto pv_parts = [&](int t, uint32_t p_col, uint32_t o_col, int sv, bool first,
                                 uint32_t parity) -> bool {
-                if (!wait_phase(bar(P_FULL + t), parity, abort_flag)) return false;
-                tc_fence_after();
-                issue_pv(p_col, o_col, sv, first, 0, Cfg::kPSplit);
-                if (!wait_phase(bar(P_REST + t), parity, abort_flag)) return false;
-                tc_fence_after();
-                issue_pv(p_col, o_col, sv, first, Cfg::kPSplit, kBN);
+                if constexpr (D == 64) {
+                    if (!wait_phase(bar(P_FULL + t), parity, abort_flag)) return false;
+                    tc_fence_after();
+                    issue_pv(p_col, o_col, sv, first, 0, Cfg::kPSplit);
+                    if (!wait_phase(bar(P_REST + t), parity, abort_flag)) return false;
+                    tc_fence_after();
+                    issue_pv(p_col, o_col, sv, first, Cfg::kPSplit, kBN);
+                } else {
+                    if (!wait_phase(bar(P_FULL + t), parity, abort_flag) ||
+                        !wait_phase(bar(P_REST + t), parity, abort_flag))
+                        return false;
+                    tc_fence_after();
+                    issue_pv(p_col, o_col, sv, first, 0, kBN);
+                }
                 return true;
             };
             bool ok = wait_phase(bar(Q_FULL), 0, abort_flag);
