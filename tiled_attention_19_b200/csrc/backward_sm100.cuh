@@ -375,13 +375,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_started = true;
             // S = X Y^T into column s_col, or dP = W Z^T into DP_COL (K-major operands: 16
             // elements = 32 bytes per step inside a 128-byte swizzle row, then the next chunk).
+            // The issue of a tcgen05.mma blocks while the tensor core's queue is full, so
+            // work between products idles it: each operand's descriptor is built once per
+            // call and offset per step (the start address is the descriptor's low field, in
+            // 16-byte units, and never carries out of it).
             auto issue_prod = [&](uint32_t a_tile, uint32_t b_tile, uint32_t d_col) {
+                const uint64_t da = sdesc_sw128(a_tile, 16, 1024), db = sdesc_sw128(b_tile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t fa = (kk >> 2) * Cfg::kFixChunk + (kk & 3) * 32;
-                    const uint32_t fb = (kk >> 2) * Cfg::kSubChunk + (kk & 3) * 32;
-                    mma_ss(tmem + d_col, sdesc_sw128(a_tile + fa, 16, 1024),
-                           sdesc_sw128(b_tile + fb, 16, 1024), kIdescSD, kk > 0 ? 1u : 0u);
+                    const uint32_t fa = ((kk >> 2) * Cfg::kFixChunk + (kk & 3) * 32) >> 4;
+                    const uint32_t fb = ((kk >> 2) * Cfg::kSubChunk + (kk & 3) * 32) >> 4;
+                    mma_ss(tmem + d_col, da + fa, db + fb, kIdescSD, kk > 0 ? 1u : 0u);
                 }
             };
             // acc += A B with A the f16/bf16 tile the softmax warps packed into TMEM at
@@ -389,11 +393,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // MN-major from a sub-tile (16 rows = two 8-row swizzle atoms, 2048 bytes;
             // D chunks kSubChunk apart).
             auto issue_grad = [&](uint32_t acc_col, uint32_t a_col, uint32_t b_tile, bool first) {
+                const uint64_t db = sdesc_sw128(b_tile, Cfg::kSubChunk, 1024);
 #pragma unroll
                 for (int ks = 0; ks < kBwdSub / 16; ++ks)
                     mma_ts(tmem + acc_col, tmem + a_col + (ks >> 2) * 64 + (ks & 3) * 8,
-                           sdesc_sw128(b_tile + ks * 2048, Cfg::kSubChunk, 1024), kIdescG,
-                           (!first || ks > 0) ? 1u : 0u);
+                           db + ks * (2048 >> 4), kIdescG, (!first || ks > 0) ? 1u : 0u);
             };
             bool ok = wait_phase(bar(FIX_FULL), 0, abort_flag) &&
                       wait_phase(bar(Y_FULL + 0), 0, abort_flag) &&
