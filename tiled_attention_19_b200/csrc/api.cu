@@ -224,6 +224,28 @@ bool encode_cache_map(CUtensorMap* tm, const void* base, bool bf16, int D, long 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view (64, rows, D / 64) of a paged cache [num_blocks, H_kv, 16, D] for the decode:
+// one box {64, 16, D / 64} is a whole block's 16 rows as D / 64 swizzled 16 x 64 tiles (the
+// second coordinate steps over rows, the third over 64-column chunks), so one TMA load
+// brings a block's K (or V).
+bool encode_block_map(CUtensorMap* tm, const void* base, bool bf16, int D, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(D / 64)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(attn::kPageSize),
+                               static_cast<cuuint32_t>(D / 64)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The decode is launched with programmatic stream serialisation: it may start while the
+// kernel before it in the stream finishes, and waits for that kernel (griddepcontrol.wait)
+// before it reads or writes any global memory. Back-to-back decode calls then overlap one
+// launch's start-up with the previous one's tail.
 template <int D, bool BF16>
 attn_status_t launch_paged(const CUtensorMap& tk, const CUtensorMap& tv, const PagedArgs& a,
                            int grid, cudaStream_t stream) {
@@ -235,8 +257,21 @@ attn_status_t launch_paged(const CUtensorMap& tk, const CUtensorMap& tv, const P
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
     if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-    kern<<<static_cast<unsigned>(grid), attn::kDecThreads, smem, stream>>>(tk, tv, a);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(attn::kDecThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
 }
 
 // Dense forward with a band of visible keys: key j is visible to query i iff
@@ -667,7 +702,7 @@ attn_status_t paged_prefill(const void* q, const attn_strides_t* q_st, const voi
                   : launch_prefill<128, false, attn::kMaskNone, true>(tq, tk, tv, args, planes, stream);
 }
 
-// Tensor maps of paged caches, cached by what they encode (base address, rows, D,
+// Decode tensor maps of paged caches (encode_block_map), cached by what they encode (base address, rows, D,
 // dtype, device): a map holds nothing else, so a cached map is exact even if the
 // memory behind an address was freed and reallocated with the same extent.
 struct CacheMapKey {
@@ -697,7 +732,7 @@ bool cached_cache_map(CUtensorMap* tm, const void* base, bool bf16, int D, long 
             *tm = maps[i];
             return true;
         }
-    if (!encode_cache_map(tm, base, bf16, D, rows)) return false;
+    if (!encode_block_map(tm, base, bf16, D, rows)) return false;
     const int slot = used < kSlots ? used++ : (next++ % kSlots);
     keys[slot] = key;
     maps[slot] = *tm;

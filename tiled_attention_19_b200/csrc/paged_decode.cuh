@@ -105,7 +105,7 @@ inline PagedLayout paged_layout(int num_seqs, int Hq, int Hkv, int D, int max_bl
     return L;
 }
 
-// 2-D TMA load (x = column, y = row) into shared memory, completion counted on `bar`.
+// ldmatrix of four 8x8 16-bit matrices from shared memory (and the transposing form).
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -169,6 +169,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t ring = smem_u32(smem);
 
+    // Launched with programmatic stream serialisation: wait for the previous kernel of the
+    // stream before touching global memory, and let the next one launch at once (its CTAs
+    // take this grid's places as they free up and wait here in turn).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -385,11 +390,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                         mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
                         const int row = (p * Hkv + hkv) * kPageSize;
                         const uint32_t dst = ring + s * Cfg::kStageBytes;
-#pragma unroll
-                        for (int c = 0; c < D / 64; ++c) {
-                            tma_load_2d(dst + c * Cfg::kTileBytes, &tm_k, fb, c * 64, row);
-                            tma_load_2d(dst + Cfg::kKBytes + c * Cfg::kTileBytes, &tm_v, fb, c * 64, row);
-                        }
+                        // one load per block and tensor: its 16 rows as D/64 swizzled tiles
+                        tma_load_3d(dst, &tm_k, fb, 0, row, 0);
+                        tma_load_3d(dst + Cfg::kKBytes, &tm_v, fb, 0, row, 0);
                     }
                     if (ok) issued = i + 1;
                 }
