@@ -192,12 +192,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     }
     // ------------------------------------------------------------ the schedule
     int unit = -1, b0 = 0, b1 = 0, chunk0 = 0, nchunk = 1;
+    int raw_len = -1;  // the unit's seq_lens entry, when the schedule already read it
     if (a.balanced && U <= 32) {
         // One warp derives the schedule for up to 32 units with shuffles only.
         if (warp == 0) {
-            int nbu = 0;
+            int nbu = 0, raw = 0;
             if (lane < U) {
-                int len = a.seq_lens[lane / Hkv];
+                raw = a.seq_lens[lane / Hkv];
+                int len = raw;
                 if (len < 0 || len > cap) len = len < 0 ? 0 : cap;
                 nbu = (len + kPageSize - 1) / kPageSize;
             }
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 s_red[2] = static_cast<int>(static_cast<long long>(k + 1) * nbu / v);
                 s_red[3] = start;
                 s_red[4] = v;
+                s_red[5] = raw;  // the unit's sequence length as read
             }
         }
         __syncthreads();
@@ -244,6 +247,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         b1 = s_red[2];
         chunk0 = s_red[3];
         nchunk = s_red[4];
+        raw_len = s_red[5];
     } else if (a.balanced) {
         // pass 1: blocks per unit, and their total T
         int part = 0;
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     }
     const int sq = unit / Hkv;
     const int hkv = unit % Hkv;
-    int len = a.seq_lens[sq];
+    int len = (a.balanced && U <= 32) ? raw_len : a.seq_lens[sq];
     if (len < 0 || len > cap) {
         if (tid == 0 && b0 == 0) report_status(ATTN_ERR_BAD_INDEX);
         len = len < 0 ? 0 : cap;
@@ -537,10 +541,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         for (int nt = 0; nt < NT; ++nt) {
             float* r0 = sm_o + (warp * kMaxGroup + g) * kRow + nt * 8 + 2 * t;
             float* r1 = sm_o + (warp * kMaxGroup + g + 8) * kRow + nt * 8 + 2 * t;
-            r0[0] = oacc[nt][0];
-            r0[1] = oacc[nt][1];
-            r1[0] = oacc[nt][2];
-            r1[1] = oacc[nt][3];
+            *reinterpret_cast<float2*>(r0) = make_float2(oacc[nt][0], oacc[nt][1]);
+            *reinterpret_cast<float2*>(r1) = make_float2(oacc[nt][2], oacc[nt][3]);
         }
     }
     __syncthreads();
@@ -613,10 +615,49 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         mbar_arrive_expect_tx(smem_u32(&merge_bar), part_bytes);
         bulk_load(smem_u32(s_part), part, part_bytes, smem_u32(&merge_bar));
     }
-    // All chunks' log2-sum-exp in shared memory (one round of parallel loads), then per
-    // row the maximum, the total weight and each chunk's normalised weight.
+    // All chunks' log2-sum-exp in shared memory (one round of parallel loads).
     for (int i = tid; i < nw; i += blockDim.x) s_w[i] = __ldcg(plse + i);
+    // Few chunks: every thread forms its row's maximum and weights from the staged values
+    // itself, so one barrier (after the bulk copy has landed) is all the merge waits on.
+    constexpr int kFewChunks = 16;
+    if (staged && nchunk <= kFewChunks) {
+        if (tid == 0 && !wait_phase(smem_u32(&merge_bar), 0, abort_flag))
+            drain_phase(smem_u32(&merge_bar), 0);  // gave up (reported): let the copy land
+        __syncthreads();
+        if (*abort_flag) return;
+        for (int i4 = tid; i4 < G * (D / 4); i4 += blockDim.x) {
+            const int r = i4 / (D / 4), d = (i4 % (D / 4)) * 4;
+            float M = -INFINITY;
+            for (int k = 0; k < nchunk; ++k) M = fmaxf(M, s_w[k * G + r]);
+            float W = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (M != -INFINITY) {
+                const float4* src = reinterpret_cast<const float4*>(s_part + r * D + d);
+                for (int k = 0; k < nchunk; ++k) {
+                    const float w = ex2_approx(s_w[k * G + r] - M);
+                    const float4 v = src[k * (G * D / 4)];
+                    W += w;
+                    acc.x = fmaf(w, v.x, acc.x);
+                    acc.y = fmaf(w, v.y, acc.y);
+                    acc.z = fmaf(w, v.z, acc.z);
+                    acc.w = fmaf(w, v.w, acc.w);
+                }
+            }
+            const float inv = W > 0.f ? 1.f / W : 0.f;
+            const size_t orow = static_cast<size_t>(sq) * a.Hq + hkv * G + r;
+            uint2 pk;
+            pk.x = pack2<BF16>(acc.x * inv, acc.y * inv);
+            pk.y = pack2<BF16>(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(a.out + orow * D + d) = pk;
+            if (d == 0 && a.lse != nullptr)
+                a.lse[orow] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
+        }
+        if (tid == 0) a.ws_count[unit] = 0;  // leave the workspace as found
+        return;
+    }
     __syncthreads();
+    // Many chunks: per row the maximum, the total weight and each chunk's normalised
+    // weight, one warp per row.
     for (int r = warp; r < G; r += kDecThreads / 32) {
         float M = -INFINITY;
         for (int k = lane; k < nchunk; k += 32) M = fmaxf(M, s_w[k * G + r]);
