@@ -169,12 +169,23 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t ring = smem_u32(smem);
 
+    const int tid = threadIdx.x;
+    // Barriers first: this needs no global memory, so under programmatic stream
+    // serialisation it overlaps the previous kernel's tail.
+    if (tid == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        mbar_init(smem_u32(&merge_bar), 1);
+        s_abort = 0;
+        fence_barrier_init();
+    }
     // Launched with programmatic stream serialisation: wait for the previous kernel of the
     // stream before touching global memory, and let the next one launch at once (its CTAs
     // take this grid's places as they free up and wait here in turn).
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int Hkv = a.Hkv, G = a.G;
@@ -342,16 +353,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     }
     const int nb = b1 - b0;
 
-    if (tid == 0) {
-        for (int s = 0; s < kDecStages; ++s) {
-            mbar_init(smem_u32(&full_bar[s]), 1);
-            mbar_init(smem_u32(&empty_bar[s]), 1);
-        }
-        mbar_init(smem_u32(&merge_bar), 1);
-        s_abort = 0;
-        fence_barrier_init();
-    }
-    __syncthreads();
+    __syncthreads();  // the barriers are initialised
 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g + 8
     float oacc[NT][4];
