@@ -84,9 +84,6 @@ struct PrefillCfg {
     static constexpr int kTmemCols = 512;
     // P is handed to the MMA warp in two parts: the first kPSplit keys, then the rest
     // (kPSplit is a multiple of kPVKeys, so each part is whole P.V instructions).
-    // One pair of exponentials in kPolyEvery is computed on the FMA pipe instead of the
-    // MUFU (0: none).
-    static constexpr int kPolyEvery = 0;
     static constexpr int kPSplit = 96;  // the softmax's stores below are laid out for 96
     static_assert(kPSplit == 96 && kBN == 128, "P hand-off layout");
     // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
@@ -678,13 +675,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int x = 0; x < kBN; x += 2) {
                     float t0, t1;
                     f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
-                    float p0, p1;
-                    if (Cfg::kPolyEvery > 0 && (x / 2) % Cfg::kPolyEvery == Cfg::kPolyEvery - 1) {
-                        ex2_fma2(t0, t1, p0, p1);  // on the FMA pipe
-                    } else {
-                        p0 = ex2_approx(t0);
-                        p1 = ex2_approx(t1);
-                    }
+                    const float p0 = ex2_approx(t0);
+                    const float p1 = ex2_approx(t1);
                     rs2 = add2(rs2, f2pack(p0, p1));
                     pk[x / 2] = pack2<BF16>(p0, p1);
                     if (x + 2 == Cfg::kPSplit) {
