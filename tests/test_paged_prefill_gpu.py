@@ -37,7 +37,11 @@ def make_cache(seed, S, Hq, Hkv, Lq, D, dtype, seq_lens, spare_blocks=3):
 
 
 def test_full_sequence_equals_dense_kernel():
-    S, H, L, D, dtype = 2, 4, 1000, 128, torch.bfloat16
+    # 40 heads: the dense grid (2 x 40 heads x 4 pairs of query tiles) is more than one
+    # wave, so the dense kernel keeps two query tiles per CTA like the paged one and the
+    # results must agree bit for bit (a smaller grid splits each tile's key tiles between
+    # the softmax warpgroups, which rounds differently).
+    S, H, L, D, dtype = 2, 40, 1000, 128, torch.bfloat16
     q, kc, vc, bt, sl = make_cache(1, S, H, H, L, D, dtype, [L, L])
     out, lse = ta.fwd_paged_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), bt.to(DEV), sl.to(DEV),
                                     causal=True)
