@@ -247,6 +247,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // key tiles this CTA loads (with split_kv each is used by one warpgroup)
     const int n_all = split ? (b0 - a0) + (b1 - a1)
                             : ((b1 > a1 || b0 > a0) ? jhi - jlo : 0);
+    // Both query tiles walking key tiles 0 .. jhi-1 together (no window, no split): one
+    // full barrier per key tile j counts K_j and V_{j-1}, and one empty barrier per key
+    // tile, committed after S1_j, releases both K_j's and V_{j-1}'s ring slots (the K
+    // ring's barriers serve as both; the V ring's are unused). The MMA warp then waits and
+    // commits once per key tile for the ring instead of twice.
+    const bool paired = MASK != kMaskWindow && !split;
+    static_assert(NK >= NV, "the empty barrier of a key tile is looked up in the K ring");
     // split_kv ring order: the two warpgroups' tiles alternate, (a0, a1, a0+1, a1+1, ...),
     // then the rest of warpgroup 0's (it has at least as many)
     const int ns0 = b0 - a0, ns1 = b1 - a1;
@@ -307,13 +314,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                 qrow1, h, b);
             }
             constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
-            for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile j
-                const int j = split ? split_tile(n) : jlo + n;
-                const int sk = n % NK, sv = n % NV;
-                // Paged keys: the tile's rows come from kBlocks cache blocks; a block past
-                // the sequence loads its first block instead (finite rows, masked), and an
-                // entry outside the pool is reported and replaced by block 0.
-                int rows[PAGED ? kBlocks : 1];
+            // Paged keys: a tile's rows come from kBlocks cache blocks; a block past the
+            // sequence loads its first block instead (finite rows, masked), and an entry
+            // outside the pool is reported and replaced by block 0.
+            auto block_rows = [&](int j, int (&rows)[PAGED ? kBlocks : 1]) {
                 if constexpr (PAGED) {
                     const int32_t* tbl = args.block_table + static_cast<size_t>(b) * args.max_blocks;
                     const int nblk = (a.Lk + kPageSize - 1) / kPageSize;
@@ -328,35 +332,65 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         rows[k] = (e * args.Hkv + hkv) * kPageSize;
                     }
                 }
-                if (n >= NK && !wait_phase(bar(K_EMPTY + sk), ((n / NK) - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
+            };
+            // K or V of key tile j into the 128-byte-swizzled tile at dst, counted on fb
+            auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t fb, int j,
+                                 const int (&rows)[PAGED ? kBlocks : 1]) {
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c) {
-                    const uint32_t dst = sK0 + sk * Cfg::kTileBytes + c * Cfg::kChunkBytes;
                     if constexpr (PAGED) {
 #pragma unroll
                         for (int k = 0; k < kBlocks; ++k)
-                            tma_load_2d(dst + k * kPageSize * 128, &tm_k, bar(K_FULL + sk), c * 64,
-                                        rows[k]);
+                            tma_load_2d(dst + c * Cfg::kChunkBytes + k * kPageSize * 128, tm, fb,
+                                        c * 64, rows[k]);
                     } else {
-                        tma_load_4d(dst, &tm_k, bar(K_FULL + sk), c * Cfg::kChunkElems, j * kBN, hkv, b);
+                        tma_load_4d(dst + c * Cfg::kChunkBytes, tm, fb, c * Cfg::kChunkElems, j * kBN,
+                                    hkv, b);
                     }
                 }
+            };
+            if (paired) {
+                // iteration j: K_j (if j < n_all) and V_{j-1} (if j >= 1) on full barrier j
+                int rows_k[PAGED ? kBlocks : 1], rows_v[PAGED ? kBlocks : 1];
+                for (int j = 0; j <= n_all; ++j) {
+                    const bool has_k = j < n_all, has_v = j >= 1;
+                    const int sf = j % NK;
+                    if (has_k) block_rows(j, rows_k);
+                    // Full barrier j % NK was last armed for j-NK, and K_j takes the slot of
+                    // K_{j-NK}: both are free once the empty barrier of j-NK completes (the
+                    // MMA warp waited on that full barrier before committing it). V_{j-1}
+                    // takes the slot of V_{j-1-NV}, freed by the empty barrier of j-NV, a
+                    // later one when NV < NK.
+                    if (j >= NK && !wait_phase(bar(K_EMPTY + sf), ((j / NK) - 1) & 1, abort_flag))
+                        break;
+                    if (NV < NK && has_v && j - 1 >= NV &&
+                        !wait_phase(bar(K_EMPTY + (j - NV) % NK), ((j - NV) / NK) & 1, abort_flag))
+                        break;
+                    mbar_arrive_expect_tx(bar(K_FULL + sf), (has_k ? Cfg::kTileBytes : 0) +
+                                                                 (has_v ? Cfg::kTileBytes : 0));
+                    if (has_k) load_tile(&tm_k, sK0 + sf * Cfg::kTileBytes, bar(K_FULL + sf), j, rows_k);
+                    if (has_v)
+                        load_tile(&tm_v, sV0 + ((j - 1) % NV) * Cfg::kTileBytes, bar(K_FULL + sf), j - 1,
+                                  rows_v);
+                    k_issued = j + 1;  // full barriers armed (drained after an abort)
+                    if constexpr (PAGED) {
+#pragma unroll
+                        for (int k = 0; k < kBlocks; ++k) rows_v[k] = rows_k[k];
+                    }
+                }
+            } else
+            for (int n = 0; n < n_all; ++n) {  // ring sequence n holds key tile j
+                const int j = split ? split_tile(n) : jlo + n;
+                const int sk = n % NK, sv = n % NV;
+                int rows[PAGED ? kBlocks : 1];
+                block_rows(j, rows);
+                if (n >= NK && !wait_phase(bar(K_EMPTY + sk), ((n / NK) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(K_FULL + sk), Cfg::kTileBytes);
+                load_tile(&tm_k, sK0 + sk * Cfg::kTileBytes, bar(K_FULL + sk), j, rows);
                 k_issued = n + 1;
                 if (n >= NV && !wait_phase(bar(V_EMPTY + sv), ((n / NV) - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar(V_FULL + sv), Cfg::kTileBytes);
-#pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c) {
-                    const uint32_t dst = sV0 + sv * Cfg::kTileBytes + c * Cfg::kChunkBytes;
-                    if constexpr (PAGED) {
-#pragma unroll
-                        for (int k = 0; k < kBlocks; ++k)
-                            tma_load_2d(dst + k * kPageSize * 128, &tm_v, bar(V_FULL + sv), c * 64,
-                                        rows[k]);
-                    } else {
-                        tma_load_4d(dst, &tm_v, bar(V_FULL + sv), c * Cfg::kChunkElems, j * kBN, hkv, b);
-                    }
-                }
+                load_tile(&tm_v, sV0 + sv * Cfg::kTileBytes, bar(V_FULL + sv), j, rows);
                 v_issued = n + 1;
             }
         }
@@ -475,43 +509,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
             } else
             if constexpr (MASK != kMaskWindow) {
-                // Query tiles both start at key tile 0: n0 = b0 <= n1 = b1.
+                // Query tiles both start at key tile 0: n0 = b0 <= n1 = b1 = n_all. Full
+                // barrier j (entry j % NK) covers K_j and V_{j-1}; the empty barrier of j,
+                // committed after S1_j (so after PV1_{j-1} too), frees both their slots.
                 const int n0 = b0, n1 = b1;
                 for (int j = 0; ok && j <= n1; ++j) {
                     const int i = j - 1;  // the key tile whose P·V is due
-                    if (i >= 0) {
-                        ok = wait_phase(bar(V_FULL + sv), vpar, abort_flag);
-                        if (!ok) break;
-                    }
+                    ok = wait_phase(bar(K_FULL + sk), kpar, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
                     // PV0_{j-1}
                     if (i >= 0 && i < n0) {
                         ok = pv_parts(0, Cfg::kSCol0, Cfg::kOCol0, sv, i == 0, i & 1);
                         if (!ok) break;
                         if (i == n0 - 1) mma_commit(bar(O_DONE + 0));
                     }
-                    if (j < n1) {
-                        ok = wait_phase(bar(K_FULL + sk), kpar, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        if (j < n0) {
-                            issue_s(dq0, Cfg::kSCol0, sk);
-                            mma_commit(bar(S_FULL + 0));
-                        }
+                    if (j < n0) {
+                        issue_s(dq0, Cfg::kSCol0, sk);
+                        mma_commit(bar(S_FULL + 0));
                     }
                     // PV1_{j-1}
                     if (i >= 0) {
                         ok = pv_parts(1, Cfg::kSCol1, Cfg::kOCol1, sv, i == 0, i & 1);
                         if (!ok) break;
-                        mma_commit(bar(V_EMPTY + sv));
                         if (i == n1 - 1) mma_commit(bar(O_DONE + 1));
-                        if (++sv == NV) sv = 0, vpar ^= 1u;
+                        if (++sv == NV) sv = 0;
                     }
                     if (j < n1) {
                         issue_s(dq1, Cfg::kSCol1, sk);
                         mma_commit(bar(S_FULL + 1));
                         mma_commit(bar(K_EMPTY + sk));
-                        if (++sk == NK) sk = 0, kpar ^= 1u;
                     }
+                    if (++sk == NK) sk = 0, kpar ^= 1u;
                 }
             } else {
                 for (int n = 0; ok && n <= n_all; ++n) {
@@ -805,6 +834,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Nothing may still be writing into this CTA's shared or tensor memory when
         // it exits: wait for the loads already issued and for every MMA issued.
         if (warp == 8 && lane == 0 && n_all > 0) {
+            // the K ring's full barriers (in the paired scheme they also count V) and the
+            // V ring's (the other schemes)
             drain_phase(bar(Q_FULL), 0);
             for (int j = max(0, k_issued - NK); j < k_issued; ++j)
                 drain_phase(bar(K_FULL + j % NK), (j / NK) & 1);
