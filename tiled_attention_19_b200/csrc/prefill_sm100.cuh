@@ -85,6 +85,7 @@ struct PrefillCfg {
     // P is handed to the MMA warp in two parts: the first kPSplit keys, then the rest
     // (kPSplit is a multiple of kPVKeys, so each part is whole P.V instructions).
     static constexpr int kPSplit = 96;  // the softmax's stores below are laid out for 96
+    static constexpr bool kSplitP = D == 64;  // the MMA warp takes the first part early
     static_assert(kPSplit == 96 && kBN == 128, "P hand-off layout");
     // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
     // S_FULL[2], P_FULL[2] (first part of P), P_REST[2] (the rest), O_DONE[2], DRAIN
@@ -445,12 +446,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             };
             // O_t += P_t V. At D = 64 the first part of P goes as soon as it is in TMEM
             // and the rest after it (there the products wait for the softmax); at D = 128,
-            // where P is always ready first, all of it after both parts (one wait fewer on
-            // the issuing thread: measured about 2 % faster). V is already known to be in
+            // where P is always ready first, all of it after the one arrival that follows
+            // both parts (fewer waits on the issuing thread). V is already known to be in
             // stage sv. Returns false if a wait gave up.
             auto pv_parts = [&](int t, uint32_t p_col, uint32_t o_col, int sv, bool first,
                                 uint32_t parity) -> bool {
-                if constexpr (D == 64) {
+                if constexpr (Cfg::kSplitP) {
                     if (!wait_phase(bar(P_FULL + t), parity, abort_flag)) return false;
                     tc_fence_after();
                     issue_pv(p_col, o_col, sv, first, 0, Cfg::kPSplit);
@@ -458,9 +459,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     tc_fence_after();
                     issue_pv(p_col, o_col, sv, first, Cfg::kPSplit, kBN);
                 } else {
-                    if (!wait_phase(bar(P_FULL + t), parity, abort_flag) ||
-                        !wait_phase(bar(P_REST + t), parity, abort_flag))
-                        return false;
+                    if (!wait_phase(bar(P_FULL + t), parity, abort_flag)) return false;
                     tc_fence_after();
                     issue_pv(p_col, o_col, sv, first, 0, kBN);
                 }
@@ -667,8 +666,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
             }
 
-            // P = 2^(s*c - m) in two parts: the first kPSplit keys are stored and handed
-            // to the MMA warp (P_FULL) while the rest are still being exponentiated.
+            // P = 2^(s*c - m), stored in two parts. At D = 64 the first kPSplit keys are
+            // handed to the MMA warp (P_FULL) while the rest are still being exponentiated
+            // (P_REST); at D = 128 the MMA warp only ever needs all of P, so one arrival
+            // (P_FULL) after both parts spares it a wait.
             float rs0 = 0.f, rs1 = 0.f;
             const uint64_t c2 = f2pack(c, c), nm2 = f2pack(neg_m, neg_m);
             uint64_t rs2 = f2pack(0.f, 0.f);
@@ -691,9 +692,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         // columns [0, 24): keys [0, 96)
                         tmem_st16(lane_base + s_col, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
                         tmem_st8(lane_base + s_col + 16, *reinterpret_cast<uint32_t(*)[8]>(&pk[16]));
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(bar(P_FULL + tile));
+                        if constexpr (Cfg::kSplitP) {
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(bar(P_FULL + tile));
+                        }
                     }
                 }
                 tmem_st8(lane_base + s_col + 24, *reinterpret_cast<uint32_t(*)[8]>(&pk[24]));
@@ -712,9 +715,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         // 16-bit pairs: columns [0, 48) hold keys [0, 96)
                         tmem_st32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
                         tmem_st16(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[32]));
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(bar(P_FULL + tile));
+                        if constexpr (Cfg::kSplitP) {
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(bar(P_FULL + tile));
+                        }
                     }
                 }
                 tmem_st16(lane_base + s_col + 48, *reinterpret_cast<uint32_t(*)[16]>(&pk[48]));
@@ -722,7 +727,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             f2unpack(rs2, rs0, rs1);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_REST + tile));
+            mbar_arrive(bar((Cfg::kSplitP ? P_REST : P_FULL) + tile));
             l = l * alpha + (rs0 + rs1);
             m_ref = m_new;
         }
