@@ -193,9 +193,24 @@ attn_status_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const
         cudaGetLastError();
         return setup;
     }
-    const dim3 grid(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_blocks));
-    kern<<<grid, attn::kPrefillThreads, smem, stream>>>(tq, tk, tv, args);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    // Programmatic stream serialisation, as for the decode: the kernel may be launched
+    // while the previous kernel of the stream finishes, and waits for it
+    // (griddepcontrol.wait) before touching global memory.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(planes), static_cast<unsigned>(args.n_q_blocks));
+    cfg.blockDim = dim3(attn::kPrefillThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, args) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
 }
 
 template <int D, bool BF16>

@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     constexpr int DRAIN = O_DONE + 2;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
 
+    // Launched with programmatic stream serialisation: wait for the previous kernel of the
+    // stream (its writes visible) before any global memory is touched.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -732,6 +735,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             m_ref = m_new;
         }
 
+        // This CTA's key tiles are done: once every CTA of the grid is this far, the next
+        // kernel of the stream may launch and take the places of CTAs that exit.
+        if (tile == 1 && t == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         if (ok && n_kv > 0) {
             const bool w = wait_phase(bar(O_DONE + tile), 0, abort_flag);
             ok = __all_sync(0xffffffffu, w);
