@@ -685,7 +685,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     float t0, t1, t2, t3;
                     f2unpack(fma2(f2pack(s[x], s[x + 1]), c2, nm2), t0, t1);
                     f2unpack(fma2(f2pack(s[x + 2], s[x + 3]), c2, nm2), t2, t3);
-                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    // an eighth of the exponentials (two of every sixteen) on the FMA pipe: the
+                    // e4m3 path has half the tensor time per exponential of the 16-bit one, so
+                    // the MUFU sets its pace; an eighth moved over balanced the two pipes best
+                    float p0, p1;
+                    if ((x / 4) % 4 == 3) {
+                        ex2_fma2(t0, t1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(t0);
+                        p1 = ex2_approx(t1);
+                    }
                     const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
                     rs2 = add2(rs2, add2(f2pack(p0, p1), f2pack(p2, p3)));
                     const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);

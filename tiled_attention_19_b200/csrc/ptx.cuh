@@ -318,4 +318,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x of two values at once on the FMA pipe, leaving the MUFU free. Cody-Waite range
+// reduction (Cody and Waite, "Software Manual for the Elementary Functions", 1980):
+// x = j + f with j = round(x) and f in [-1/2, 1/2]; j comes from adding 1.5 * 2^23,
+// which rounds x to an integer in the low mantissa bits. 2^f is a degree-4 polynomial
+// fitted to minimax relative error on [-1/2, 1/2] by a Remez exchange (relative error
+// 2.6e-6); 2^j is built directly in the exponent field. x is clamped to >= -127, where
+// that scale is exactly 0, so -inf (a masked score) gives exactly 0. Valid for x <= 127.
+__device__ __forceinline__ void ex2_fma2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kC0 = 0.9999992847442627f, kC1 = 0.6931217908859253f,
+                    kC2 = 0.240247443318367f, kC3 = 0.05591785907745361f,
+                    kC4 = 0.009570102207362652f;
+    const uint64_t x = f2pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t r = f2pack(kRound, kRound);
+    const uint64_t t = add2(x, r);          // 1.5 * 2^23 + j, exactly
+    const uint64_t f = sub2(x, sub2(t, r));  // x - j, exactly
+    uint64_t p = fma2(f2pack(kC4, kC4), f, f2pack(kC3, kC3));
+    p = fma2(p, f, f2pack(kC2, kC2));
+    p = fma2(p, f, f2pack(kC1, kC1));
+    p = fma2(p, f, f2pack(kC0, kC0));
+    float t0, t1;
+    f2unpack(t, t0, t1);
+    // the low bits of t hold j: (j + 127) << 23 is 2^j as a float (0 for j = -127)
+    const float s0 = __uint_as_float((__float_as_uint(t0) << 23) + 0x3F800000u);
+    const float s1 = __uint_as_float((__float_as_uint(t1) << 23) + 0x3F800000u);
+    f2unpack(mul2(p, f2pack(s0, s1)), y0, y1);
+}
+
 }  // namespace attn
