@@ -80,7 +80,14 @@ struct PrefillCfg {
     static constexpr int kPCols = kBN * kElem / 4;     // TMEM columns P takes
     static constexpr int kKStages = (kTileBytes == 16384) ? 5 : 3;
     static constexpr int kVStages = (kTileBytes == 16384) ? 5 : 2;
-    static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 384;
+    // At D = 64 the O accumulators take 64 columns each, which leaves room for a third
+    // S buffer (kSCol2). The split-KV form rotates S through all three (kTriS) while a
+    // warpgroup has at most kTriMaxTiles key tiles: S issued ahead shortens the start of
+    // short loops; in long ones the two-buffer order measured faster.
+    static constexpr int kSCol0 = 0, kSCol1 = 128, kSCol2 = 256;
+    static constexpr int kOCol0 = D == 64 ? 384 : 256, kOCol1 = D == 64 ? 448 : 384;
+    static constexpr bool kTriS = D == 64;
+    static constexpr int kTriMaxTiles = 4;
     static constexpr int kTmemCols = 512;
     // P is handed to the MMA warp in two parts: the first kPSplit keys, then the rest
     // (kPSplit is a multiple of kPVKeys, so each part is whole P.V instructions).
@@ -88,8 +95,9 @@ struct PrefillCfg {
     static constexpr bool kSplitP = D == 64;  // the MMA warp takes the first part early
     static_assert(kPSplit == 96 && kBN == 128, "P hand-off layout");
     // barriers: Q_FULL, K_FULL/K_EMPTY per K stage, V_FULL/V_EMPTY per V stage,
-    // S_FULL[2], P_FULL[2] (first part of P), P_REST[2] (the rest), O_DONE[2], DRAIN
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 9;
+    // S_FULL[3], P_FULL[2] (first part of P), P_REST[2] (the rest), O_READY[2],
+    // O_DONE[2], DRAIN
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 12;
     static constexpr int kTileRegion = kTileBytes * (2 + kKStages + kVStages);
     static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTileRegion + kNumBars * 8 + 16;
     static_assert(kSmemBytes <= 232448, "shared-memory budget");
@@ -174,10 +182,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     constexpr int K_EMPTY = K_FULL + NK;
     constexpr int V_FULL = K_EMPTY + NK;
     constexpr int V_EMPTY = V_FULL + NV;
-    constexpr int S_FULL = V_EMPTY + NV;  // [2]
-    constexpr int P_FULL = S_FULL + 2;    // [2] the first kPSplit keys of P are in TMEM
+    constexpr int S_FULL = V_EMPTY + NV;  // [3] per S buffer (the third only with kTriS)
+    constexpr int P_FULL = S_FULL + 3;    // [2] the first kPSplit keys of P are in TMEM
     constexpr int P_REST = P_FULL + 2;    // [2] the rest of P is in TMEM
-    constexpr int O_DONE = P_REST + 2;    // [2]
+    constexpr int O_READY = P_REST + 2;   // [2] a P.V into O_t completed (kTriS)
+    constexpr int O_DONE = O_READY + 2;   // [2]
     constexpr int DRAIN = O_DONE + 2;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
 
@@ -275,10 +284,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_init(bar(V_FULL + s), 1);
             mbar_init(bar(V_EMPTY + s), 1);
         }
+        for (int t = 0; t < 3; ++t) mbar_init(bar(S_FULL + t), 1);
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(S_FULL + t), 1);
             mbar_init(bar(P_FULL + t), kBM);
             mbar_init(bar(P_REST + t), kBM);
+            mbar_init(bar(O_READY + t), 1);
             mbar_init(bar(O_DONE + t), 1);
         }
         mbar_init(bar(DRAIN), 1);
@@ -472,7 +482,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // ring positions: K of the tile whose S is due, V of the tile whose P.V is due
             int sk = 0, sv = 0;
             uint32_t kpar = 0, vpar = 0;
-            if (split) {
+            if (split && Cfg::kTriS && ns0 <= Cfg::kTriMaxTiles) {
+                // Three S buffers (D = 64): ring sequence g (the alternating order below)
+                // is S product g, in buffer g % 3, for warpgroup owner(g). S(g + 3) is
+                // issued right after P.V(g), which frees its buffer (MMAs of one thread run
+                // in issue order), so each warpgroup finds its next S computed while its
+                // softmax ran. O_READY(t) signals each P.V into O_t: with S issued ahead,
+                // S completing no longer implies the warpgroup's previous P.V did.
+                auto owner = [&](int g) { return g < 2 * ns1 ? (g & 1) : 0; };
+                auto local = [&](int g) { return g < 2 * ns1 ? (g >> 1) : g - ns1; };
+                auto issue_s_seq = [&](int g) -> bool {
+                    const int skg = g % NK;
+                    if (!wait_phase(bar(K_FULL + skg), static_cast<uint32_t>(g / NK) & 1u, abort_flag))
+                        return false;
+                    tc_fence_after();
+                    const int buf = g % 3;
+                    issue_s(dq0, static_cast<uint32_t>(buf) * 128u, skg);
+                    mma_commit(bar(S_FULL + buf));
+                    mma_commit(bar(K_EMPTY + skg));
+                    return true;
+                };
+                for (int g = 0; ok && g < min(3, n_all); ++g) ok = issue_s_seq(g);
+                for (int g = 0; ok && g < n_all; ++g) {
+                    const int t = owner(g), m = local(g);
+                    const int svg = g % NV;
+                    ok = wait_phase(bar(V_FULL + svg), static_cast<uint32_t>(g / NV) & 1u, abort_flag) &&
+                         pv_parts(t, static_cast<uint32_t>(g % 3) * 128u,
+                                  t == 0 ? Cfg::kOCol0 : Cfg::kOCol1, svg, m == 0, m & 1);
+                    if (!ok) break;
+                    mma_commit(bar(O_READY + t));
+                    if (m == (t == 0 ? ns0 : ns1) - 1) mma_commit(bar(O_DONE + t));
+                    mma_commit(bar(V_EMPTY + svg));
+                    if (g + 3 < n_all) ok = issue_s_seq(g + 3);
+                }
+            } else if (split) {
                 // Both warpgroups work on Q0 (the only query tile), warpgroup t over its own
                 // key tiles, which sit at ring sequence seq(t, m) in the alternating order.
                 // Per step m: PV0 of its tile m-1, S0 of tile m, then the same for
@@ -599,7 +642,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int tb = tile == 0 ? b0 : b1;
         const int n_kv = tb > ta ? tb - ta : 0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const uint32_t s_col = tile == 0 ? Cfg::kSCol0 : Cfg::kSCol1;
+        const uint32_t s_col_t = tile == 0 ? Cfg::kSCol0 : Cfg::kSCol1;
         const uint32_t o_col = tile == 0 ? Cfg::kOCol0 : Cfg::kOCol1;
         const float c = args.scale_log2;
         int row_lo, row_hi;  // this row's visible keys [row_lo, row_hi)
@@ -612,9 +655,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         float l = 0.f;            // running sum of 2^(s*c - m_ref)
         bool ok = true;
 
+        const bool tri = Cfg::kTriS && split && ns0 <= Cfg::kTriMaxTiles;  // three S buffers
         for (int jj = 0; jj < n_kv; ++jj) {
             const int j = ta + jj;  // key tile
-            const bool w = wait_phase(bar(S_FULL + tile), jj & 1, abort_flag);
+            // S buffer and barrier phase of this tile: its own buffer, or with three
+            // buffers those of S product g (the ring sequence of the split order)
+            uint32_t s_col = s_col_t;
+            int s_bar = S_FULL + tile;
+            uint32_t s_par = jj & 1;
+            if (tri) {
+                const int g = tile == 0 ? jj + min(jj, ns1) : 2 * jj + 1;
+                s_col = static_cast<uint32_t>(g % 3) * 128u;
+                s_bar = S_FULL + g % 3;
+                s_par = static_cast<uint32_t>(g / 3) & 1u;
+            }
+            const bool w = wait_phase(bar(s_bar), s_par, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[kBN];
@@ -656,8 +711,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
             // Correct O when the reference max moved, before any part of this tile's P
             // is handed over. S_t(j) completing implies the P.V of tile j-1 (issued
-            // before it) has completed too.
+            // before it) has completed too; with three S buffers S runs ahead, so the
+            // P.V of tile j-1 is waited for here. (P.V of tile j-2 completed before this
+            // S was issued, so the barrier is at most one phase behind.)
             if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (tri) {
+                    if (!__all_sync(0xffffffffu,
+                                    wait_phase(bar(O_READY + tile), (jj - 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 32) {
                     uint32_t o[32];
