@@ -274,7 +274,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return n < 2 * ns1 ? ((n & 1) ? a1 : a0) + (n >> 1) : a0 + (n - ns1);
     };
 
-    if (threadIdx.x == 0) {
+    // The producer lane initialises the barriers and issues the query tile(s) at once,
+    // so their load overlaps the TMEM allocation and the start-up barrier; it only
+    // arrives there (the other warps wait for the barriers and the TMEM address).
+    if (warp == 8 && lane == 0) {
         mbar_init(bar(Q_FULL), 1);
         for (int s = 0; s < NK; ++s) {
             mbar_init(bar(K_FULL + s), 1);
@@ -294,20 +297,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        if (n_all > 0) {
+            mbar_arrive_expect_tx(bar(Q_FULL), (split ? 1 : 2) * Cfg::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < Cfg::kChunks; ++c) {
+                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow0,
+                            h, b);
+                if (!split)
+                    tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems,
+                                qrow1, h, b);
+            }
+        }
     }
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
+    if (warp == 8) {
+        __syncwarp();
+        named_barrier_arrive(2, kPrefillThreads);
+    } else {
+        tc_fence_before();
+        named_barrier_sync(2, kPrefillThreads);
+        tc_fence_after();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;  // (not read by the producer warp, which did not wait)
 
     int k_issued = 0, v_issued = 0;  // producer: tiles issued per ring (for the abort drain)
     bool mma_started = false;
@@ -318,15 +335,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ------------------------------------------------------------ producer
         regs_decrease<kOtherRegs>();
         if (lane == 0 && n_all > 0) {
-            mbar_arrive_expect_tx(bar(Q_FULL), (split ? 1 : 2) * Cfg::kTileBytes);
-#pragma unroll
-            for (int c = 0; c < Cfg::kChunks; ++c) {
-                tma_load_4d(sQ0 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems, qrow0,
-                            h, b);
-                if (!split)
-                    tma_load_4d(sQ1 + c * Cfg::kChunkBytes, &tm_q, bar(Q_FULL), c * Cfg::kChunkElems,
-                                qrow1, h, b);
-            }
+            // (the query tiles were issued before the start-up barrier)
             constexpr int kBlocks = kBN / kPageSize;  // cache blocks per key tile
             // Paged keys: a tile's rows come from kBlocks cache blocks; a block past the
             // sequence loads its first block instead (finite rows, masked), and an entry

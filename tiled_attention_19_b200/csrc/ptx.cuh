@@ -264,6 +264,11 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrives on named barrier `id` over `count` threads without waiting for it.
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Register reallocation between warpgroups (all warps of a warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void regs_increase() {
