@@ -190,9 +190,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     constexpr int DRAIN = O_DONE + 2;
     static_assert(DRAIN + 1 == Cfg::kNumBars, "barrier count");
 
-    // Launched with programmatic stream serialisation: wait for the previous kernel of the
-    // stream (its writes visible) before any global memory is touched.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -209,6 +206,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Set-up that touches no global memory runs before the wait for the previous kernel
+    // of the stream (programmatic stream serialisation): the producer lane initialises
+    // the barriers and warp 9 allocates TMEM while that kernel finishes.
+    if (warp == 8 && lane == 0) {
+        mbar_init(bar(Q_FULL), 1);
+        for (int s = 0; s < NK; ++s) {
+            mbar_init(bar(K_FULL + s), 1);
+            mbar_init(bar(K_EMPTY + s), 1);
+        }
+        for (int s = 0; s < NV; ++s) {
+            mbar_init(bar(V_FULL + s), 1);
+            mbar_init(bar(V_EMPTY + s), 1);
+        }
+        for (int t = 0; t < 3; ++t) mbar_init(bar(S_FULL + t), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(P_FULL + t), kBM);
+            mbar_init(bar(P_REST + t), kBM);
+            mbar_init(bar(O_READY + t), 1);
+            mbar_init(bar(O_DONE + t), 1);
+        }
+        mbar_init(bar(DRAIN), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    // Wait for the previous kernel of the stream (its writes visible) before any global
+    // memory is touched.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int bh = blockIdx.x;                           // b * Hq + h
     const int h = bh % args.Hq;
     const int b = bh / args.Hq;
@@ -274,32 +305,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return n < 2 * ns1 ? ((n & 1) ? a1 : a0) + (n >> 1) : a0 + (n - ns1);
     };
 
-    // The producer lane initialises the barriers and issues the query tile(s) at once,
-    // so their load overlaps the TMEM allocation and the start-up barrier; it only
-    // arrives there (the other warps wait for the barriers and the TMEM address).
+    // The producer lane issues the query tile(s) at once, so their load overlaps the
+    // start-up barrier, on which it only arrives (the other warps wait there for the
+    // barriers and the TMEM address).
     if (warp == 8 && lane == 0) {
-        mbar_init(bar(Q_FULL), 1);
-        for (int s = 0; s < NK; ++s) {
-            mbar_init(bar(K_FULL + s), 1);
-            mbar_init(bar(K_EMPTY + s), 1);
-        }
-        for (int s = 0; s < NV; ++s) {
-            mbar_init(bar(V_FULL + s), 1);
-            mbar_init(bar(V_EMPTY + s), 1);
-        }
-        for (int t = 0; t < 3; ++t) mbar_init(bar(S_FULL + t), 1);
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(P_FULL + t), kBM);
-            mbar_init(bar(P_REST + t), kBM);
-            mbar_init(bar(O_READY + t), 1);
-            mbar_init(bar(O_DONE + t), 1);
-        }
-        mbar_init(bar(DRAIN), 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
         if (n_all > 0) {
             mbar_arrive_expect_tx(bar(Q_FULL), (split ? 1 : 2) * Cfg::kTileBytes);
 #pragma unroll
@@ -311,10 +320,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                 qrow1, h, b);
             }
         }
-    }
-    if (warp == 9) {
-        tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
-        tmem_relinquish();
     }
     if (warp == 8) {
         __syncwarp();
