@@ -403,6 +403,20 @@ attn_status_t attn_get_device_status(void* stream);
  */
 attn_status_t attn_selftest_bounded_wait(void* stream);
 
+/*
+ * attn_selftest_fill_noalloc_scratch -- test hook for attn_fwd_paged_noalloc:
+ * overwrites every byte of its fixed 4 MiB scratch array on the current device with
+ * (byte_value & 0xFF), enqueued on `stream`. This stands in for what an interrupted
+ * call (one whose bounded wait expired) can leave behind: completion counters that
+ * are not zero and stale partial results. Tests use it to check that the next
+ * no-allocation call does not depend on what the array held. Like any call that
+ * touches the array, it races with no-allocation calls in flight on other streams.
+ * Returns ATTN_OK once enqueued, ATTN_ERR_DEVICE without an sm_100 device,
+ * ATTN_ERR_CUDA if the array's address cannot be looked up or the fill fails to
+ * enqueue.
+ */
+attn_status_t attn_selftest_fill_noalloc_scratch(int byte_value, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

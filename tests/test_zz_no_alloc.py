@@ -5,7 +5,9 @@ framework that owns the allocator) cannot provide the split-KV workspace that
 attn_fwd_paged takes. The no-allocation entry point uses a fixed 4 MiB scratch array
 inside the library instead. These tests call it through the C ABI and check that two
 calls in a row match the fp64 oracle and attn_fwd_paged with a caller workspace, within
-the parity tolerances, and that a problem too large for the fixed array is refused.
+the parity tolerances, that a call after the array was overwritten with junk (as an
+interrupted call can leave it) still matches the oracle, and that a problem too large
+for the fixed array is refused.
 
 This file is collected last on purpose; it must pass both on its own in a fresh
 process and after every other test.
@@ -67,6 +69,29 @@ def test_noalloc_matches_workspace_entry_point(name):
         assert torch.all(lse[~fin] == ref_lse[~fin])
         rel = ((lse[fin] - ref_lse[fin]).abs() / ref_lse[fin].abs().clamp_min(1.0)).max().item()
         assert rel <= LSE_REL, rel
+
+
+@pytest.mark.parametrize("fill", [0x07, 0xFF])
+def test_noalloc_does_not_depend_on_what_the_scratch_held(fill):
+    # An interrupted call can leave the completion counters non-zero and stale partials
+    # in the fixed array. Every byte is overwritten first (0x07070707 or -1 as counters):
+    # without the per-call counter clear no CTA would see its unit's count complete and
+    # no split sequence would be merged.
+    s = inputs.WORKLOADS["paged_decode_s16_hq12_hkv2_d128_bf16"]
+    xh = inputs.make(s)
+    x = {k: v.to(DEV) for k, v in xh.items()}
+    oro, orl = oracle.attn_paged(xh["q"], xh["k_cache"], xh["v_cache"], xh["block_table"],
+                                 xh["seq_lens"], s.scale)
+    lib = ta.load()
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):
+        assert lib.attn_selftest_fill_noalloc_scratch(fill, stream) == 0
+        out = torch.full((s.num_seqs, s.Hq, s.D), 7.0, dtype=s.dtype, device=DEV)
+        lse = torch.full((s.num_seqs, s.Hq), 7.0, device=DEV)
+        assert call_noalloc(x, s, out, lse) == 0
+        torch.cuda.synchronize()
+        assert ta.device_status() == 0
+        check_parity(out, lse, oro, orl, s.dtype, f"no-alloc after filling the scratch with {fill:#x}")
 
 
 def test_noalloc_refuses_problems_past_the_scratch_limit():

@@ -64,6 +64,7 @@ SIGNATURES = {
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_get_device_status": (_i, [_vp]),
     "attn_selftest_bounded_wait": (_i, [_vp]),
+    "attn_selftest_fill_noalloc_scratch": (_i, [_i, _vp]),
 }
 
 _lib = None

@@ -1088,6 +1088,19 @@ attn_status_t attn_fwd_paged_noalloc(const void* q, const void* k_cache, const v
     return paged_launch(c, scratch, stream);
 }
 
+attn_status_t attn_selftest_fill_noalloc_scratch(int byte_value, void* stream_) {
+    const attn_status_t dev = check_device();
+    if (dev != ATTN_OK) return dev;
+    void* scratch = static_scratch_address();
+    if (scratch == nullptr) return ATTN_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, byte_value & 0xFF, kStaticScratchBytes,
+                        static_cast<cudaStream_t>(stream_)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
 const char* attn_error_string(attn_status_t status) {
     switch (status) {
         case ATTN_OK: return "ok";
