@@ -502,7 +502,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 // issued right after P.V(g), which frees its buffer (MMAs of one thread run
                 // in issue order), so each warpgroup finds its next S computed while its
                 // softmax ran. O_READY(t) signals each P.V into O_t: with S issued ahead,
-                // S completing no longer implies the warpgroup's previous P.V did.
+                // S completing no longer implies the warpgroup's previous P.V did, so the
+                // softmax waits for it before an O correction and before announcing P
+                // (which keeps P_FULL(t) within one phase of this warp's wait on it).
                 auto owner = [&](int g) { return g < 2 * ns1 ? (g & 1) : 0; };
                 auto local = [&](int g) { return g < 2 * ns1 ? (g >> 1) : g - ns1; };
                 auto issue_s_seq = [&](int g) -> bool {
@@ -808,13 +810,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         tmem_st16(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[32]));
                         if constexpr (Cfg::kSplitP) {
                             tmem_wait_st();
+                            // With three S buffers this tile's S can be ready before the
+                            // MMA warp has taken the previous tile's P (it may still be
+                            // waiting for that tile's V). P is announced only once the
+                            // previous P.V has completed, so P_FULL never runs two phases
+                            // ahead of the MMA warp's wait on it.
+                            if (tri && jj > 0)
+                                ok = __all_sync(0xffffffffu, wait_phase(bar(O_READY + tile),
+                                                                        (jj - 1) & 1, abort_flag));
                             tc_fence_before();
-                            mbar_arrive(bar(P_FULL + tile));
+                            if (ok) mbar_arrive(bar(P_FULL + tile));
                         }
                     }
                 }
                 tmem_st16(lane_base + s_col + 48, *reinterpret_cast<uint32_t(*)[16]>(&pk[48]));
             }
+            if (!ok) break;  // a wait gave up (the abort flag is set)
             f2unpack(rs2, rs0, rs1);
             tmem_wait_st();
             tc_fence_before();
