@@ -206,10 +206,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Set-up that touches no global memory runs before the wait for the previous kernel
-    // of the stream (programmatic stream serialisation): the producer lane initialises
-    // the barriers and warp 9 allocates TMEM while that kernel finishes.
-    if (warp == 8 && lane == 0) {
+    // Barrier initialisation (by the producer lane, which then issues the first loads)
+    // and the TMEM allocation (warp 9). With kEarlySetup they run before the wait for the
+    // previous kernel of the stream (programmatic stream serialisation), while that
+    // kernel finishes; otherwise after the wait, where at D = 128 the registers come out
+    // without spills (ptxas spilled with the early form there, and the e4m3 kernel ran
+    // 6 % slower).
+    constexpr bool kEarlySetup = D == 64;
+    auto init_barriers = [&] {
         mbar_init(bar(Q_FULL), 1);
         for (int s = 0; s < NK; ++s) {
             mbar_init(bar(K_FULL + s), 1);
@@ -232,10 +236,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-    }
-    if (warp == 9) {
+    };
+    auto alloc_tmem = [&] {
         tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
         tmem_relinquish();
+    };
+    if constexpr (kEarlySetup) {
+        if (warp == 8 && lane == 0) init_barriers();
+        if (warp == 9) alloc_tmem();
     }
     // Wait for the previous kernel of the stream (its writes visible) before any global
     // memory is touched.
@@ -309,6 +317,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // start-up barrier, on which it only arrives (the other warps wait there for the
     // barriers and the TMEM address).
     if (warp == 8 && lane == 0) {
+        if constexpr (!kEarlySetup) init_barriers();
         if (n_all > 0) {
             mbar_arrive_expect_tx(bar(Q_FULL), (split ? 1 : 2) * Cfg::kTileBytes);
 #pragma unroll
@@ -320,6 +329,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                 qrow1, h, b);
             }
         }
+    }
+    if constexpr (!kEarlySetup) {
+        if (warp == 9) alloc_tmem();
     }
     if (warp == 8) {
         __syncwarp();
