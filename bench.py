@@ -56,13 +56,47 @@ KERNEL_SOURCES = {
 
 
 # ------------------------------------------------------------------------ helpers
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _find_number(d, key, depth=2):
+    """d[key] as a float, looked up at the top level or up to `depth` levels of nested
+    objects below it; None if absent or not a number."""
+    if isinstance(d, dict):
+        v = d.get(key)
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            return float(v)
+        if depth > 0:
+            for sub in d.values():
+                r = _find_number(sub, key, depth - 1)
+                if r is not None:
+                    return r
+    return None
+
+
+def load_peaks(path=None):
+    """The measured peaks (hbm_gbs, bf16_tflops, bf16_tflops_sustained) from
+    MEASURED_PEAKS.json; a key the file lacks (or a missing or unreadable file) takes the
+    fallback figure, and the returned label says which."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = None
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(PEAKS_FALLBACK), "fallback"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+        except (OSError, ValueError):
+            d = None
+    if d is None:
+        return dict(PEAKS_FALLBACK), "fallback"
+    peaks, missing = {}, []
+    for k, fb in PEAKS_FALLBACK.items():
+        v = _find_number(d, k)
+        if v is None:
+            missing.append(k)
+            v = fb
+        peaks[k] = v
+    if not missing:
+        return peaks, "measured"
+    if len(missing) == len(PEAKS_FALLBACK):
+        return peaks, "fallback"
+    return peaks, "measured (fallback for " + ", ".join(missing) + ")"
 
 
 def kernel_source_hash(kernel: str) -> str:

@@ -82,3 +82,23 @@ def test_decode_seqs_option_scales_the_decode_workload(monkeypatch, capsys):
     assert bench.DECODE.num_seqs == 4 and bench.DECODE.Hq == 12 and bench.DECODE.seed == 5
     with pytest.raises(SystemExit):
         bench.main(["--decode-seqs", "0"])
+
+
+def test_peaks_file_missing_keys_and_nesting(tmp_path):
+    # No file: every figure is the fallback.
+    peaks, src = bench.load_peaks(str(tmp_path / "absent.json"))
+    assert src == "fallback" and peaks == bench.PEAKS_FALLBACK
+    # Nested objects are searched; a key the file lacks takes its fallback, and the
+    # label names it.
+    p = tmp_path / "peaks.json"
+    p.write_text('{"hbm": {"hbm_gbs": 6530.0}, "gemm": {"bf16_tflops": 1626.0}}')
+    peaks, src = bench.load_peaks(str(p))
+    assert peaks["hbm_gbs"] == 6530.0 and peaks["bf16_tflops"] == 1626.0
+    assert peaks["bf16_tflops_sustained"] == bench.PEAKS_FALLBACK["bf16_tflops_sustained"]
+    assert src == "measured (fallback for bf16_tflops_sustained)"
+    p.write_text('{"hbm_gbs": 6530, "bf16_tflops": 1626, "bf16_tflops_sustained": 1402}')
+    peaks, src = bench.load_peaks(str(p))
+    assert src == "measured" and peaks["bf16_tflops_sustained"] == 1402.0
+    # An unreadable file is the fallback, not a crash.
+    p.write_text("{not json")
+    assert bench.load_peaks(str(p))[1] == "fallback"
