@@ -236,6 +236,26 @@ class ClockSampler:
                 "source": f"{self.source}; {how}"}
 
 
+DENSE_BF16_FLOP_PER_CLOCK_PER_SM = 8192  # 2.25 PFLOP/s dense at about 1.855 GHz on 148 SMs
+
+
+def clock_peak_fields(tflops, clock_record, device) -> dict:
+    """The nominal dense bf16 tensor rate at the SM clock actually seen in the timed
+    region (SMs x 8192 FLOP per clock x the median SM clock) and the fraction of it, so
+    that a power-capped or throttled run reads against the rate it ran at."""
+    mhz = (clock_record or {}).get("sm_mhz")
+    if not tflops or not mhz:
+        return {"clock_peak": None, "frac_of_clock_peak": None}
+    try:
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+    except (RuntimeError, AssertionError, AttributeError):
+        return {"clock_peak": None, "frac_of_clock_peak": None}
+    peak = sms * DENSE_BF16_FLOP_PER_CLOCK_PER_SM * float(mhz) * 1e6 / 1e12
+    return {"clock_peak": round(peak, 1), "frac_of_clock_peak": round(tflops / peak, 4),
+            "clock_peak_note": f"{sms} SMs x {DENSE_BF16_FLOP_PER_CLOCK_PER_SM} dense bf16 FLOP per "
+                               f"clock x the median SM clock in the timed region ({mhz:.0f} MHz)"}
+
+
 def tensor_peak(peaks: dict, region_ms: float):
     """The measured tensor peak that applies to a kernel timed over `region_ms`: the
     burst GEMM rate below one second of timed work, the sustained (power-capped) rate
@@ -498,6 +518,7 @@ def _run_ours(args, ws, rank, ta, device, clocks):
             "unit": "TFLOP/s",
             "frac": r2(per_gpu_tflops and per_gpu_tflops / pk_t, 4),
             "frac_of_sustained_peak": r2(per_gpu_tflops and per_gpu_tflops / peaks["bf16_tflops_sustained"], 4),
+            **clock_peak_fields(per_gpu_tflops, region_clocks, device),
             "traffic": None if args.window else profiled_traffic("prefill", PREFILL.name),
             "timed_region_ms": round(total_ms, 3),
             "avg_launch_ms": round(pre_avg, 5),
